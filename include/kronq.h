@@ -1,0 +1,241 @@
+/*
+ * kronq.h -- C ABI of libkronq.so, KronQ's per-layer quantization pass on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The pass (KronQ README intro; KronQ arXiv abstract):
+ *   1. accumulate the Kronecker factors of the layer Hessian H ~ H_X (x) H_G,
+ *      H_X = sum x x^T over calibration inputs, H_G = sum g g^T over output
+ *      gradients                                   -> kronq_accumulate_factors
+ *   2. the inter-layer sensitivity tr(H_G) * tr(H_X) -> kronq_sensitivity,
+ *      and the bit allocation it drives            -> kronq_allocate_bits*
+ *   3. bidirectional incoherence processing (BiIP): rescale + randomized
+ *      Hadamard rotation on the input and output side -> kronq_biip_forward,
+ *      and its inverse for unrotated export          -> kronq_biip_inverse
+ *   4. GPTQ-style blocked column quantization under the K-FAC loss with the
+ *      Cholesky factor of the damped inverse H_X, lazy-batch error feedback
+ *      and per-group scales at 2/3/4 bits           -> kronq_quantize_layer
+ *   5. packed int4/int2 storage (KronQ README "Model zoo") -> kronq_pack
+ *
+ * Conventions (all calls):
+ *   - Matrices are row-major.  W is m x n (out x in), X is T x n, G is T x m.
+ *   - Every array argument is DEVICE memory owned by the caller, except where
+ *     a comment says "host".  The library allocates no memory: scratch comes
+ *     from the caller's workspace (query its size with *_workspace_bytes).
+ *   - Calls are asynchronous on the given stream, except kronq_sensitivity
+ *     and kronq_device_status, which synchronise that stream.
+ *   - Arguments are checked on the host before anything is launched; a bad
+ *     argument returns KRONQ_ERR_INVALID_ARG (or KRONQ_ERR_UNSUPPORTED for a
+ *     valid but unimplemented combination) and touches no memory.
+ *   - A failure inside a kernel never traps: non-positive-definite factors
+ *     are reported through *info (LAPACK convention), and any bounded wait
+ *     that gives up records KRONQ_ERR_TIMEOUT in the library's device status
+ *     word (read it with kronq_device_status).
+ *   - kronq_last_error() returns a thread-local message for the last non-OK
+ *     status returned on the calling thread.
+ */
+#ifndef KRONQ_H
+#define KRONQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st* kronq_stream_t;
+
+typedef enum {
+  KRONQ_OK = 0,
+  KRONQ_ERR_INVALID_ARG = 1,
+  KRONQ_ERR_UNSUPPORTED = 2,
+  KRONQ_ERR_CUDA = 3,
+  KRONQ_ERR_NOT_PD = 4,
+  KRONQ_ERR_TIMEOUT = 5
+} kronq_status;
+
+typedef enum { KRONQ_BF16 = 0, KRONQ_F32 = 1 } kronq_dtype;
+
+/* BiIP ablation modes (KronQ README, "Mapping paper results to flags":
+ * --incoh_mode {full,no_rescale,su_only,sv_only}).  SU is the output-side
+ * (left, m) transform, SV the input-side (right, n) transform. */
+typedef enum {
+  KRONQ_BIIP_FULL = 0,       /* rescale + rotation on both sides          */
+  KRONQ_BIIP_NO_RESCALE = 1, /* rotation on both sides, no rescale        */
+  KRONQ_BIIP_SU_ONLY = 2,    /* output side only (U, D_out)               */
+  KRONQ_BIIP_SV_ONLY = 3     /* input side only (V, D_in)                 */
+} kronq_biip_mode;
+
+/* kronq_quant_params.flags */
+#define KRONQ_U_GIVEN      1u /* HX already holds U (upper): skip dead columns, damping, factorisation */
+#define KRONQ_ORDERED_FP32 2u /* fixed-order float32 trailing update (bit-exact test mode)             */
+#define KRONQ_WRITE_E      4u /* keep the scaled error E (m x n) in the E argument                      */
+
+/* Quantizer settings (KronQ README, "Reproduce from scratch":
+ * --w_bits --w_groupsize --w_asym).
+ *   bits     2, 3 or 4.
+ *   group    -1 (one group per row) or g > 0 with block % g == 0 or
+ *            g % block == 0; a ragged last group is allowed.
+ *   asym     1: asymmetric grid, zero = rint(-min/scale); 0: symmetric.
+ *   damp_rel damping lambda = damp_rel * mean(diag H~_X) (0.01 typical).
+ *   block    lazy-batch width; 128 is the only value implemented.
+ *   flags    KRONQ_* flags above. */
+typedef struct {
+  int bits;
+  int group;
+  int asym;
+  float damp_rel;
+  int block;
+  unsigned flags;
+} kronq_quant_params;
+
+/* ---------------------------------------------------------------------------
+ * Step 1 -- factor accumulation.  KronQ README intro (H ~ H_X (x) H_G);
+ * "WaterKron and FlipFlop Hessian", Table 1, "Marginal" row (A = E[x x^T],
+ * B = E[g g^T]); read here as sums over tokens, not means.
+ *
+ *   H (d x d, float32, row-major, full symmetric storage) += A^T A
+ *   A     T x d token rows, row stride lda elements (lda >= d), dtype dt.
+ *         KRONQ_BF16 runs on the tcgen05 tensor cores (bf16 x bf16 -> fp32);
+ *         it needs A 16-byte aligned and lda % 8 == 0.  KRONQ_F32 runs an
+ *         exact-fp32 SIMT kernel (small layers).
+ *   zero_first  nonzero: H is overwritten with A^T A instead of added to.
+ *   Call once per token chunk to stream T (pass zero_first only first).
+ *   Both triangles of H are kept equal.  T == 0 is allowed (no-op, or a
+ *   zero fill when zero_first).
+ * ------------------------------------------------------------------------- */
+kronq_status kronq_accumulate_factors(const void* A, kronq_dtype dt, int64_t T, int64_t d,
+                                      int64_t lda, float* H, int zero_first, kronq_stream_t s);
+
+/* ---------------------------------------------------------------------------
+ * Step 2 -- sensitivity.  KronQ abstract point (2); README bullet
+ * "Inter-layer mixed precision": s = tr(H_G) * tr(H_X).
+ *   HX n x n, HG m x m (device, float32).  out3 (HOST, 3 doubles) receives
+ *   { tr(H_X), tr(H_G), tr(H_G) * tr(H_X) }, diagonals summed in float64.
+ *   workspace: >= 16 bytes of device memory, 8-byte aligned.
+ *   Synchronises the stream.
+ * ------------------------------------------------------------------------- */
+kronq_status kronq_sensitivity(const float* HX, int64_t n, const float* HG, int64_t m,
+                               double* out3, void* workspace, size_t ws_bytes, kronq_stream_t s);
+
+/* Bit allocation over L sublayers (host only; KronQ README "Mapping paper
+ * results to flags", --inter_layer_mp).  Budget mode: start at bmin bits,
+ * repeatedly give +1 bit to the sublayer with the largest
+ * s_i (4^-b_i - 4^-(b_i+1)) / size_i among those whose upgrade keeps
+ * sum b_i size_i <= avg_bits * sum size_i and b_i < bmax; ties to the lower
+ * index.  sens, sizes, bits_out are HOST arrays of length L. */
+kronq_status kronq_allocate_bits(const double* sens, const int64_t* sizes, int L, double avg_bits,
+                                 int bmin, int bmax, int* bits_out);
+
+/* Type-level rule (--inter_layer_mp N): the N sublayer types with the
+ * largest summed sensitivity get base_bits + 1, the rest base_bits.
+ * type_ids[i] in [0, n_types) names sublayer i's type; ties to the lower
+ * type id.  HOST arrays of length L. */
+kronq_status kronq_allocate_topn_types(const double* sens, const int* type_ids, int L, int n_types,
+                                       int base_bits, int N, int* bits_out);
+
+/* ---------------------------------------------------------------------------
+ * Step 3 -- BiIP.  KronQ abstract point (1); README bullet "Bidirectional
+ * incoherence processing"; flags --incoh_rotate --incoh_kernel had
+ * --incoh_mode --alpha; the incoherence follows QuIP# (README
+ * "Acknowledgements").  Reading fixed by this library:
+ *   d_in[j]  = (H_X[j,j] / ||W[:,j]||^2)^alpha, d_out[i] = (H_G[i,i] / ||W[i,:]||^2)^alpha,
+ *   degenerate (zero) entries 1, each vector scaled to geometric mean 1;
+ *   V = (Had_{2^k}/sqrt(2^k) (x) DCT-II_K) diag(s_in) for n = 2^k K, K odd
+ *   (K <= 255); U likewise for m with s_out; signs from SplitMix64:
+ *   s_side[i] = 1 - 2 * bit63(mix64(2*seed + side + (i+1) * 0x9E3779B97F4A7C15)),
+ *   side 0 = input, 1 = output.
+ *   W~ = U D_out W D_in V^T,  H~_X = V D_in^-1 H_X D_in^-1 V^T,
+ *   H~_G = U D_out^-1 H_G D_out^-1 U^T.
+ *
+ * kronq_biip_forward
+ *   W   m x n, dtype wdt (bf16 or f32), read only.
+ *   Wt  m x n float32 out (may not alias W).
+ *   HX  n x n float32, transformed in place.
+ *   HG  m x m float32, transformed in place; may be NULL in modes
+ *       NO_RESCALE and SV_ONLY (then it is left alone).
+ *   alpha   rescale exponent (0.25 weight-only).
+ *   d_in (n), d_out (m)  float32 out: the rescale vectors (1 where unused).
+ *   workspace  >= kronq_biip_workspace_bytes(m, n) bytes, 256-byte aligned.
+ * kronq_biip_inverse
+ *   W (m x n float32) in place: W <- D_out^-1 U^T W V D_in^-1.
+ * ------------------------------------------------------------------------- */
+size_t kronq_biip_workspace_bytes(int64_t m, int64_t n);
+
+kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64_t m, int64_t n,
+                                float* HX, float* HG, uint64_t seed, float alpha,
+                                kronq_biip_mode mode, float* d_in, float* d_out,
+                                void* workspace, size_t ws_bytes, kronq_stream_t s);
+
+kronq_status kronq_biip_inverse(float* W, int64_t m, int64_t n, uint64_t seed,
+                                kronq_biip_mode mode, const float* d_in, const float* d_out,
+                                void* workspace, size_t ws_bytes, kronq_stream_t s);
+
+/* ---------------------------------------------------------------------------
+ * Step 4 -- quantization.  KronQ README intro ("extends GPTQ/GPTAQ");
+ * "Reproduce from scratch" flags.  Readings fixed by this library:
+ *   dead columns (diag 0): H_jj := 1, W[:, j] := 0; lambda = damp_rel *
+ *   mean diag; U upper with U^T U = (H~_X + lambda I)^-1, computed as the
+ *   upper "reverse" Cholesky factor R of H~_X + lambda I = R R^T followed by
+ *   U = R^-1.  For every column j in order: at a group start, per-row grid
+ *   from the current values of the group's columns (x_min = min(0, min w),
+ *   x_max = max(0, max w), equal -> (-1, 1); scale = (x_max - x_min) /
+ *   (2^b - 1), zero = rint(-x_min / scale)); q = clamp(rint(w / scale) +
+ *   zero, 0, 2^b - 1) (round half to even); e = (w - scale (q - zero)) /
+ *   U_jj; later columns -= e U[j, later], batched per `block` columns.
+ *
+ *   Wt     m x n float32: in W~, out the dequantised W~_q.
+ *   HX     n x n float32: in H~_X (or U with KRONQ_U_GIVEN), out U (upper
+ *          triangle; the strict lower triangle is scratch on return).
+ *   codes  m x n uint8 out, values 0 .. 2^bits - 1.
+ *   scales, zeros  m x ngroups float32 out, ngroups = 1 if group == -1 else
+ *          ceil(n / group); zeros are integer valued.
+ *   E      m x n float32 out (scaled errors) with KRONQ_WRITE_E, else NULL.
+ *   info   one int (device) out: 0, or 1 + the largest index j for which the
+ *          trailing submatrix (H~_X + lambda I)[j:, j:] was found not
+ *          positive definite (codes etc. are then unspecified).
+ *   workspace >= kronq_quantize_workspace_bytes(m, n, p), 256-byte aligned.
+ * ------------------------------------------------------------------------- */
+size_t kronq_quantize_workspace_bytes(int64_t m, int64_t n, const kronq_quant_params* p);
+
+kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
+                                  const kronq_quant_params* p, uint8_t* codes, float* scales,
+                                  float* zeros, float* E, int* info, void* workspace,
+                                  size_t ws_bytes, kronq_stream_t s);
+
+/* ---------------------------------------------------------------------------
+ * Step 5 -- packing.  KronQ README "Model zoo": W4/W2 as packed int4/int2,
+ * W3 not bit-packable (bits == 3 -> KRONQ_ERR_INVALID_ARG).  Layout: per
+ * row, along n, codes fill uint32 words from the least significant bit up
+ * (8 per word at 4 bits, 16 at 2 bits); words per row = ceil(n*bits/32),
+ * a ragged last word zero-padded.  codes m x n uint8; words m x wpr uint32.
+ * ------------------------------------------------------------------------- */
+kronq_status kronq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* out,
+                        kronq_stream_t s);
+kronq_status kronq_unpack(const uint32_t* in, int64_t m, int64_t n, int bits, uint8_t* codes,
+                          kronq_stream_t s);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics (no counterpart on the pages).
+ * kronq_device_status: synchronises the stream, returns in *out (host) the
+ *   library's device status word (KRONQ_OK or KRONQ_ERR_TIMEOUT) and clears it.
+ * kronq_kfac_loss: out (HOST double) = sum_j e_j^T HG e_j for the columns e_j
+ *   of E (m x n), HG m x m -- the K-FAC loss of the sweep,
+ *   tr(dW (H~_X + lambda I) dW^T H~_G), because dW = E U.  Workspace of
+ *   kronq_kfac_loss_workspace_bytes(m, n) bytes, 256-byte aligned.
+ *   Synchronises the stream.
+ * ------------------------------------------------------------------------- */
+kronq_status kronq_device_status(int* out, kronq_stream_t s);
+size_t kronq_kfac_loss_workspace_bytes(int64_t m, int64_t n);
+kronq_status kronq_kfac_loss(const float* E, const float* HG, int64_t m, int64_t n, double* out,
+                             void* workspace, size_t ws_bytes, kronq_stream_t s);
+
+const char* kronq_last_error(void);
+const char* kronq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KRONQ_H */

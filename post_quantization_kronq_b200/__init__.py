@@ -1,0 +1,156 @@
+"""KronQ per-layer quantization pass on NVIDIA B200 (sm_100a).
+
+Python binding of libkronq.so: one wrapper per C entry point, same names,
+argument marshalling only (torch tensors -> device pointers, the current CUDA
+stream).  Every step of the pass runs in the library's CUDA kernels; PyTorch
+supplies device memory and streams.  See ``include/kronq.h`` for the
+contract of each call.
+"""
+from __future__ import annotations
+
+import ctypes
+
+from ._lib import (BF16, BIIP_MODES, F32, ORDERED_FP32, U_GIVEN, WRITE_E, KronqError,
+                   QuantParams, check, lib)
+
+__all__ = [
+    "KronqError", "QuantParams", "U_GIVEN", "ORDERED_FP32", "WRITE_E",
+    "kronq_accumulate_factors", "kronq_sensitivity", "kronq_allocate_bits",
+    "kronq_allocate_topn_types", "kronq_biip_workspace_bytes", "kronq_biip_forward",
+    "kronq_biip_inverse", "kronq_quantize_workspace_bytes", "kronq_quantize_layer",
+    "kronq_pack", "kronq_unpack", "kronq_device_status", "kronq_kfac_loss_workspace_bytes",
+    "kronq_kfac_loss", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
+]
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def workspace(nbytes: int, device="cuda"):
+    """A device byte buffer for the calls that take a workspace (256-byte aligned)."""
+    import torch
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def words_per_row(n: int, bits: int) -> int:
+    return (n * bits + 31) // 32
+
+
+def kronq_version() -> str:
+    return lib.kronq_version().decode()
+
+
+def kronq_last_error() -> str:
+    return lib.kronq_last_error().decode(errors="replace")
+
+
+def kronq_accumulate_factors(A, H, zero_first: bool = False, lda: int | None = None, stream=None):
+    """H (d x d float32) += A^T A for A (T x d, bf16 or float32, row stride lda)."""
+    T, d = A.shape
+    lda = A.stride(0) if lda is None else lda
+    check(lib.kronq_accumulate_factors(_ptr(A), _dtype_code(A), T, d, lda, _ptr(H),
+                                       1 if zero_first else 0, _stream(stream)))
+
+
+def kronq_sensitivity(HX, HG, ws=None, stream=None):
+    """(tr(H_X), tr(H_G), tr(H_G) * tr(H_X)) as Python floats (synchronises)."""
+    out = (ctypes.c_double * 3)()
+    ws = workspace(256, HX.device) if ws is None else ws
+    check(lib.kronq_sensitivity(_ptr(HX), HX.shape[0], _ptr(HG), HG.shape[0], out, _ptr(ws),
+                                ws.numel(), _stream(stream)))
+    return out[0], out[1], out[2]
+
+
+def kronq_allocate_bits(sens, sizes, avg_bits: float = 2.5, bmin: int = 2, bmax: int = 4):
+    L = len(sens)
+    s = (ctypes.c_double * L)(*[float(v) for v in sens])
+    z = (ctypes.c_int64 * L)(*[int(v) for v in sizes])
+    out = (ctypes.c_int * L)()
+    check(lib.kronq_allocate_bits(s, z, L, float(avg_bits), bmin, bmax, out))
+    return list(out)
+
+
+def kronq_allocate_topn_types(sens, type_ids, n_types: int, base_bits: int, N: int):
+    L = len(sens)
+    s = (ctypes.c_double * L)(*[float(v) for v in sens])
+    t = (ctypes.c_int * L)(*[int(v) for v in type_ids])
+    out = (ctypes.c_int * L)()
+    check(lib.kronq_allocate_topn_types(s, t, L, n_types, base_bits, N, out))
+    return list(out)
+
+
+def kronq_biip_workspace_bytes(m: int, n: int) -> int:
+    return int(lib.kronq_biip_workspace_bytes(m, n))
+
+
+def kronq_biip_forward(W, Wt, HX, HG, seed: int, alpha: float, mode: str, d_in, d_out, ws=None,
+                       stream=None):
+    m, n = W.shape
+    ws = workspace(kronq_biip_workspace_bytes(m, n), W.device) if ws is None else ws
+    check(lib.kronq_biip_forward(_ptr(W), _dtype_code(W), _ptr(Wt), m, n, _ptr(HX), _ptr(HG),
+                                 int(seed), float(alpha), BIIP_MODES[mode], _ptr(d_in), _ptr(d_out),
+                                 _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def kronq_biip_inverse(W, seed: int, mode: str, d_in, d_out, ws=None, stream=None):
+    m, n = W.shape
+    ws = workspace(kronq_biip_workspace_bytes(m, n), W.device) if ws is None else ws
+    check(lib.kronq_biip_inverse(_ptr(W), m, n, int(seed), BIIP_MODES[mode], _ptr(d_in),
+                                 _ptr(d_out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def kronq_quantize_workspace_bytes(m: int, n: int, params: QuantParams) -> int:
+    return int(lib.kronq_quantize_workspace_bytes(m, n, ctypes.byref(params)))
+
+
+def kronq_quantize_layer(Wt, HX, params: QuantParams, codes, scales, zeros, info, E=None, ws=None,
+                         stream=None):
+    m, n = Wt.shape
+    ws = workspace(kronq_quantize_workspace_bytes(m, n, params), Wt.device) if ws is None else ws
+    check(lib.kronq_quantize_layer(_ptr(Wt), _ptr(HX), m, n, ctypes.byref(params), _ptr(codes),
+                                   _ptr(scales), _ptr(zeros), _ptr(E), _ptr(info), _ptr(ws),
+                                   ws.numel(), _stream(stream)))
+
+
+def kronq_pack(codes, bits: int, out, stream=None):
+    m, n = codes.shape
+    check(lib.kronq_pack(_ptr(codes), m, n, bits, _ptr(out), _stream(stream)))
+
+
+def kronq_unpack(words, m: int, n: int, bits: int, codes, stream=None):
+    check(lib.kronq_unpack(_ptr(words), m, n, bits, _ptr(codes), _stream(stream)))
+
+
+def kronq_device_status(stream=None) -> int:
+    v = ctypes.c_int(0)
+    check(lib.kronq_device_status(ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
+def kronq_kfac_loss_workspace_bytes(m: int, n: int) -> int:
+    return int(lib.kronq_kfac_loss_workspace_bytes(m, n))
+
+
+def kronq_kfac_loss(E, HG, ws=None, stream=None) -> float:
+    m, n = E.shape
+    ws = workspace(kronq_kfac_loss_workspace_bytes(m, n), E.device) if ws is None else ws
+    out = ctypes.c_double(0.0)
+    check(lib.kronq_kfac_loss(_ptr(E), _ptr(HG), m, n, ctypes.byref(out), _ptr(ws), ws.numel(),
+                              _stream(stream)))
+    return out.value

@@ -1,0 +1,318 @@
+// Bidirectional incoherence processing (BiIP) kernels.
+//
+// KronQ abstract point (1) and README bullet "Bidirectional incoherence
+// processing (BiIP)": rotation + rescale on the input and the output side;
+// README flags --incoh_kernel had --alpha.  The rotation of a length
+// L = P K vector (P = 2^k, K odd) is (Had_P / sqrt(P) (x) C_K) diag(s): view
+// the vector as a P x K matrix Y (index a K + b), apply the orthonormal
+// DCT-II C_K along b and the Walsh-Hadamard transform along a.  Signs come
+// from SplitMix64 (no table).
+//
+// One CTA holds R whole rows in shared memory, applies the DCT (K > 1) and
+// the FWHT in radix-16 register passes, and stores the result transposed
+// (R consecutive floats per output row), so two launches make the two-sided
+// transform U M V^T at two HBM round trips.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kq {
+namespace {
+
+constexpr int RP_THREADS = 256;
+constexpr int KREG = 16;     // odd factors up to this size are transformed in registers
+constexpr int KMAX = 255;    // largest odd factor supported
+
+__device__ __forceinline__ int64_t padx(int64_t x) { return x + (x >> 5); }
+
+__device__ __forceinline__ float sign_of(uint64_t state, int64_t j) {
+  return (splitmix64(state, (uint64_t)j) >> 63) ? -1.f : 1.f;
+}
+
+struct RPArgs {
+  RowPass p;
+  int R;        // rows per CTA
+  int P, K, logP;
+  int64_t RS;   // padded row stride in shared memory (floats)
+  float norm;   // 1 / sqrt(P)
+  int two_buf;  // K > KREG: DCT writes to a second buffer
+};
+
+__global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
+  extern __shared__ __align__(16) float sm[];
+  const RowPass& p = A.p;
+  const int R = A.R, P = A.P, K = A.K;
+  const int64_t L = p.L, RS = A.RS;
+  float* buf0 = sm;
+  float* buf1 = sm + (int64_t)R * RS;
+  float* Cm = sm + (int64_t)R * RS * (A.two_buf ? 2 : 1);
+  const int64_t r0 = (int64_t)blockIdx.x * R;
+  const int tid = threadIdx.x;
+
+  if (p.rotate && K > 1) {
+    for (int t = tid; t < K * K; t += RP_THREADS) {
+      const int i = t / K, j = t % K;
+      const double ci = (i == 0) ? sqrt(0.5) : 1.0;
+      Cm[t] = (float)(sqrt(2.0 / K) * ci * cospi((double)((2 * j + 1) * i) / (2.0 * K)));
+    }
+  }
+
+  // 1. load (+ forward pre-scale and signs)
+  const int64_t tot = (int64_t)R * L;
+  for (int64_t t = tid; t < tot; t += RP_THREADS) {
+    const int rr = (int)(t / L);
+    const int64_t j = t - (int64_t)rr * L;
+    const int64_t r = r0 + rr;
+    float v = 0.f;
+    if (r < p.rows) {
+      if (p.in_bf16)
+        v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[r * p.ld_in + j]);
+      else
+        v = reinterpret_cast<const float*>(p.in)[r * p.ld_in + j];
+      if (!p.inverse) {
+        if (p.scale_mode == 1) v = v * p.scale[j];
+        else if (p.scale_mode == 2) v = v / p.scale[j];
+        if (p.rotate) v = v * sign_of(p.sign_state, j);
+      }
+    }
+    buf0[rr * RS + padx(j)] = v;
+  }
+  __syncthreads();
+
+  float* cur = buf0;
+  if (p.rotate) {
+    // 2. DCT along b (odd factor)
+    if (K > 1) {
+      const int64_t items = (int64_t)R * P;
+      for (int64_t t = tid; t < items; t += RP_THREADS) {
+        const int rr = (int)(t / P);
+        const int a = (int)(t - (int64_t)rr * P);
+        float* row = buf0 + rr * RS;
+        const int64_t base = (int64_t)a * K;
+        if (!A.two_buf) {
+          float y[KREG];
+#pragma unroll
+          for (int b = 0; b < KREG; ++b) y[b] = (b < K) ? row[padx(base + b)] : 0.f;
+#pragma unroll
+          for (int o = 0; o < KREG; ++o) {
+            if (o < K) {
+              float acc = 0.f;
+#pragma unroll
+              for (int b = 0; b < KREG; ++b)
+                if (b < K) acc = fmaf(p.inverse ? Cm[b * K + o] : Cm[o * K + b], y[b], acc);
+              row[padx(base + o)] = acc;
+            }
+          }
+        } else {
+          float* orow = buf1 + rr * RS;
+          for (int o = 0; o < K; ++o) {
+            float acc = 0.f;
+            for (int b = 0; b < K; ++b)
+              acc = fmaf(p.inverse ? Cm[b * K + o] : Cm[o * K + b], row[padx(base + b)], acc);
+            orow[padx(base + o)] = acc;
+          }
+        }
+      }
+      if (A.two_buf) cur = buf1;
+      __syncthreads();
+    }
+    // 3. FWHT along a, radix-16 passes over bit groups of a
+    for (int lo = 0; lo < A.logP; lo += 4) {
+      const int nb = (A.logP - lo) < 4 ? (A.logP - lo) : 4;
+      const int G = 1 << nb;
+      const int64_t per_row = L >> nb;  // items per row
+      const int64_t items = (int64_t)R * per_row;
+      const int64_t lo_span = (int64_t)1 << lo;
+      for (int64_t t = tid; t < items; t += RP_THREADS) {
+        const int rr = (int)(t / per_row);
+        int64_t rem = t - (int64_t)rr * per_row;
+        const int b = (int)(rem % K);
+        rem /= K;
+        const int64_t a_lo = rem & (lo_span - 1);
+        const int64_t a_hi = rem >> lo;
+        const int64_t a0 = (a_hi << (lo + nb)) | a_lo;
+        float* row = cur + rr * RS;
+        float x[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (u < G) x[u] = row[padx((a0 + ((int64_t)u << lo)) * K + b)];
+#pragma unroll
+        for (int h = 1; h < 16; h <<= 1) {
+          if (h < G) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              if (u < G && (u & h) == 0) {
+                const float s0 = x[u], s1 = x[u | h];
+                x[u] = s0 + s1;
+                x[u | h] = s0 - s1;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (u < G) row[padx((a0 + ((int64_t)u << lo)) * K + b)] = x[u];
+      }
+      __syncthreads();
+    }
+  }
+
+  // 4. transposed store (+ normalisation, inverse post-scale and signs)
+  for (int64_t t = tid; t < tot; t += RP_THREADS) {
+    const int rr = (int)(t % R);
+    const int64_t j = t / R;
+    const int64_t r = r0 + rr;
+    if (r >= p.rows) continue;
+    float v = cur[rr * RS + padx(j)];
+    if (p.rotate) v = v * A.norm;
+    if (p.inverse) {
+      if (p.rotate) v = v * sign_of(p.sign_state, j);
+      if (p.scale_mode == 1) v = v * p.scale[j];
+      else if (p.scale_mode == 2) v = v / p.scale[j];
+    }
+    p.out[j * p.ld_out + r] = v;
+  }
+}
+
+// ------------------------------------------------------------ norms
+template <typename T>
+__device__ __forceinline__ float ld_val(const void* W, int64_t idx) {
+  if constexpr (sizeof(T) == 2)
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[idx]);
+  else
+    return reinterpret_cast<const float*>(W)[idx];
+}
+
+template <typename T>
+__global__ void rownorm_kernel(const void* W, int64_t m, int64_t n, float* rowsq) {
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (r >= m) return;
+  double acc = 0.0;
+  for (int64_t j = lane; j < n; j += 32) {
+    const double v = ld_val<T>(W, r * n + j);
+    acc += v * v;
+  }
+  acc = warp_sum_d(acc);
+  if (lane == 0) rowsq[r] = (float)acc;
+}
+
+constexpr int COL_CHUNK = 256;
+
+template <typename T>
+__global__ void colnorm_partial_kernel(const void* W, int64_t m, int64_t n, double* partial) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t i0 = (int64_t)blockIdx.y * COL_CHUNK;
+  if (j >= n) return;
+  double acc = 0.0;
+  const int64_t i1 = (i0 + COL_CHUNK < m) ? i0 + COL_CHUNK : m;
+  for (int64_t i = i0; i < i1; ++i) {
+    const double v = ld_val<T>(W, i * n + j);
+    acc += v * v;
+  }
+  partial[(int64_t)blockIdx.y * n + j] = acc;
+}
+
+__global__ void colnorm_final_kernel(const double* partial, int64_t chunks, int64_t n, float* colsq) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  double acc = 0.0;
+  for (int64_t c = 0; c < chunks; ++c) acc += partial[c * n + j];
+  colsq[j] = (float)acc;
+}
+
+__global__ void __launch_bounds__(1024) rescale_kernel(const float* H, int64_t ldh, const float* nrm,
+                                                       int64_t len, float alpha, float* d) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int64_t j = threadIdx.x; j < len; j += blockDim.x) {
+    const double h = H[j * ldh + j], w = nrm[j];
+    const double raw = (h > 0.0 && w > 0.0) ? pow(h / w, (double)alpha) : 1.0;
+    acc += log(raw);
+  }
+  acc = warp_sum_d(acc);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double v = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0;
+    v = warp_sum_d(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const double inv_gm = exp(-red[0] / (double)len);
+  for (int64_t j = threadIdx.x; j < len; j += blockDim.x) {
+    const double h = H[j * ldh + j], w = nrm[j];
+    const double raw = (h > 0.0 && w > 0.0) ? pow(h / w, (double)alpha) : 1.0;
+    d[j] = (float)(raw * inv_gm);
+  }
+}
+
+}  // namespace
+
+kronq_status rowpass(const RowPass& p, cudaStream_t s) {
+  if (p.rows <= 0 || p.L <= 0) return KRONQ_OK;
+  RPArgs A;
+  A.p = p;
+  int P = 1;
+  while (p.L % (2 * (int64_t)P) == 0) P *= 2;
+  const int64_t K = p.L / P;
+  if (p.rotate && K > KMAX)
+    return fail(KRONQ_ERR_UNSUPPORTED, "BiIP rotation: odd factor of the length exceeds 255");
+  A.P = P;
+  A.K = (int)K;
+  A.logP = 0;
+  while ((1 << A.logP) < P) ++A.logP;
+  A.norm = (float)(1.0 / sqrt((double)P));
+  A.two_buf = (p.rotate && K > KREG) ? 1 : 0;
+  const int64_t base = p.L + (p.L >> 5);
+  A.RS = base | 1;
+  const int64_t bytes_per_row = A.RS * 4 * (A.two_buf ? 2 : 1);
+  const int64_t cbytes = (p.rotate && K > 1) ? K * K * 4 : 0;
+  const int64_t budget = 200 * 1024;
+  int64_t R = (budget - cbytes) / bytes_per_row;
+  if (R > 8) R = 8;
+  if (R < 1) return fail(KRONQ_ERR_UNSUPPORTED, "BiIP rotation: row does not fit in shared memory");
+  A.R = (int)R;
+  const int64_t smem = R * bytes_per_row + cbytes;
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(&rowpass_kernel), (int)smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rowpass)");
+  const int64_t grid = ceil_div(p.rows, R);
+  rowpass_kernel<<<(unsigned)grid, RP_THREADS, (size_t)smem, s>>>(A);
+  KQ_LAUNCH_CHECK("rowpass_kernel");
+  return KRONQ_OK;
+}
+
+size_t wnorms_partial_floats(int64_t m, int64_t n) {
+  return (size_t)(ceil_div(m, COL_CHUNK) * n * 2);  // doubles, counted in floats
+}
+
+kronq_status wnorms(const void* W, bool bf16, int64_t m, int64_t n, float* colsq, float* rowsq,
+                    float* partial, cudaStream_t s) {
+  double* part = reinterpret_cast<double*>(partial);
+  const int64_t chunks = ceil_div(m, COL_CHUNK);
+  if (rowsq) {
+    const int64_t grid = ceil_div(m, 8);
+    if (bf16) rownorm_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, s>>>(W, m, n, rowsq);
+    else rownorm_kernel<float><<<(unsigned)grid, 256, 0, s>>>(W, m, n, rowsq);
+    KQ_LAUNCH_CHECK("rownorm_kernel");
+  }
+  if (colsq) {
+    dim3 g1((unsigned)ceil_div(n, 256), (unsigned)chunks);
+    if (bf16) colnorm_partial_kernel<__nv_bfloat16><<<g1, 256, 0, s>>>(W, m, n, part);
+    else colnorm_partial_kernel<float><<<g1, 256, 0, s>>>(W, m, n, part);
+    KQ_LAUNCH_CHECK("colnorm_partial_kernel");
+    colnorm_final_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(part, chunks, n, colsq);
+    KQ_LAUNCH_CHECK("colnorm_final_kernel");
+  }
+  return KRONQ_OK;
+}
+
+kronq_status rescale_vector(const float* H, int64_t ldh, const float* nrm, int64_t len, float alpha,
+                            float* d, cudaStream_t s) {
+  rescale_kernel<<<1, 1024, 0, s>>>(H, ldh, nrm, len, alpha, d);
+  KQ_LAUNCH_CHECK("rescale_kernel");
+  return KRONQ_OK;
+}
+
+}  // namespace kq

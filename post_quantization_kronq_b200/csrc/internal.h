@@ -1,0 +1,112 @@
+// Internal launchers of libkronq (C++ linkage, not exported).  Every
+// launcher assumes its arguments were validated by the C ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kronq.h"
+
+namespace kq {
+
+// ------------------------------------------------------------ SIMT GEMM
+// C = beta * C + alpha * op(A) op(B), float32, one launch, optional batch.
+//   op(A)(i,k) = transA ? A[k*lda + i] : A[i*lda + k]          (M x K)
+//   op(B)(k,j) = transB ? B[j*ldb + k] : B[k*ldb + j]          (K x N)
+//   a_upper: op(A)(i,k) is taken as 0 for k < i; b_upper: op(B)(k,j) = 0 for k > j
+//   c_mode : 0 all entries, 1 only i <= j, 2 i <= j plus the mirror C[j][i] = C[i][j]
+//   ordered: every product and sum rounded separately in ascending k and the
+//            result applied as C = C - acc (alpha must be -1, beta 1)
+//   beta == 0 never reads C.  If info != nullptr and *info != 0, no-op.
+struct GemmDesc {
+  int64_t M = 0, N = 0, K = 0;
+  const float* A = nullptr;
+  int64_t lda = 0;
+  bool transA = false;
+  const float* B = nullptr;
+  int64_t ldb = 0;
+  bool transB = false;
+  float* C = nullptr;
+  int64_t ldc = 0;
+  float alpha = 1.f, beta = 0.f;
+  bool a_upper = false, b_upper = false;
+  int c_mode = 0;
+  bool ordered = false;
+  int batch = 1;
+  int64_t strideA = 0, strideB = 0, strideC = 0;
+  const int* info = nullptr;
+};
+cudaError_t gemm_f32(const GemmDesc& g, cudaStream_t s);
+
+// ------------------------------------------------------------ factors
+kronq_status syrk_bf16_tc(const void* A, int64_t T, int64_t d, int64_t lda, float* H,
+                          bool zero_first, cudaStream_t s);
+cudaError_t status_fetch_syrk(int* out, cudaStream_t s);
+cudaError_t fill_f32(float* p, int64_t count, float v, cudaStream_t s);
+
+// ------------------------------------------------------------ BiIP
+// One pass of the row transform with a transposed store:
+//   out[j * ld_out + r] = T(in row r)[j],  r < rows, j < L
+// forward: v = in * scale * sign  ->  (Had/sqrt(P) (x) C_K) v
+// inverse: v = (Had/sqrt(P) (x) C_K^T) in  ->  v * sign / scale
+// scale_mode: 0 none, 1 multiply by scale[j], 2 divide by scale[j].
+// rotate == false: only the scaling and the transposed store.
+struct RowPass {
+  const void* in = nullptr;
+  bool in_bf16 = false;
+  int64_t ld_in = 0;
+  float* out = nullptr;
+  int64_t ld_out = 0;
+  int64_t rows = 0, L = 0;
+  const float* scale = nullptr;
+  int scale_mode = 0;
+  bool rotate = true;
+  bool inverse = false;
+  uint64_t sign_state = 0;  // 2 * seed + side
+};
+kronq_status rowpass(const RowPass& p, cudaStream_t s);
+// sum of squares along columns (colsq[n]) and rows (rowsq[m]) of W.
+kronq_status wnorms(const void* W, bool bf16, int64_t m, int64_t n, float* colsq, float* rowsq,
+                    float* partial, cudaStream_t s);
+size_t wnorms_partial_floats(int64_t m, int64_t n);
+// d[j] = (H[j,j] / nrm[j])^alpha, degenerate -> 1, normalised to geometric mean 1.
+kronq_status rescale_vector(const float* H, int64_t ldh, const float* nrm, int64_t len, float alpha,
+                            float* d, cudaStream_t s);
+
+// ------------------------------------------------------------ factorisation
+// In: H (n x n) full symmetric.  Out: U (upper) with U^T U = (H + lambda I)^-1,
+// dead-column flags, info.  ws: see chol_workspace_bytes.
+size_t chol_workspace_bytes(int64_t n);
+kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
+                                uint8_t* dead, int* info, void* ws, cudaStream_t s);
+
+// ------------------------------------------------------------ sweep
+struct SweepDesc {
+  float* W = nullptr;  // m x n, row stride n
+  const float* U = nullptr;  // n x n upper
+  int64_t m = 0, n = 0;
+  int bits = 4, group = 128;
+  bool asym = true;
+  uint8_t* codes = nullptr;
+  float* scales = nullptr;
+  float* zeros = nullptr;
+  int64_t ngroups = 1;
+  float* E = nullptr;  // m x n (caller) or nullptr
+  float* Eblk = nullptr;  // m x 128 workspace
+  const uint8_t* dead = nullptr;
+  const int* info = nullptr;
+  bool ordered = false;
+};
+kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s);
+
+// ------------------------------------------------------------ pack / misc
+kronq_status pack_codes(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* out,
+                        cudaStream_t s);
+kronq_status unpack_codes(const uint32_t* in, int64_t m, int64_t n, int bits, uint8_t* codes,
+                          cudaStream_t s);
+kronq_status diag_sums(const float* HX, int64_t n, const float* HG, int64_t m, double* dev2,
+                       cudaStream_t s);
+kronq_status dot_sum(const float* a, const float* b, int64_t count, double* dev1, double* partial,
+                     cudaStream_t s);
+
+}  // namespace kq

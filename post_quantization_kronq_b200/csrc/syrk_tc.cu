@@ -1,0 +1,277 @@
+// Factor accumulation H += A^T A on the 5th-generation tensor cores.
+//
+// KronQ README intro / "WaterKron and FlipFlop Hessian" Table 1 ("Marginal"
+// row): H_X = sum_t x_t x_t^T and H_G = sum_t g_t g_t^T.  For row-major
+// token data A (T x d) this is the GEMM C = A^T A with M = N = d and K = T;
+// both operands are read straight from A, so both are MN-major in shared
+// memory (d contiguous), which tcgen05 supports for bf16.
+//
+// Design (sm_100a):
+//  * one CTA per 128 x 256 output tile of the upper triangle (tiles entirely
+//    below the diagonal are never launched: ~half of the dense work);
+//  * warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner), warps 2-5 =
+//    epilogue; 4-stage smem ring of 64-token slices (48 KB per stage);
+//  * tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M = 128, N = 256, K = 16,
+//    accumulator in 256 TMEM columns;
+//  * epilogue: tcgen05.ld 32x32b, each element written once: (i, j) for
+//    i <= j and its mirror (j, i) for i < j, so H stays fully symmetric.
+//    Each output element belongs to exactly one CTA: no atomics.
+//  * the whole token range is one K loop, so concurrently running CTAs walk
+//    the same token slices and each slice of A is read from HBM about once
+//    per wave (the rest hits L2).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kq {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BOX_BYTES = 64 * BK * 2;                 // one 64-column x 64-token box
+constexpr int A_BYTES = BM * BK * 2;                   // 16 KB
+constexpr int B_BYTES = BN * BK * 2;                   // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;         // 48 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = BN;
+
+struct SyrkArgs {
+  float* H;
+  int64_t d;
+  int nk;       // number of 64-token slices
+  int nr, nc;   // row / column tile counts
+  int accumulate;
+};
+
+__device__ __forceinline__ void tile_of(int t, int nr, int nc, int& tr, int& tc) {
+  for (tr = 0; tr < nr; ++tr) {
+    const int first = (tr * BM) / BN;
+    const int cnt = nc - first;
+    if (t < cnt) {
+      tc = first + t;
+      return;
+    }
+    t -= cnt;
+  }
+  tc = nc;  // unreachable for a valid grid
+}
+
+__device__ __forceinline__ void put(float* p, float x, int acc) { *p = acc ? (*p + x) : x; }
+
+__global__ void __launch_bounds__(THREADS, 1)
+    syrk_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmap, SyrkArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  const uint32_t full0 = smem_u32(&bars[0]);
+  const uint32_t empty0 = smem_u32(&bars[STAGES]);
+  const uint32_t accbar = smem_u32(&bars[2 * STAGES]);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int tr, tc;
+  tile_of(blockIdx.x, args.nr, args.nc, tr, tc);
+  const int r0 = tr * BM, c0 = tc * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accbar, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t stage0 = smem_u32(smem);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < args.nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (kb / STAGES) & 1;
+        if (!mbar_wait(empty0 + 8 * s, ph ^ 1)) break;
+        const uint32_t full = full0 + 8 * s;
+        mbar_arrive_expect_tx(full, STAGE_BYTES);
+        const uint32_t a = stage0 + s * STAGE_BYTES;
+        const uint32_t b = a + A_BYTES;
+        const int y = kb * BK;
+        tma_load_2d(a, &tmap, full, r0, y);
+        tma_load_2d(a + BOX_BYTES, &tmap, full, r0 + 64, y);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) tma_load_2d(b + h * BOX_BYTES, &tmap, full, c0 + 64 * h, y);
+        issued = kb + 1;
+      }
+      // Make sure no copy is still landing when the CTA leaves (normally
+      // these phases completed long ago and each test returns at once).
+      for (int kb = issued - STAGES > 0 ? issued - STAGES : 0; kb < issued; ++kb)
+        mbar_wait(full0 + 8 * (kb % STAGES), (kb / STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, true, true);
+      for (int kb = 0; kb < args.nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (kb / STAGES) & 1;
+        if (!mbar_wait(full0 + 8 * s, ph)) break;
+        tc_fence_after();
+        const uint32_t a = stage0 + s * STAGE_BYTES;
+        const uint32_t b = a + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          // 16 tokens = 16 rows of 128 B inside every box: +2048 B per step.
+          const uint64_t ad = smem_desc_sw128(a + kk * 2048, BOX_BYTES, 1024);
+          const uint64_t bd = smem_desc_sw128(b + kk * 2048, BOX_BYTES, 1024);
+          mma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        mma_commit(empty0 + 8 * s);
+      }
+      mma_commit(accbar);
+    }
+    __syncwarp();
+  } else {
+    // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (its sub-partition).
+    const int q = warp & 3;
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(accbar, 0);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    if (ok) {
+      tc_fence_after();
+      const int64_t d = args.d;
+      const int64_t i = r0 + q * 32 + lane;
+      float* H = args.H;
+      const int acc = args.accumulate;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + cc * 32, v);
+        tmem_wait_ld();
+        const int64_t jb = c0 + cc * 32;
+        if (i < d) {
+          const bool dense = (jb >= i) && (jb + 32 <= d) &&
+                             ((reinterpret_cast<uintptr_t>(H + i * d + jb) & 15) == 0);
+          if (dense) {
+            float4* dst = reinterpret_cast<float4*>(H + i * d + jb);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              float4 x = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
+                                     __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3]));
+              if (acc) {
+                const float4 o = dst[t];
+                x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
+              }
+              dst[t] = x;
+            }
+          } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              const int64_t j = jb + t;
+              if (j < d && i <= j) put(H + i * d + j, __uint_as_float(v[t]), acc);
+            }
+          }
+        }
+        // Mirror (j, i) for i < j: 32 lanes write 32 consecutive floats.
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const int64_t j = jb + t;
+          if (i < d && j < d && i < j) put(H + j * d + i, __uint_as_float(v[t]), acc);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+__global__ void fill_kernel(float* p, int64_t count, float v) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count;
+       i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = v;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t fill_f32(float* p, int64_t count, float v, cudaStream_t s) {
+  if (count <= 0) return cudaSuccess;
+  const int threads = 256;
+  int64_t blocks = ceil_div(count, threads);
+  if (blocks > 4 * 148 * 8) blocks = 4 * 148 * 8;
+  fill_kernel<<<(unsigned)blocks, threads, 0, s>>>(p, count, v);
+  return cudaGetLastError();
+}
+
+cudaError_t status_fetch_syrk(int* out, cudaStream_t s) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  *out = v;
+  return e;
+}
+
+kronq_status syrk_bf16_tc(const void* A, int64_t T, int64_t d, int64_t lda, float* H,
+                          bool zero_first, cudaStream_t s) {
+  auto encode = encode_fn();
+  if (!encode) return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  CUtensorMap map;
+  cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)T};
+  cuuint64_t gstride[1] = {(cuuint64_t)(lda * 2)};
+  cuuint32_t box[2] = {64, (cuuint32_t)BK};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A), gdim, gstride,
+                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+  SyrkArgs args;
+  args.H = H;
+  args.d = d;
+  args.nk = (int)ceil_div(T, BK);
+  args.nr = (int)ceil_div(d, BM);
+  args.nc = (int)ceil_div(d, BN);
+  args.accumulate = zero_first ? 0 : 1;
+  int64_t ntiles = 0;
+  for (int tr = 0; tr < args.nr; ++tr) ntiles += args.nc - (tr * BM) / BN;
+
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(&syrk_bf16_tc_kernel), SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(syrk)");
+  syrk_bf16_tc_kernel<<<(unsigned)ntiles, THREADS, SMEM_BYTES, s>>>(map, args);
+  KQ_LAUNCH_CHECK("syrk_bf16_tc_kernel");
+  return KRONQ_OK;
+}
+
+}  // namespace kq

@@ -10,6 +10,10 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # The C-ABI library is built in-tree (nvcc cross-compiles for sm_100a,
+    # no GPU needed); an up-to-date build returns at once.
+    from post_quantization_kronq_b200.build import build
+    build()
 
 
 @pytest.fixture(scope="session")

@@ -1,0 +1,172 @@
+"""The C ABI without a GPU: exports, argument validation, host-only calls."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import alloc
+from post_quantization_kronq_b200 import _lib
+from post_quantization_kronq_b200.dist import shard_units
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = ctypes.c_void_p(4096)   # never dereferenced: every call below fails validation first
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "kronq.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(kronq_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert len(names) >= 15
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_version_and_error_strings():
+    assert b"sm_100a" in _lib.lib.kronq_version()
+    assert isinstance(_lib.lib.kronq_last_error(), bytes)
+
+
+def _st(v):
+    return int(v)
+
+
+def test_pack_rejects_three_bits():
+    assert _st(_lib.lib.kronq_pack(FAKE, 4, 8, 3, FAKE, None)) == _lib.ERR_INVALID_ARG
+    assert b"3-bit" in _lib.lib.kronq_last_error()
+    assert _st(_lib.lib.kronq_unpack(FAKE, 4, 8, 5, FAKE, None)) == _lib.ERR_INVALID_ARG
+    assert _st(_lib.lib.kronq_pack(None, 4, 8, 4, FAKE, None)) == _lib.ERR_INVALID_ARG
+
+
+def _qp(**kw):
+    base = dict(bits=4, group=128, asym=1, damp_rel=0.01, block=128, flags=0)
+    base.update(kw)
+    return _lib.QuantParams(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=5), _lib.ERR_INVALID_ARG),
+    (dict(bits=1), _lib.ERR_INVALID_ARG),
+    (dict(group=96), _lib.ERR_INVALID_ARG),
+    (dict(group=0), _lib.ERR_INVALID_ARG),
+    (dict(block=64), _lib.ERR_UNSUPPORTED),
+    (dict(asym=2), _lib.ERR_INVALID_ARG),
+    (dict(damp_rel=-1.0), _lib.ERR_INVALID_ARG),
+    (dict(damp_rel=float("nan")), _lib.ERR_INVALID_ARG),
+    (dict(flags=64), _lib.ERR_INVALID_ARG),
+    (dict(flags=_lib.WRITE_E), _lib.ERR_INVALID_ARG),   # E is NULL below
+])
+def test_quantize_layer_validation(kw, status):
+    p = _qp(**kw)
+    r = _lib.lib.kronq_quantize_layer(FAKE, FAKE, 64, 256, ctypes.byref(p), FAKE, FAKE, FAKE, None,
+                                      FAKE, FAKE, 1 << 40, None)
+    assert _st(r) == status
+
+
+def test_quantize_layer_null_and_workspace():
+    p = _qp()
+    assert _st(_lib.lib.kronq_quantize_layer(FAKE, FAKE, 64, 256, None, FAKE, FAKE, FAKE, None, FAKE,
+                                             FAKE, 1 << 40, None)) == _lib.ERR_INVALID_ARG
+    need = _lib.lib.kronq_quantize_workspace_bytes(64, 256, ctypes.byref(p))
+    assert need > 64 * 128 * 4
+    r = _lib.lib.kronq_quantize_layer(FAKE, FAKE, 64, 256, ctypes.byref(p), FAKE, FAKE, FAKE, None,
+                                      FAKE, FAKE, need - 1, None)
+    assert _st(r) == _lib.ERR_INVALID_ARG
+    r = _lib.lib.kronq_quantize_layer(FAKE, FAKE, 0, 256, ctypes.byref(p), FAKE, FAKE, FAKE, None,
+                                      FAKE, FAKE, need, None)
+    assert _st(r) == _lib.ERR_INVALID_ARG
+
+
+def test_accumulate_validation():
+    L = _lib.lib
+    assert _st(L.kronq_accumulate_factors(FAKE, 7, 16, 8, 8, FAKE, 1, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_accumulate_factors(FAKE, 0, 16, 8, 4, FAKE, 1, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_accumulate_factors(FAKE, 0, -1, 8, 8, FAKE, 1, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_accumulate_factors(None, 0, 16, 8, 8, FAKE, 1, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_accumulate_factors(FAKE, 0, 16, 8, 8, None, 1, None)) == _lib.ERR_INVALID_ARG
+
+
+def test_biip_validation():
+    L = _lib.lib
+    ws = L.kronq_biip_workspace_bytes(64, 128)
+    assert ws >= 128 * 128 * 4
+    ok_ws = ctypes.c_void_p(4096 * 256)
+    # H_G required for the output-side rescale
+    r = L.kronq_biip_forward(FAKE, 0, ctypes.c_void_p(8192), 64, 128, FAKE, None, 0, 0.25, 0, FAKE,
+                             FAKE, ok_ws, ws, None)
+    assert _st(r) == _lib.ERR_INVALID_ARG
+    # odd factor 257 of n = 514 is beyond the DCT limit
+    ws2 = L.kronq_biip_workspace_bytes(64, 514)
+    r = L.kronq_biip_forward(FAKE, 0, ctypes.c_void_p(8192), 64, 514, FAKE, FAKE, 0, 0.25, 0, FAKE,
+                             FAKE, ok_ws, ws2, None)
+    assert _st(r) == _lib.ERR_UNSUPPORTED
+    # bad mode, aliasing, misaligned workspace
+    r = L.kronq_biip_forward(FAKE, 0, ctypes.c_void_p(8192), 64, 128, FAKE, FAKE, 0, 0.25, 9, FAKE,
+                             FAKE, ok_ws, ws, None)
+    assert _st(r) == _lib.ERR_INVALID_ARG
+    r = L.kronq_biip_forward(FAKE, 0, FAKE, 64, 128, FAKE, FAKE, 0, 0.25, 0, FAKE, FAKE, ok_ws, ws, None)
+    assert _st(r) == _lib.ERR_INVALID_ARG
+    r = L.kronq_biip_forward(FAKE, 0, ctypes.c_void_p(8192), 64, 128, FAKE, FAKE, 0, 0.25, 0, FAKE,
+                             FAKE, ctypes.c_void_p(4096 + 16), ws, None)
+    assert _st(r) == _lib.ERR_INVALID_ARG
+    r = L.kronq_biip_inverse(FAKE, 64, 128, 0, 0, FAKE, FAKE, ok_ws, ws - 256, None)
+    assert _st(r) == _lib.ERR_INVALID_ARG
+
+
+def test_sensitivity_and_loss_validation():
+    L = _lib.lib
+    out = (ctypes.c_double * 3)()
+    assert _st(L.kronq_sensitivity(None, 4, FAKE, 4, out, FAKE, 16, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_sensitivity(FAKE, 4, FAKE, 4, out, FAKE, 8, None)) == _lib.ERR_INVALID_ARG
+    d = ctypes.c_double()
+    assert _st(L.kronq_kfac_loss(FAKE, FAKE, 4, 4, ctypes.byref(d), FAKE, 0, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_device_status(None, None)) == _lib.ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ host allocation
+def test_budget_allocation_matches_oracle():
+    from post_quantization_kronq_b200 import kronq_allocate_bits
+    rng = np.random.default_rng(0)
+    sizes = [4096 * 4096, 1024 * 4096, 1024 * 4096, 4096 * 4096, 14336 * 4096, 14336 * 4096,
+             4096 * 14336] * 32
+    for trial in range(10):
+        s = list(np.exp(rng.normal(size=len(sizes)) * 3))
+        assert kronq_allocate_bits(s, sizes, 2.5, 2, 4) == alloc.allocate_budget(s, sizes, 2.5, 2, 4)
+    s = [1.0] * 8
+    assert kronq_allocate_bits(s, [1] * 8, 2.5) == alloc.allocate_budget(s, [1] * 8, 2.5)
+
+
+def test_topn_allocation_matches_oracle():
+    from post_quantization_kronq_b200 import kronq_allocate_topn_types
+    rng = np.random.default_rng(1)
+    names = ["q", "k", "v", "o", "gate", "up", "down"]
+    types = names * 32
+    ids = [names.index(t) for t in types]
+    for N in (0, 1, 3, 7):
+        s = list(np.exp(rng.normal(size=len(types))))
+        assert kronq_allocate_topn_types(s, ids, 7, 2, N) == alloc.allocate_topn_types(s, types, 2, N)
+
+
+def test_allocation_validation():
+    L = _lib.lib
+    out = (ctypes.c_int * 2)()
+    s = (ctypes.c_double * 2)(1.0, 2.0)
+    z = (ctypes.c_int64 * 2)(1, 0)
+    assert _st(L.kronq_allocate_bits(s, z, 2, 2.5, 2, 4, out)) == _lib.ERR_INVALID_ARG
+    z = (ctypes.c_int64 * 2)(1, 1)
+    assert _st(L.kronq_allocate_bits(s, z, 2, 1.5, 2, 4, out)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_allocate_bits(s, z, 2, 2.5, 2, 4, out)) == _lib.OK
+
+
+def test_shard_units_partition():
+    for n in (0, 1, 7, 224):
+        for w in (1, 2, 3, 8):
+            got = sum((shard_units(n, r, w) for r in range(w)), [])
+            assert got == list(range(n))

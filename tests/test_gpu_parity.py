@@ -1,0 +1,319 @@
+"""GPU parity: every library call against the float64 oracle on the same
+seeded inputs.  Tolerances (from the pass's statement of the problem):
+factors and traces 1e-3 relative Frobenius; codes bit-exact against the
+float32 schedule-mirroring oracle when fed the same fp32 W~ and U, and at
+most 0.5 % code disagreement end to end; K-FAC loss within 1 %; packing
+bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import post_quantization_kronq_b200 as kq
+from oracle import biip, factors, loss, pack, pipeline, sweep
+from post_quantization_kronq_b200.layer import LayerPass
+from synth import llama_layer, tiny_layer
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+# ------------------------------------------------------------------ factors
+@pytest.mark.parametrize("T,d", [(4096, 256), (3037, 392), (1000, 1000), (64, 128), (2048, 640)])
+def test_factor_bf16_tensor_core(T, d):
+    g = torch.Generator(device=DEV).manual_seed(T + d)
+    X = (torch.randn(T, d, device=DEV, generator=g) * torch.exp(torch.randn(d, device=DEV, generator=g))).bfloat16()
+    H = torch.full((d, d), float("nan"), device=DEV)
+    kq.kronq_accumulate_factors(X, H, zero_first=True)
+    torch.cuda.synchronize()
+    ref = factors.factor(to_np(X))
+    Hn = to_np(H)
+    assert rel(Hn, ref) < 1e-5
+    assert np.array_equal(Hn, Hn.T)
+    assert kq.kronq_device_status() == 0
+
+
+def test_factor_bf16_streamed_chunks_and_strided_view():
+    T, d, full = 5000, 384, 512
+    g = torch.Generator(device=DEV).manual_seed(7)
+    Xb = torch.randn(T, full, device=DEV, generator=g).bfloat16()
+    X = Xb[:, :d]                       # lda = 512 > d
+    H = torch.empty(d, d, device=DEV)
+    for t0 in range(0, T, 1024):        # chunk starts stay 16-byte aligned
+        kq.kronq_accumulate_factors(X[t0:t0 + 1024], H, zero_first=(t0 == 0))
+    torch.cuda.synchronize()
+    assert rel(to_np(H), factors.factor(to_np(X))) < 1e-5
+
+
+def test_factor_small_and_empty():
+    X = torch.randn(50, 96, device=DEV).bfloat16()      # below the tensor-core tile: SIMT kernel
+    H = torch.empty(96, 96, device=DEV)
+    kq.kronq_accumulate_factors(X, H, zero_first=True)
+    torch.cuda.synchronize()
+    assert rel(to_np(H), factors.factor(to_np(X))) < 1e-5
+    H.fill_(3.0)
+    kq.kronq_accumulate_factors(X[:0], H, zero_first=True)   # T = 0
+    torch.cuda.synchronize()
+    assert float(H.abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("T,d", [(2048, 256), (777, 200)])
+def test_factor_f32(T, d):
+    _, X, _ = tiny_layer(m=8, n=d, T=T, seed=1)
+    Xt = torch.from_numpy(X).to(DEV)
+    H = torch.empty(d, d, device=DEV)
+    kq.kronq_accumulate_factors(Xt, H, zero_first=True)
+    kq.kronq_accumulate_factors(Xt, H, zero_first=False)
+    torch.cuda.synchronize()
+    assert rel(to_np(H), 2 * factors.factor(X)) < 1e-5
+
+
+def test_factor_max_dimension_sampled():
+    T, d = 256, 28672
+    g = torch.Generator(device=DEV).manual_seed(3)
+    X = torch.randn(T, d, device=DEV, generator=g).bfloat16()
+    H = torch.empty(d, d, device=DEV)
+    kq.kronq_accumulate_factors(X, H, zero_first=True)
+    torch.cuda.synchronize()
+    cols = np.random.default_rng(0).choice(d, 16, replace=False)
+    Xn = to_np(X)
+    ref = factors.factor_columns(Xn, cols)
+    got = to_np(H[:, torch.as_tensor(cols, device=DEV)])
+    assert rel(got, ref) < 1e-5
+    del H
+
+
+def test_sensitivity_traces():
+    W, X, G = tiny_layer(m=192, n=256, T=2048, seed=5)
+    Xt, Gt = torch.from_numpy(X).to(DEV), torch.from_numpy(G).to(DEV)
+    HX = torch.empty(256, 256, device=DEV)
+    HG = torch.empty(192, 192, device=DEV)
+    kq.kronq_accumulate_factors(Xt, HX, True)
+    kq.kronq_accumulate_factors(Gt, HG, True)
+    trx, trg, s = kq.kronq_sensitivity(HX, HG)
+    rx, rg = factors.trace_from_rows(X), factors.trace_from_rows(G)
+    assert abs(trx - rx) / rx < 1e-3 and abs(trg - rg) / rg < 1e-3
+    assert abs(s - rx * rg) / (rx * rg) < 2e-3
+
+
+# ------------------------------------------------------------------ BiIP
+def _biip_case(m, n, seed, wdtype=torch.float32):
+    W, X, G = tiny_layer(m=m, n=n, T=3 * max(m, n), seed=seed)
+    HX = (X.astype(np.float64).T @ X.astype(np.float64)).astype(np.float32)
+    HG = (G.astype(np.float64).T @ G.astype(np.float64)).astype(np.float32)
+    Wg = torch.from_numpy(W).to(DEV).to(wdtype)
+    return Wg, to_np(Wg), HX, HG
+
+
+@pytest.mark.parametrize("m,n", [(256, 256), (200, 448), (96, 392), (3, 5), (1, 24)])
+def test_biip_forward_inverse(m, n):
+    Wg, W, HX, HG = _biip_case(m, n, seed=m + n)
+    HXg, HGg = torch.from_numpy(HX).to(DEV), torch.from_numpy(HG).to(DEV)
+    Wt = torch.empty(m, n, device=DEV)
+    din = torch.empty(n, device=DEV)
+    dout = torch.empty(m, device=DEV)
+    kq.kronq_biip_forward(Wg, Wt, HXg, HGg, 11, 0.25, "full", din, dout)
+    torch.cuda.synchronize()
+    rWt, rHX, rHG, rdin, rdout = biip.biip_forward(W, HX, HG, 11, 0.25, "full")
+    assert rel(to_np(din), rdin) < 1e-6 and rel(to_np(dout), rdout) < 1e-6
+    assert rel(to_np(Wt), rWt) < 1e-5
+    assert rel(to_np(HXg), rHX) < 1e-5
+    assert rel(to_np(HGg), rHG) < 1e-5
+    back = Wt.clone()
+    kq.kronq_biip_inverse(back, 11, "full", din, dout)
+    torch.cuda.synchronize()
+    assert rel(to_np(back), W) < 1e-5
+
+
+@pytest.mark.parametrize("mode", ["full", "no_rescale", "su_only", "sv_only"])
+def test_biip_modes_bf16(mode):
+    m, n = 160, 224          # 160 = 32*5, 224 = 32*7
+    Wg, W, HX, HG = _biip_case(m, n, seed=2, wdtype=torch.bfloat16)
+    HXg, HGg = torch.from_numpy(HX).to(DEV), torch.from_numpy(HG).to(DEV)
+    Wt = torch.empty(m, n, device=DEV)
+    din, dout = torch.empty(n, device=DEV), torch.empty(m, device=DEV)
+    kq.kronq_biip_forward(Wg, Wt, HXg, HGg, 5, 0.25, mode, din, dout)
+    torch.cuda.synchronize()
+    rWt, rHX, rHG, _, _ = biip.biip_forward(W, HX, HG, 5, 0.25, mode)
+    assert rel(to_np(Wt), rWt) < 1e-5
+    assert rel(to_np(HXg), rHX) < 1e-5
+    assert rel(to_np(HGg), rHG) < 1e-5
+
+
+# ------------------------------------------------------------------ factorisation
+def _spd(n, seed, T=None):
+    _, X, _ = tiny_layer(m=4, n=n, T=T or 3 * n, seed=seed)
+    return (X.astype(np.float64).T @ X.astype(np.float64)).astype(np.float32)
+
+
+@pytest.mark.parametrize("n", [256, 200, 640, 1000])
+def test_cholesky_of_damped_inverse(n):
+    H = _spd(n, seed=n)
+    m = 32
+    W = np.zeros((m, n), dtype=np.float32)
+    lp = LayerPass(m, n, bits=4, group=128)
+    lp.HX.copy_(torch.from_numpy(H))
+    lp.Wt.copy_(torch.from_numpy(W))
+    lp.quantize()
+    torch.cuda.synchronize()
+    assert int(lp.info.item()) == 0
+    H1, _, _ = sweep.dead_columns(H, W)
+    A, _ = sweep.damp(H1, 0.01)
+    U = sweep.chol_upper_of_inverse(A)
+    got = np.triu(to_np(lp.HX))
+    assert rel(got, U) < 2e-4
+
+
+def test_cholesky_not_positive_definite_reports_info():
+    n = 130
+    H = np.eye(n, dtype=np.float32)
+    H[37, 37] = -5.0
+    lp = LayerPass(8, n, bits=4, group=128)
+    lp.HX.copy_(torch.from_numpy(H))
+    lp.Wt.zero_()
+    lp.quantize()
+    torch.cuda.synchronize()
+    A, _ = sweep.damp(H.astype(np.float64), 0.01)
+    assert int(lp.info.item()) == sweep.reverse_chol_failure(A) == 38
+
+
+# ------------------------------------------------------------------ sweep
+def _sweep_inputs(m, n, seed):
+    W, X, _ = tiny_layer(m=m, n=n, T=4 * n, seed=seed)
+    H = X.astype(np.float64).T @ X.astype(np.float64)
+    Wt, HXt, _, _, _ = biip.biip_forward(W, H, None, seed, 0.25, "sv_only")
+    A, _ = sweep.damp(HXt, 0.01)
+    U = sweep.chol_upper_of_inverse(A)
+    return Wt.astype(np.float32), U.astype(np.float32)
+
+
+@pytest.mark.parametrize("m,n,bits,group,asym", [
+    (69, 424, 4, 128, True), (69, 424, 2, 64, True), (69, 424, 3, -1, True),
+    (40, 512, 2, 256, True), (33, 300, 4, 32, False), (16, 128, 3, 128, True), (5, 7, 2, -1, True),
+])
+def test_sweep_bit_exact_against_f32_oracle(m, n, bits, group, asym):
+    Wt, U = _sweep_inputs(m, n, seed=m * n)
+    ref = sweep.gptq_sweep_f32(Wt, U, bits, group, asym, 128)
+    p = kq.QuantParams(bits=bits, group=group, asym=1 if asym else 0, damp_rel=0.01, block=128,
+                       flags=kq.U_GIVEN | kq.ORDERED_FP32 | kq.WRITE_E)
+    ng = 1 if group == -1 else -(-n // group)
+    Wg = torch.from_numpy(Wt).to(DEV)
+    Ug = torch.from_numpy(U).to(DEV)
+    codes = torch.empty(m, n, dtype=torch.uint8, device=DEV)
+    sc = torch.empty(m, ng, device=DEV)
+    zp = torch.empty(m, ng, device=DEV)
+    E = torch.empty(m, n, device=DEV)
+    info = torch.ones(1, dtype=torch.int32, device=DEV)
+    kq.kronq_quantize_layer(Wg, Ug, p, codes, sc, zp, info, E=E)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    assert np.array_equal(codes.cpu().numpy().astype(np.int64), ref["codes"])
+    assert np.array_equal(sc.cpu().numpy(), ref["scales"])
+    assert np.array_equal(zp.cpu().numpy(), ref["zeros"])
+    assert np.array_equal(Wg.cpu().numpy(), ref["Q"])
+    assert np.array_equal(E.cpu().numpy(), ref["E"])
+
+
+def test_sweep_fast_path_close_to_ordered():
+    m, n = 256, 640
+    Wt, U = _sweep_inputs(m, n, seed=9)
+    ref = sweep.gptq_sweep_f32(Wt, U, 2, 128, True, 128)
+    lp = LayerPass(m, n, bits=2, group=128, flags=kq.U_GIVEN)
+    lp.Wt.copy_(torch.from_numpy(Wt))
+    lp.HX.copy_(torch.from_numpy(U))
+    lp.quantize()
+    torch.cuda.synchronize()
+    dis = np.mean(lp.codes.cpu().numpy().astype(np.int64) != ref["codes"])
+    assert dis <= 0.005
+
+
+# ------------------------------------------------------------------ end to end
+def _gpu_pass(X, G, W, bits, group, mode="full", seed=0):
+    m, n = W.shape
+    lp = LayerPass(m, n, bits=bits, group=group, seed=seed, mode=mode)
+    lp.run(X, G, W)
+    What = lp.Wt.clone()
+    kq.kronq_biip_inverse(What, seed, mode, lp.d_in, lp.d_out)
+    torch.cuda.synchronize()
+    return lp, What
+
+
+def _compare_end_to_end(X, G, W, bits, group, seed=0):
+    lp, What = _gpu_pass(X, G, W, bits, group, seed=seed)
+    Xn, Gn, Wn = to_np(X), to_np(G), to_np(W)
+    ref = pipeline.quantize_layer(Xn, Gn, Wn, bits=bits, group=group, seed=seed, block=128)
+    assert int(lp.info.item()) == 0
+    dis = np.mean(lp.codes.cpu().numpy().astype(np.int64) != ref["codes"])
+    gl = loss.kfac_loss(Wn - to_np(What), ref["HX"], ref["HG"])
+    trx, trg, s = lp.sens
+    assert abs(trx - ref["trX"]) / ref["trX"] < 1e-3
+    assert abs(trg - ref["trG"]) / ref["trG"] < 1e-3
+    return dis, gl, ref["loss"]
+
+
+def test_end_to_end_tiny_config():
+    W, X, G = tiny_layer()
+    dis, gl, rl = _compare_end_to_end(torch.from_numpy(X).to(DEV), torch.from_numpy(G).to(DEV),
+                                      torch.from_numpy(W).to(DEV), 4, 128)
+    assert dis <= 0.005, dis
+    assert abs(gl - rl) / rl < 0.01, (gl, rl)
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (2, 128), (3, 64), (2, -1)])
+def test_end_to_end_bf16_llama_like(bits, group):
+    W, X, G = llama_layer(384, 768, 4096, seed=bits * 10 + (group % 7), device=DEV)
+    dis, gl, rl = _compare_end_to_end(X, G, W, bits, group)
+    assert dis <= 0.005, dis
+    assert abs(gl - rl) / rl < 0.01, (gl, rl)
+
+
+def test_factors_of_end_to_end_pass():
+    W, X, G = llama_layer(256, 512, 3000, seed=4, device=DEV)
+    lp = LayerPass(256, 512, bits=4, group=128)
+    lp.accumulate(X, G, chunk=1024)
+    torch.cuda.synchronize()
+    assert rel(to_np(lp.HX), factors.factor(to_np(X))) < 1e-3
+    assert rel(to_np(lp.HG), factors.factor(to_np(G))) < 1e-3
+
+
+def test_kfac_loss_diagnostic():
+    m, n = 128, 256
+    W, X, G = tiny_layer(m=m, n=n, T=1024, seed=8)
+    ref = pipeline.quantize_layer(X, G, W, bits=3, group=64, seed=1, block=128)
+    lp = LayerPass(m, n, bits=3, group=64, seed=1, flags=kq.WRITE_E)
+    lp.accumulate(torch.from_numpy(X).to(DEV), torch.from_numpy(G).to(DEV))
+    lp.transform(torch.from_numpy(W).to(DEV))
+    E = torch.empty(m, n, device=DEV)
+    kq.kronq_quantize_layer(lp.Wt, lp.HX, lp.params, lp.codes, lp.scales, lp.zeros, lp.info,
+                            E=E, ws=lp.ws_quant)
+    got = kq.kronq_kfac_loss(E, lp.HG)
+    want = loss.sweep_loss_from_errors(ref["E"], ref["HGt"])
+    assert abs(got - want) / want < 0.01, (got, want)
+
+
+# ------------------------------------------------------------------ packing
+@pytest.mark.parametrize("bits,m,n", [(4, 64, 4096), (2, 33, 1000), (4, 5, 13), (2, 1, 16)])
+def test_pack_unpack_bit_exact(bits, m, n):
+    rng = np.random.default_rng(n)
+    codes = rng.integers(0, 2 ** bits, size=(m, n)).astype(np.uint8)
+    cg = torch.from_numpy(codes).to(DEV)
+    words = torch.empty(m, kq.words_per_row(n, bits), dtype=torch.int32, device=DEV)
+    kq.kronq_pack(cg, bits, words)
+    back = torch.empty(m, n, dtype=torch.uint8, device=DEV)
+    kq.kronq_unpack(words, m, n, bits, back)
+    torch.cuda.synchronize()
+    assert np.array_equal(words.cpu().numpy().view(np.uint32), pack.pack(codes, bits))
+    assert np.array_equal(back.cpu().numpy(), codes)
+
+
+def test_device_status_clean():
+    assert kq.kronq_device_status() == 0
