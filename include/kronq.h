@@ -231,6 +231,10 @@ size_t kronq_kfac_loss_workspace_bytes(int64_t m, int64_t n);
 kronq_status kronq_kfac_loss(const float* E, const float* HG, int64_t m, int64_t n, double* out,
                              void* workspace, size_t ws_bytes, kronq_stream_t s);
 
+/* Number of kernels this library has launched in the process so far (all
+ * devices and streams); a host counter, no synchronisation. */
+uint64_t kronq_launch_count(void);
+
 const char* kronq_last_error(void);
 const char* kronq_version(void);
 

@@ -19,12 +19,21 @@ __all__ = [
     "kronq_allocate_topn_types", "kronq_biip_workspace_bytes", "kronq_biip_forward",
     "kronq_biip_inverse", "kronq_quantize_workspace_bytes", "kronq_quantize_layer",
     "kronq_pack", "kronq_unpack", "kronq_device_status", "kronq_kfac_loss_workspace_bytes",
-    "kronq_kfac_loss", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
+    "kronq_kfac_loss", "kronq_launch_count", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
 ]
 
 
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _rowmajor(t, name):
+    """The C ABI takes dense row-major arrays; refuse anything else loudly."""
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous row-major tensor")
+    if t is not None and not t.is_cuda:
+        raise ValueError(f"{name} must live in device memory")
+    return t
 
 
 def _stream(stream=None):
@@ -56,6 +65,10 @@ def kronq_version() -> str:
     return lib.kronq_version().decode()
 
 
+def kronq_launch_count() -> int:
+    return int(lib.kronq_launch_count())
+
+
 def kronq_last_error() -> str:
     return lib.kronq_last_error().decode(errors="replace")
 
@@ -63,6 +76,9 @@ def kronq_last_error() -> str:
 def kronq_accumulate_factors(A, H, zero_first: bool = False, lda: int | None = None, stream=None):
     """H (d x d float32) += A^T A for A (T x d, bf16 or float32, row stride lda)."""
     T, d = A.shape
+    if A.stride(1) != 1:
+        raise ValueError("A must have unit stride along d (row-major token rows)")
+    _rowmajor(H, "H")
     lda = A.stride(0) if lda is None else lda
     check(lib.kronq_accumulate_factors(_ptr(A), _dtype_code(A), T, d, lda, _ptr(H),
                                        1 if zero_first else 0, _stream(stream)))
@@ -70,6 +86,7 @@ def kronq_accumulate_factors(A, H, zero_first: bool = False, lda: int | None = N
 
 def kronq_sensitivity(HX, HG, ws=None, stream=None):
     """(tr(H_X), tr(H_G), tr(H_G) * tr(H_X)) as Python floats (synchronises)."""
+    _rowmajor(HX, "HX"), _rowmajor(HG, "HG")
     out = (ctypes.c_double * 3)()
     ws = workspace(256, HX.device) if ws is None else ws
     check(lib.kronq_sensitivity(_ptr(HX), HX.shape[0], _ptr(HG), HG.shape[0], out, _ptr(ws),
@@ -102,6 +119,8 @@ def kronq_biip_workspace_bytes(m: int, n: int) -> int:
 def kronq_biip_forward(W, Wt, HX, HG, seed: int, alpha: float, mode: str, d_in, d_out, ws=None,
                        stream=None):
     m, n = W.shape
+    for t, name in ((W, "W"), (Wt, "Wt"), (HX, "HX"), (HG, "HG"), (d_in, "d_in"), (d_out, "d_out")):
+        _rowmajor(t, name)
     ws = workspace(kronq_biip_workspace_bytes(m, n), W.device) if ws is None else ws
     check(lib.kronq_biip_forward(_ptr(W), _dtype_code(W), _ptr(Wt), m, n, _ptr(HX), _ptr(HG),
                                  int(seed), float(alpha), BIIP_MODES[mode], _ptr(d_in), _ptr(d_out),
@@ -110,6 +129,7 @@ def kronq_biip_forward(W, Wt, HX, HG, seed: int, alpha: float, mode: str, d_in, 
 
 def kronq_biip_inverse(W, seed: int, mode: str, d_in, d_out, ws=None, stream=None):
     m, n = W.shape
+    _rowmajor(W, "W")
     ws = workspace(kronq_biip_workspace_bytes(m, n), W.device) if ws is None else ws
     check(lib.kronq_biip_inverse(_ptr(W), m, n, int(seed), BIIP_MODES[mode], _ptr(d_in),
                                  _ptr(d_out), _ptr(ws), ws.numel(), _stream(stream)))
@@ -122,6 +142,9 @@ def kronq_quantize_workspace_bytes(m: int, n: int, params: QuantParams) -> int:
 def kronq_quantize_layer(Wt, HX, params: QuantParams, codes, scales, zeros, info, E=None, ws=None,
                          stream=None):
     m, n = Wt.shape
+    for t, name in ((Wt, "Wt"), (HX, "HX"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
+                    (info, "info"), (E, "E")):
+        _rowmajor(t, name)
     ws = workspace(kronq_quantize_workspace_bytes(m, n, params), Wt.device) if ws is None else ws
     check(lib.kronq_quantize_layer(_ptr(Wt), _ptr(HX), m, n, ctypes.byref(params), _ptr(codes),
                                    _ptr(scales), _ptr(zeros), _ptr(E), _ptr(info), _ptr(ws),
@@ -130,6 +153,7 @@ def kronq_quantize_layer(Wt, HX, params: QuantParams, codes, scales, zeros, info
 
 def kronq_pack(codes, bits: int, out, stream=None):
     m, n = codes.shape
+    _rowmajor(codes, "codes"), _rowmajor(out, "out")
     check(lib.kronq_pack(_ptr(codes), m, n, bits, _ptr(out), _stream(stream)))
 
 
@@ -149,6 +173,7 @@ def kronq_kfac_loss_workspace_bytes(m: int, n: int) -> int:
 
 def kronq_kfac_loss(E, HG, ws=None, stream=None) -> float:
     m, n = E.shape
+    _rowmajor(E, "E"), _rowmajor(HG, "HG")
     ws = workspace(kronq_kfac_loss_workspace_bytes(m, n), E.device) if ws is None else ws
     out = ctypes.c_double(0.0)
     check(lib.kronq_kfac_loss(_ptr(E), _ptr(HG), m, n, ctypes.byref(out), _ptr(ws), ws.numel(),

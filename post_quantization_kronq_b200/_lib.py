@@ -1,7 +1,9 @@
 """ctypes declarations of libkronq.so (the C ABI in include/kronq.h).
 
-The shared library is loaded from this package directory; if it is missing
-the import fails loudly -- there is no other implementation to fall back to.
+The shared library is loaded from this package directory on first use; if it
+is missing or stale that first call fails loudly -- there is no other
+implementation to fall back to.  (Loading lazily lets the build module be
+imported before the library exists.)
 """
 from __future__ import annotations
 
@@ -56,6 +58,7 @@ SIGNATURES = {
     "kronq_device_status": (_int, [_ip, _vp]),
     "kronq_kfac_loss_workspace_bytes": (_sz, [_i64, _i64]),
     "kronq_kfac_loss": (_int, [_vp, _vp, _i64, _i64, _dp, _vp, _sz, _vp]),
+    "kronq_launch_count": (ctypes.c_uint64, []),
     "kronq_last_error": (ctypes.c_char_p, []),
     "kronq_version": (ctypes.c_char_p, []),
 }
@@ -74,7 +77,19 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     return lib
 
 
-lib = load()
+class _LazyLib:
+    """Loads libkronq.so at the first attribute access."""
+
+    def __init__(self):
+        self._lib = None
+
+    def __getattr__(self, name):
+        if self._lib is None:
+            self._lib = load()
+        return getattr(self._lib, name)
+
+
+lib = _LazyLib()
 
 
 def check(status: int) -> None:

@@ -3,6 +3,7 @@
 // computes on the host except the bit allocation (a host-only call).
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -13,6 +14,9 @@
 namespace kq {
 
 static thread_local std::string g_last_error;
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 void set_error(const std::string& msg) { g_last_error = msg; }
 
@@ -106,6 +110,8 @@ extern "C" {
 const char* kronq_last_error(void) { return g_last_error.c_str(); }
 
 const char* kronq_version(void) { return "kronq-b200 0.1 (sm_100a)"; }
+
+uint64_t kronq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 kronq_status kronq_accumulate_factors(const void* A, kronq_dtype dt, int64_t T, int64_t d,
                                       int64_t lda, float* H, int zero_first, kronq_stream_t s) {

@@ -23,8 +23,12 @@ kronq_status cuda_fail(cudaError_t e, const char* what);
     if (e__ != cudaSuccess) return ::kq::cuda_fail(e__, #call);        \
   } while (0)
 
+// Counts every kernel launch of the library (kronq_launch_count).
+void count_launch();
+
 #define KQ_LAUNCH_CHECK(name)                                          \
   do {                                                                 \
+    ::kq::count_launch();                                              \
     cudaError_t e__ = cudaGetLastError();                              \
     if (e__ != cudaSuccess) return ::kq::cuda_fail(e__, name);         \
   } while (0)

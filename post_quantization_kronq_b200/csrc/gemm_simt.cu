@@ -140,6 +140,7 @@ cudaError_t gemm_f32(const GemmDesc& g, cudaStream_t s) {
   dim3 grid((unsigned)ceil_div(g.N, TN), (unsigned)ceil_div(g.M, TM), (unsigned)g.batch);
   if (g.ordered) gemm_kernel<true><<<grid, NT, 0, s>>>(g);
   else gemm_kernel<false><<<grid, NT, 0, s>>>(g);
+  count_launch();
   return cudaGetLastError();
 }
 

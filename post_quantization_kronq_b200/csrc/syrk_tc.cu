@@ -226,6 +226,7 @@ cudaError_t fill_f32(float* p, int64_t count, float v, cudaStream_t s) {
   int64_t blocks = ceil_div(count, threads);
   if (blocks > 4 * 148 * 8) blocks = 4 * 148 * 8;
   fill_kernel<<<(unsigned)blocks, threads, 0, s>>>(p, count, v);
+  count_launch();
   return cudaGetLastError();
 }
 

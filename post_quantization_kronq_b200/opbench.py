@@ -1,0 +1,88 @@
+"""Run (and time) one library call on a synthetic input of a chosen size.
+
+    python -m post_quantization_kronq_b200.opbench accumulate --tokens 16384 --d 4096 [--reps 3]
+    python -m post_quantization_kronq_b200.opbench biip --m 4096 --n 4096
+    python -m post_quantization_kronq_b200.opbench quantize --m 4096 --n 4096 --bits 2
+    python -m post_quantization_kronq_b200.opbench pack --m 8192 --n 28672 --bits 2
+
+Meant for profiling a single kernel family (e.g. under ncu) at a size that
+is smaller than the full benchmark; prints one JSON line with the mean
+CUDA-event time per call.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def main(argv=None):
+    import torch
+
+    import post_quantization_kronq_b200 as kq
+    from post_quantization_kronq_b200.layer import LayerPass
+    from synth import llama_layer
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("op", choices=["accumulate", "biip", "quantize", "pack"])
+    ap.add_argument("--tokens", type=int, default=16384)
+    ap.add_argument("--d", type=int, default=4096)
+    ap.add_argument("--m", type=int, default=4096)
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--bits", type=int, default=2)
+    ap.add_argument("--group", type=int, default=128)
+    ap.add_argument("--reps", type=int, default=3)
+    a = ap.parse_args(argv)
+    dev = torch.device("cuda", 0)
+    s = torch.cuda.current_stream()
+    if a.op == "accumulate":
+        X = llama_layer(8, a.d, a.tokens, seed=1, device=dev)[1]
+        H = torch.empty(a.d, a.d, device=dev)
+        run = lambda: kq.kronq_accumulate_factors(X, H, zero_first=True)  # noqa: E731
+        units = {"flops": a.tokens * a.d * (a.d + 1)}
+    else:
+        W, X, G = llama_layer(a.m, a.n, 2 * max(a.m, a.n), seed=1, device=dev)
+        lp = LayerPass(a.m, a.n, bits=a.bits, group=a.group, device=dev)
+        lp.accumulate(X, G)
+        if a.op == "biip":
+            HX0, HG0 = lp.HX.clone(), lp.HG.clone()
+
+            def run():
+                lp.HX.copy_(HX0)
+                lp.HG.copy_(HG0)
+                lp.transform(W)
+            units = {"bytes": 2 * (2 + 4) * a.m * a.n + 16 * a.n * a.n + 16 * a.m * a.m}
+        elif a.op == "quantize":
+            lp.transform(W)
+            HX0, W0 = lp.HX.clone(), lp.Wt.clone()
+
+            def run():
+                lp.HX.copy_(HX0)
+                lp.Wt.copy_(W0)
+                lp.quantize()
+            units = {"weights": a.m * a.n}
+        else:
+            codes = torch.randint(0, 2 ** a.bits, (a.m, a.n), dtype=torch.uint8, device=dev)
+            out = torch.empty(a.m, kq.words_per_row(a.n, a.bits), dtype=torch.int32, device=dev)
+            run = lambda: kq.kronq_pack(codes, a.bits, out)  # noqa: E731
+            units = {"bytes": a.m * a.n * (1 + a.bits / 8)}
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(a.reps):
+        run()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.reps
+    print(json.dumps({"op": a.op, "ms_per_call": ms, "args": vars(a), **units}))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

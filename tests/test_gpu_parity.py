@@ -37,7 +37,7 @@ def test_factor_bf16_tensor_core(T, d):
     torch.cuda.synchronize()
     ref = factors.factor(to_np(X))
     Hn = to_np(H)
-    assert rel(Hn, ref) < 1e-5
+    assert rel(Hn, ref) < 1e-4
     assert np.array_equal(Hn, Hn.T)
     assert kq.kronq_device_status() == 0
 
@@ -51,7 +51,7 @@ def test_factor_bf16_streamed_chunks_and_strided_view():
     for t0 in range(0, T, 1024):        # chunk starts stay 16-byte aligned
         kq.kronq_accumulate_factors(X[t0:t0 + 1024], H, zero_first=(t0 == 0))
     torch.cuda.synchronize()
-    assert rel(to_np(H), factors.factor(to_np(X))) < 1e-5
+    assert rel(to_np(H), factors.factor(to_np(X))) < 1e-4
 
 
 def test_factor_small_and_empty():
@@ -59,7 +59,7 @@ def test_factor_small_and_empty():
     H = torch.empty(96, 96, device=DEV)
     kq.kronq_accumulate_factors(X, H, zero_first=True)
     torch.cuda.synchronize()
-    assert rel(to_np(H), factors.factor(to_np(X))) < 1e-5
+    assert rel(to_np(H), factors.factor(to_np(X))) < 1e-4
     H.fill_(3.0)
     kq.kronq_accumulate_factors(X[:0], H, zero_first=True)   # T = 0
     torch.cuda.synchronize()
@@ -74,7 +74,7 @@ def test_factor_f32(T, d):
     kq.kronq_accumulate_factors(Xt, H, zero_first=True)
     kq.kronq_accumulate_factors(Xt, H, zero_first=False)
     torch.cuda.synchronize()
-    assert rel(to_np(H), 2 * factors.factor(X)) < 1e-5
+    assert rel(to_np(H), 2 * factors.factor(X)) < 1e-4
 
 
 def test_factor_max_dimension_sampled():
@@ -88,7 +88,7 @@ def test_factor_max_dimension_sampled():
     Xn = to_np(X)
     ref = factors.factor_columns(Xn, cols)
     got = to_np(H[:, torch.as_tensor(cols, device=DEV)])
-    assert rel(got, ref) < 1e-5
+    assert rel(got, ref) < 1e-4
     del H
 
 
@@ -193,7 +193,7 @@ def _sweep_inputs(m, n, seed):
     Wt, HXt, _, _, _ = biip.biip_forward(W, H, None, seed, 0.25, "sv_only")
     A, _ = sweep.damp(HXt, 0.01)
     U = sweep.chol_upper_of_inverse(A)
-    return Wt.astype(np.float32), U.astype(np.float32)
+    return np.ascontiguousarray(Wt, dtype=np.float32), np.ascontiguousarray(U, dtype=np.float32)
 
 
 @pytest.mark.parametrize("m,n,bits,group,asym", [
