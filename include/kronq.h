@@ -204,6 +204,29 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
                                   float* zeros, float* E, int* info, void* workspace,
                                   size_t ws_bytes, kronq_stream_t s);
 
+/* kronq_quantize_layer_static -- the same call for callers that cannot
+ * allocate device memory (no counterpart on the pages; the paper has none).
+ * Such callers hold only pointers handed to them by another runtime (a
+ * plugin inside a framework whose memory pool owns all device memory and
+ * exposes no allocator, or a foreign-language caller without a CUDA
+ * allocation binding), or run where cudaMalloc is not allowed because it
+ * synchronises the device.  Arguments as kronq_quantize_layer, minus the
+ * workspace: the scratch is a file-scope static device array of 32 MiB that
+ * every GPU loading the library holds until the process exits.
+ *   - Layers whose kronq_quantize_workspace_bytes(m, n, p) exceeds 32 MiB
+ *     (for example n = 4096 with m up to ~28000, or n up to ~5600 with small
+ *     m) are rejected with KRONQ_ERR_INVALID_ARG before anything runs.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents; nothing in it has to start at zero, but calls that overlap
+ *     on the GPU (two streams, two threads) race on it. */
+kronq_status kronq_quantize_layer_static(float* Wt, float* HX, int64_t m, int64_t n,
+                                         const kronq_quant_params* p, uint8_t* codes, float* scales,
+                                         float* zeros, float* E, int* info, kronq_stream_t s);
+
 /* ---------------------------------------------------------------------------
  * Step 5 -- packing.  KronQ README "Model zoo": W4/W2 as packed int4/int2,
  * W3 not bit-packable (bits == 3 -> KRONQ_ERR_INVALID_ARG).  Layout: per

@@ -18,6 +18,7 @@ __all__ = [
     "kronq_accumulate_factors", "kronq_sensitivity", "kronq_allocate_bits",
     "kronq_allocate_topn_types", "kronq_biip_workspace_bytes", "kronq_biip_forward",
     "kronq_biip_inverse", "kronq_quantize_workspace_bytes", "kronq_quantize_layer",
+    "kronq_quantize_layer_static",
     "kronq_pack", "kronq_unpack", "kronq_device_status", "kronq_kfac_loss_workspace_bytes",
     "kronq_kfac_loss", "kronq_launch_count", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
 ]
@@ -149,6 +150,20 @@ def kronq_quantize_layer(Wt, HX, params: QuantParams, codes, scales, zeros, info
     check(lib.kronq_quantize_layer(_ptr(Wt), _ptr(HX), m, n, ctypes.byref(params), _ptr(codes),
                                    _ptr(scales), _ptr(zeros), _ptr(E), _ptr(info), _ptr(ws),
                                    ws.numel(), _stream(stream)))
+
+
+def kronq_quantize_layer_static(Wt, HX, params: QuantParams, codes, scales, zeros, info, E=None,
+                                stream=None):
+    """kronq_quantize_layer without a workspace, for callers that cannot
+    allocate device memory: the scratch is the library's 32 MiB static device
+    array (shared by all calls on a device; overlapping calls race)."""
+    m, n = Wt.shape
+    for t, name in ((Wt, "Wt"), (HX, "HX"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
+                    (info, "info"), (E, "E")):
+        _rowmajor(t, name)
+    check(lib.kronq_quantize_layer_static(_ptr(Wt), _ptr(HX), m, n, ctypes.byref(params),
+                                          _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(E),
+                                          _ptr(info), _stream(stream)))
 
 
 def kronq_pack(codes, bits: int, out, stream=None):

@@ -53,6 +53,8 @@ SIGNATURES = {
     "kronq_quantize_workspace_bytes": (_sz, [_i64, _i64, _qp]),
     "kronq_quantize_layer": (_int, [_vp, _vp, _i64, _i64, _qp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                     _vp]),
+    "kronq_quantize_layer_static": (_int, [_vp, _vp, _i64, _i64, _qp, _vp, _vp, _vp, _vp, _vp,
+                                           _vp]),
     "kronq_pack": (_int, [_vp, _i64, _i64, _int, _vp, _vp]),
     "kronq_unpack": (_int, [_vp, _i64, _i64, _int, _vp, _vp]),
     "kronq_device_status": (_int, [_ip, _vp]),
