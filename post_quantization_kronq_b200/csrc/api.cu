@@ -92,11 +92,17 @@ size_t biip_ws(int64_t m, int64_t n) {
   return c.size();
 }
 
+int64_t quant_ldu(int64_t n) { return (n + 7) / 8 * 8; }
+
 size_t quant_ws(int64_t m, int64_t n) {
   Carver c(nullptr);
   c.take<uint8_t>(chol_workspace_bytes(n));
   c.take<uint8_t>((size_t)n);
   c.take<float>((size_t)(m * 128));
+  c.take<__nv_bfloat16>((size_t)(m * 128));
+  c.take<__nv_bfloat16>((size_t)(m * 128));
+  c.take<__nv_bfloat16>((size_t)(128 * quant_ldu(n)));
+  c.take<__nv_bfloat16>((size_t)(128 * quant_ldu(n)));
   return c.size();
 }
 
@@ -369,6 +375,10 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
   void* cws = c.take<uint8_t>(chol_workspace_bytes(n));
   uint8_t* dead = c.take<uint8_t>((size_t)n);
   float* Eblk = c.take<float>((size_t)(m * 128));
+  __nv_bfloat16* Eh = c.take<__nv_bfloat16>((size_t)(m * 128));
+  __nv_bfloat16* El = c.take<__nv_bfloat16>((size_t)(m * 128));
+  __nv_bfloat16* Uh = c.take<__nv_bfloat16>((size_t)(128 * quant_ldu(n)));
+  __nv_bfloat16* Ul = c.take<__nv_bfloat16>((size_t)(128 * quant_ldu(n)));
   const bool u_given = (p->flags & KRONQ_U_GIVEN) != 0;
   kronq_status r;
   if (u_given) {
@@ -387,6 +397,7 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
   d.dead = u_given ? nullptr : dead;
   d.info = info;
   d.ordered = (p->flags & KRONQ_ORDERED_FP32) != 0;
+  d.Eh = Eh; d.El = El; d.Uh = Uh; d.Ul = Ul; d.ldu = quant_ldu(n);
   return gptq_sweep(d, st);
 }
 
@@ -408,10 +419,12 @@ kronq_status kronq_unpack(const uint32_t* in, int64_t m, int64_t n, int bits, ui
 
 kronq_status kronq_device_status(int* out, kronq_stream_t s) {
   if (!out) return fail(KRONQ_ERR_INVALID_ARG, "device_status: out is NULL");
-  int v = 0;
+  int v = 0, w = 0, x = 0;
   cudaError_t e = status_fetch_syrk(&v, as_stream(s));
+  if (e == cudaSuccess) e = status_fetch_trailing(&w, as_stream(s));
+  if (e == cudaSuccess) e = status_fetch_schur(&x, as_stream(s));
   if (e != cudaSuccess) return cuda_fail(e, "device_status");
-  *out = v;
+  *out = v != 0 ? v : (w != 0 ? w : x);
   return KRONQ_OK;
 }
 

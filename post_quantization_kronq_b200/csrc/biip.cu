@@ -20,63 +20,73 @@
 namespace kq {
 namespace {
 
-constexpr int RP_THREADS = 256;
+constexpr int RP_THREADS = 512;
 constexpr int KREG = 16;     // odd factors up to this size are transformed in registers
 constexpr int KMAX = 255;    // largest odd factor supported
 
-__device__ __forceinline__ int64_t padx(int64_t x) { return x + (x >> 5); }
+__device__ __forceinline__ int padx(int x) { return x + (x >> 5); }
 
-__device__ __forceinline__ float sign_of(uint64_t state, int64_t j) {
+__device__ __forceinline__ float sign_of(uint64_t state, int j) {
   return (splitmix64(state, (uint64_t)j) >> 63) ? -1.f : 1.f;
 }
 
 struct RPArgs {
   RowPass p;
-  int R;        // rows per CTA
+  int R, logR;  // rows per CTA (a power of two)
   int P, K, logP;
-  int64_t RS;   // padded row stride in shared memory (floats)
+  int RS;       // padded row stride in shared memory (floats, odd)
   float norm;   // 1 / sqrt(P)
-  int two_buf;  // K > KREG: DCT writes to a second buffer
+  int two_buf;  // K > KREG: the DCT writes to a second buffer
 };
+
+// Per-column factor of the forward pre-scale or the inverse post-scale:
+// the sign of column j times d[j] (scale_mode 1) or 1/d[j] (scale_mode 2).
+__device__ __forceinline__ float col_factor(const RowPass& p, int j) {
+  float f = p.rotate ? sign_of(p.sign_state, j) : 1.f;
+  if (p.scale_mode == 1) f = f * p.scale[j];
+  else if (p.scale_mode == 2) f = f / p.scale[j];
+  return f;
+}
 
 __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
   extern __shared__ __align__(16) float sm[];
   const RowPass& p = A.p;
   const int R = A.R, P = A.P, K = A.K;
-  const int64_t L = p.L, RS = A.RS;
+  const int L = (int)p.L, RS = A.RS;
   float* buf0 = sm;
-  float* buf1 = sm + (int64_t)R * RS;
-  float* Cm = sm + (int64_t)R * RS * (A.two_buf ? 2 : 1);
+  float* buf1 = sm + R * RS;
+  float* Cm = sm + R * RS * (A.two_buf ? 2 : 1);
   const int64_t r0 = (int64_t)blockIdx.x * R;
+  const int rows_here = (int)((p.rows - r0) < R ? (p.rows - r0) : R);
   const int tid = threadIdx.x;
 
   if (p.rotate && K > 1) {
     for (int t = tid; t < K * K; t += RP_THREADS) {
-      const int i = t / K, j = t % K;
+      const int i = t / K, j = t - (t / K) * K;
       const double ci = (i == 0) ? sqrt(0.5) : 1.0;
       Cm[t] = (float)(sqrt(2.0 / K) * ci * cospi((double)((2 * j + 1) * i) / (2.0 * K)));
     }
   }
 
-  // 1. load (+ forward pre-scale and signs)
-  const int64_t tot = (int64_t)R * L;
-  for (int64_t t = tid; t < tot; t += RP_THREADS) {
-    const int rr = (int)(t / L);
-    const int64_t j = t - (int64_t)rr * L;
-    const int64_t r = r0 + rr;
-    float v = 0.f;
-    if (r < p.rows) {
-      if (p.in_bf16)
-        v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[r * p.ld_in + j]);
-      else
-        v = reinterpret_cast<const float*>(p.in)[r * p.ld_in + j];
-      if (!p.inverse) {
-        if (p.scale_mode == 1) v = v * p.scale[j];
-        else if (p.scale_mode == 2) v = v / p.scale[j];
-        if (p.rotate) v = v * sign_of(p.sign_state, j);
+  // 1. load rows (forward: times sign and scale of the column); the column
+  //    factor is computed once per column and reused for the R rows.
+  //    All R loads of a column are issued before any is used.
+  for (int j = tid; j < L; j += RP_THREADS) {
+    const float f = p.inverse ? 1.f : col_factor(p, j);
+    const int pj = padx(j);
+    float v[8];
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) {
+      v[rr] = 0.f;
+      if (rr < rows_here) {
+        const int64_t idx = (r0 + rr) * p.ld_in + j;
+        v[rr] = p.in_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[idx])
+                          : reinterpret_cast<const float*>(p.in)[idx];
       }
     }
-    buf0[rr * RS + padx(j)] = v;
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr)
+      if (rr < R) buf0[rr * RS + pj] = v[rr] * f;
   }
   __syncthreads();
 
@@ -84,12 +94,12 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
   if (p.rotate) {
     // 2. DCT along b (odd factor)
     if (K > 1) {
-      const int64_t items = (int64_t)R * P;
-      for (int64_t t = tid; t < items; t += RP_THREADS) {
-        const int rr = (int)(t / P);
-        const int a = (int)(t - (int64_t)rr * P);
+      const int items = R * P;
+      for (int t = tid; t < items; t += RP_THREADS) {
+        const int rr = t / P;
+        const int a = t - rr * P;
         float* row = buf0 + rr * RS;
-        const int64_t base = (int64_t)a * K;
+        const int base = a * K;
         if (!A.two_buf) {
           float y[KREG];
 #pragma unroll
@@ -117,26 +127,57 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
       if (A.two_buf) cur = buf1;
       __syncthreads();
     }
-    // 3. FWHT along a, radix-16 passes over bit groups of a
+    // 3. FWHT along a: radix-16 register passes over 4-bit groups of a.
+    //    Item order (b fastest, then the low bits of a, then the high bits)
+    //    keeps neighbouring threads on neighbouring shared-memory words.
     for (int lo = 0; lo < A.logP; lo += 4) {
       const int nb = (A.logP - lo) < 4 ? (A.logP - lo) : 4;
       const int G = 1 << nb;
-      const int64_t per_row = L >> nb;  // items per row
-      const int64_t items = (int64_t)R * per_row;
-      const int64_t lo_span = (int64_t)1 << lo;
-      for (int64_t t = tid; t < items; t += RP_THREADS) {
-        const int rr = (int)(t / per_row);
-        int64_t rem = t - (int64_t)rr * per_row;
-        const int b = (int)(rem % K);
-        rem /= K;
-        const int64_t a_lo = rem & (lo_span - 1);
-        const int64_t a_hi = rem >> lo;
-        const int64_t a0 = (a_hi << (lo + nb)) | a_lo;
+      const int per_row = L >> nb;
+      const int items = per_row << A.logR;
+      const int lo_mask = (1 << lo) - 1;
+      if (K == 1 && G == 16) {
+        // power-of-two length, full radix-16 pass: shifts and masks only
+        int lpr = 0;
+        while ((1 << lpr) < per_row) ++lpr;
+        for (int t = tid; t < items; t += RP_THREADS) {
+          const int rr = t >> lpr;
+          const int rem = t & (per_row - 1);
+          const int a0 = ((rem >> lo) << (lo + 4)) | (rem & lo_mask);
+          float* row = cur + rr * RS;
+          float x[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) x[u] = row[padx(a0 + (u << lo))];
+#pragma unroll
+          for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+              if ((u & h) == 0) {
+                const float s0 = x[u], s1 = x[u | h];
+                x[u] = s0 + s1;
+                x[u | h] = s0 - s1;
+              }
+#pragma unroll
+          for (int u = 0; u < 16; ++u) row[padx(a0 + (u << lo))] = x[u];
+        }
+        __syncthreads();
+        continue;
+      }
+      for (int t = tid; t < items; t += RP_THREADS) {
+        const int rr = t / per_row;
+        int rem = t - rr * per_row;
+        int b = 0;
+        if (K > 1) {
+          const int q = rem / K;
+          b = rem - q * K;
+          rem = q;
+        }
+        const int a0 = ((rem >> lo) << (lo + nb)) | (rem & lo_mask);
         float* row = cur + rr * RS;
         float x[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u)
-          if (u < G) x[u] = row[padx((a0 + ((int64_t)u << lo)) * K + b)];
+          if (u < G) x[u] = row[padx((a0 + (u << lo)) * K + b)];
 #pragma unroll
         for (int h = 1; h < 16; h <<= 1) {
           if (h < G) {
@@ -152,26 +193,27 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
         }
 #pragma unroll
         for (int u = 0; u < 16; ++u)
-          if (u < G) row[padx((a0 + ((int64_t)u << lo)) * K + b)] = x[u];
+          if (u < G) row[padx((a0 + (u << lo)) * K + b)] = x[u];
       }
       __syncthreads();
     }
   }
 
-  // 4. transposed store (+ normalisation, inverse post-scale and signs)
-  for (int64_t t = tid; t < tot; t += RP_THREADS) {
-    const int rr = (int)(t % R);
-    const int64_t j = t / R;
-    const int64_t r = r0 + rr;
-    if (r >= p.rows) continue;
-    float v = cur[rr * RS + padx(j)];
-    if (p.rotate) v = v * A.norm;
-    if (p.inverse) {
-      if (p.rotate) v = v * sign_of(p.sign_state, j);
-      if (p.scale_mode == 1) v = v * p.scale[j];
-      else if (p.scale_mode == 2) v = v / p.scale[j];
+  // 4. transposed store: consecutive threads take consecutive rows of one
+  //    column, so every warp writes R-float runs of the output rows.
+  const float nrm = p.rotate ? A.norm : 1.f;
+  const int tot = L << A.logR;
+  const int rr = tid & (R - 1);
+  const int jstep = RP_THREADS >> A.logR;
+  if (rr < rows_here) {
+    float* o = p.out + (int64_t)(tid >> A.logR) * p.ld_out + r0 + rr;
+    const int64_t ostep = (int64_t)jstep * p.ld_out;
+    const float* src = cur + rr * RS;
+    for (int t = tid, j = tid >> A.logR; t < tot; t += RP_THREADS, j += jstep, o += ostep) {
+      float v = src[padx(j)] * nrm;
+      if (p.inverse) v = v * col_factor(p, j);
+      *o = v;
     }
-    p.out[j * p.ld_out + r] = v;
   }
 }
 
@@ -252,6 +294,7 @@ __global__ void __launch_bounds__(1024) rescale_kernel(const float* H, int64_t l
 
 kronq_status rowpass(const RowPass& p, cudaStream_t s) {
   if (p.rows <= 0 || p.L <= 0) return KRONQ_OK;
+  if (p.L > (1 << 24)) return fail(KRONQ_ERR_UNSUPPORTED, "BiIP rotation: row too long");
   RPArgs A;
   A.p = p;
   int P = 1;
@@ -266,14 +309,17 @@ kronq_status rowpass(const RowPass& p, cudaStream_t s) {
   A.norm = (float)(1.0 / sqrt((double)P));
   A.two_buf = (p.rotate && K > KREG) ? 1 : 0;
   const int64_t base = p.L + (p.L >> 5);
-  A.RS = base | 1;
-  const int64_t bytes_per_row = A.RS * 4 * (A.two_buf ? 2 : 1);
+  A.RS = (int)(base | 1);
+  const int64_t bytes_per_row = (int64_t)A.RS * 4 * (A.two_buf ? 2 : 1);
   const int64_t cbytes = (p.rotate && K > 1) ? K * K * 4 : 0;
   const int64_t budget = 200 * 1024;
-  int64_t R = (budget - cbytes) / bytes_per_row;
-  if (R > 8) R = 8;
-  if (R < 1) return fail(KRONQ_ERR_UNSUPPORTED, "BiIP rotation: row does not fit in shared memory");
-  A.R = (int)R;
+  int R = 8;
+  while (R > 1 && R * bytes_per_row + cbytes > budget) R >>= 1;
+  if (R * bytes_per_row + cbytes > budget)
+    return fail(KRONQ_ERR_UNSUPPORTED, "BiIP rotation: row does not fit in shared memory");
+  A.R = R;
+  A.logR = 0;
+  while ((1 << A.logR) < R) ++A.logR;
   const int64_t smem = R * bytes_per_row + cbytes;
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(&rowpass_kernel), (int)smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rowpass)");

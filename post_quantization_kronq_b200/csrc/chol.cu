@@ -7,10 +7,12 @@
 // U = R^-1, since A^-1 = R^-T R^-1 = U^T U.  That is 2 n^3 / 3 flops in total.
 //
 // Blocked with nb = 64, bottom-right first.  For each diagonal block J:
-//   K_A  one CTA factors A_JJ = R_JJ R_JJ^T and writes U_JJ = R_JJ^-1 in place;
-//   K_B  R[0:j0, J] = A[0:j0, J] U_JJ^T                 (panel)
-//   K_C  A[0:j0, 0:j0] -= R[0:j0, J] R[0:j0, J]^T         (upper triangle only)
-// Then the off-diagonal blocks of U come from the recursive formula
+//   diag_panel_kernel  factor A_JJ = R_JJ R_JJ^T and solve R[0:j0, J] R_JJ^T
+//                      = A[0:j0, J] (every CTA factors the small block itself)
+//   schur_tc_kernel    A[0:j0, 0:j0] -= R[0:j0, J] R[0:j0, J]^T on the tensor
+//                      cores (upper triangle only, fp32-level split products)
+// Then every diagonal block is inverted at once (U_JJ = R_JJ^-1), and the
+// off-diagonal blocks of U come from the recursive formula
 //   inv([[R11, R12], [0, R22]]) = [[U11, -U11 R12 U22], [0, U22]]
 // evaluated level by level (block sizes nb, 2 nb, 4 nb, ...), each level one
 // batched pair of GEMMs.  A non-positive pivot stops the chain and records
@@ -55,101 +57,165 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* H, int64_t n, float d
 
 __global__ void zero_info_kernel(int* info) { *info = 0; }
 
-// Factor the nb x nb diagonal block at j0 (reverse order), then invert R_JJ.
-__global__ void __launch_bounds__(256) diag_kernel(float* H, int64_t n, int64_t j0, int nb,
-                                                   int* info) {
+// Factor the diagonal block A_JJ = R_JJ R_JJ^T (reverse order) in shared
+// memory and solve the panel rows above it, R[i, J] R_JJ^T = A[i, J].
+// Every CTA factors the (small) block itself, so no extra launch sits on the
+// sequential path; CTA 0 writes R_JJ back.  A short block (nb < 64) is padded
+// with the identity.  The panel rows are also written as bf16 hi/mid/lo
+// splits for the tensor-core Schur update.
+__global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, int64_t j0, int nb,
+                                                         int* info, __nv_bfloat16* splits) {
   if (*info != 0) return;
   __shared__ float a[NB][NB + 1];
-  __shared__ float u[NB][NB + 1];
-  __shared__ int bad;
+  __shared__ float rdiag[NB], rinv[NB];
   const int tid = threadIdx.x;
-  for (int t = tid; t < nb * nb; t += blockDim.x) {
-    const int r = t / nb, c = t % nb;
-    // upper triangle (symmetric storage may hold only it reliably)
-    a[r][c] = (r <= c) ? H[(j0 + r) * n + j0 + c] : H[(j0 + c) * n + j0 + r];
-    u[r][c] = 0.f;
+  const int tx = tid & 63, ty = tid >> 6;
+  {
+    float x[NB / 4];
+#pragma unroll
+    for (int sl = 0; sl < NB / 4; ++sl) {  // all sixteen loads in flight
+      const int r = 4 * sl + ty;
+      x[sl] = (r <= tx && tx < nb) ? H[(j0 + r) * n + j0 + tx] : 0.f;
+    }
+#pragma unroll
+    for (int sl = 0; sl < NB / 4; ++sl) {
+      const int r = 4 * sl + ty;
+      a[r][tx] = (tx < nb) ? x[sl] : (r == tx ? 1.f : 0.f);
+    }
   }
-  if (tid == 0) bad = 0;
-  __syncthreads();
-  for (int k = nb - 1; k >= 0; --k) {
+  // One barrier per pivot: the update of column c < k uses
+  // r_ik r_ck = a_ik a_ck / pivot, so column k itself is left unscaled until
+  // the end (it is never written again once its pivot is done).
+  for (int k = NB - 1; k >= 0; --k) {
+    __syncthreads();
     const float piv = a[k][k];
     if (!(piv > 0.f) || !isfinite(piv)) {
-      if (tid == 0) {
-        *info = (int)(j0 + k + 1);
-        bad = 1;
+      if (tid == 0 && blockIdx.x == 0) *info = (int)(j0 + k + 1);
+      return;  // uniform: every thread read the same pivot
+    }
+    if (tid == 0) {
+      const float rk = sqrtf(piv);
+      rdiag[k] = rk;
+      rinv[k] = 1.f / rk;
+    }
+    if (tx < k) {
+      // all loads first: stores to column tx cannot be proven not to alias
+      // column k, so interleaving would serialise the sixteen updates
+      const float act = a[tx][k] * (1.f / piv);
+      float ck[NB / 4], ct[NB / 4];
+#pragma unroll
+      for (int sl = 0; sl < NB / 4; ++sl) {
+        ck[sl] = a[4 * sl + ty][k];
+        ct[sl] = a[4 * sl + ty][tx];
       }
-      __syncthreads();
-      return;
-    }
-    const float rk = sqrtf(piv);
-    __syncthreads();
-    for (int i = tid; i < k; i += blockDim.x) a[i][k] = a[i][k] / rk;
-    if (tid == 0) a[k][k] = rk;
-    __syncthreads();
-    // Schur complement on the leading k x k upper triangle
-    for (int t = tid; t < k * k; t += blockDim.x) {
-      const int i = t / k, j = t % k;
-      if (i <= j) a[i][j] = a[i][j] - a[i][k] * a[j][k];
-    }
-    __syncthreads();
-  }
-  // U_JJ = R_JJ^-1, column c by back substitution (one thread per column)
-  if (tid < nb) {
-    const int c = tid;
-    u[c][c] = 1.f / a[c][c];
-    for (int i = c - 1; i >= 0; --i) {
-      float acc = 0.f;
-      for (int k = i + 1; k <= c; ++k) acc = fmaf(a[i][k], u[k][c], acc);
-      u[i][c] = -acc / a[i][i];
+#pragma unroll
+      for (int sl = 0; sl < NB / 4; ++sl) {
+        const int i = 4 * sl + ty;
+        if (i <= tx) a[i][tx] = ct[sl] - ck[sl] * act;
+      }
     }
   }
   __syncthreads();
-  for (int t = tid; t < nb * nb; t += blockDim.x) {
-    const int r = t / nb, c = t % nb;
-    H[(j0 + r) * n + j0 + c] = (r <= c) ? u[r][c] : 0.f;
+  // scale every column k of R above the diagonal by 1 / r_kk
+#pragma unroll
+  for (int sl = 0; sl < NB / 4; ++sl) {
+    const int i = 4 * sl + ty;
+    if (i < tx) a[i][tx] *= rinv[tx];
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int t = tid; t < nb * NB; t += blockDim.x) {
+      const int r = t >> 6, c = t & 63;
+      if (c < nb) H[(j0 + r) * n + j0 + c] = (r < c) ? a[r][c] : (r == c ? rdiag[r] : 0.f);
+    }
+  }
+  // Panel rows: x R_JJ^T = a, back substitution from the last column; one
+  // warp per row, lane l holds columns l and l + 32.
+  const int warp = tid >> 5, lane = tid & 31;
+  const int64_t plane = (int64_t)n * NB;
+  for (int64_t i = (int64_t)blockIdx.x * 8 + warp; i < j0; i += (int64_t)gridDim.x * 8) {
+    float* row = H + i * n + j0;
+    float acc0 = (lane < nb) ? row[lane] : 0.f;
+    float acc1 = (lane + 32 < nb) ? row[lane + 32] : 0.f;
+    float x0 = 0.f, x1 = 0.f;
+    for (int k = NB - 1; k >= 0; --k) {
+      const bool upper_half = k >= 32;
+      const int owner = k & 31;
+      float xk = (upper_half ? acc1 : acc0) * rinv[k];
+      xk = __shfl_sync(0xffffffffu, xk, owner);
+      if (lane == owner) {
+        if (upper_half) x1 = xk;
+        else x0 = xk;
+      }
+      if (lane < k) acc0 -= a[lane][k] * xk;
+      if (lane + 32 < k) acc1 -= a[lane + 32][k] * xk;
+    }
+    if (lane < nb) row[lane] = x0;
+    if (lane + 32 < nb) row[lane + 32] = x1;
+    const float xs[2] = {x0, x1};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float x = xs[h];
+      const __nv_bfloat16 bh = __float2bfloat16_rn(x);
+      const float r1 = x - __bfloat162float(bh);
+      const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 bl = __float2bfloat16_rn(r1 - __bfloat162float(bm));
+      const int64_t o = i * NB + lane + 32 * h;
+      splits[o] = bh;
+      splits[plane + o] = bm;
+      splits[2 * plane + o] = bl;
+    }
   }
 }
 
-// R[0:j0, J] = A[0:j0, J] * U_JJ^T, rows in place.  One warp per row.
-__global__ void __launch_bounds__(256) panel_kernel(float* H, int64_t n, int64_t j0, int nb,
-                                                    const int* info) {
+// U_JJ = R_JJ^-1 for every diagonal block at once (one CTA per block).
+// Entry (i, i + dd) depends only on entries of smaller distance dd, so the
+// diagonals are computed one after the other, four adjacent lanes per entry.
+__global__ void __launch_bounds__(256) diag_inverse_kernel(float* H, int64_t n, const int* info) {
   if (*info != 0) return;
+  __shared__ float a[NB][NB + 1];
   __shared__ float u[NB][NB + 1];
-  __shared__ float rowbuf[8][NB];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int t = tid; t < nb * nb; t += blockDim.x) {
-    const int r = t / nb, c = t % nb;
-    u[r][c] = (r <= c) ? H[(j0 + r) * n + j0 + c] : 0.f;
+  __shared__ float rinv[NB];
+  const int64_t j0 = (int64_t)blockIdx.x * NB;
+  const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
+  const int tid = threadIdx.x;
+  for (int t = tid; t < NB * NB; t += blockDim.x) {
+    const int r = t >> 6, c = t & 63;
+    float x = 0.f;
+    if (r <= c) x = (c < nb) ? H[(j0 + r) * n + j0 + c] : (r == c ? 1.f : 0.f);
+    a[r][c] = x;
+    u[r][c] = 0.f;
   }
   __syncthreads();
-  for (int64_t i = (int64_t)blockIdx.x * 8 + warp; i < j0; i += (int64_t)gridDim.x * 8) {
-    float* row = H + i * n + j0;
-    for (int k = lane; k < nb; k += 32) rowbuf[warp][k] = row[k];
-    __syncwarp();
-    float out[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = lane + 32 * h;
-      float acc = 0.f;
-      if (c < nb)
-        for (int k = c; k < nb; ++k) acc = fmaf(rowbuf[warp][k], u[c][k], acc);
-      out[h] = acc;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = lane + 32 * h;
-      if (c < nb) row[c] = out[h];
-    }
-    __syncwarp();
+  if (tid < NB) rinv[tid] = 1.f / a[tid][tid];
+  __syncthreads();
+  const int ii = tid >> 2, part = tid & 3;
+  if (part == 0) u[ii][ii] = rinv[ii];
+  __syncthreads();
+  for (int dd = 1; dd < NB; ++dd) {
+    const int jj = ii + dd;
+    float acc = 0.f;
+    if (jj < NB)
+      for (int k = ii + 1 + part; k <= jj; k += 4) acc = fmaf(a[ii][k], u[k][jj], acc);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (jj < NB && part == 0) u[ii][jj] = -acc * rinv[ii];
+    __syncthreads();
+  }
+  for (int t = tid; t < nb * NB; t += blockDim.x) {
+    const int r = t >> 6, c = t & 63;
+    if (c < nb) H[(j0 + r) * n + j0 + c] = (r <= c) ? u[r][c] : 0.f;
   }
 }
 
 }  // namespace
 
 size_t chol_workspace_bytes(int64_t n) {
-  // recursive inverse: products T of the pairs of one level, at most n*n/4
-  return (size_t)((n * n) / 4 + n + 64) * sizeof(float);
+  // recursive inverse: products T of the pairs of one level (at most n*n/4
+  // floats); bf16 hi/mid/lo splits of the current panel (3 x n x 64)
+  const size_t tbytes = (size_t)((n * n) / 4 + n + 64) * sizeof(float);
+  const size_t sbytes = (size_t)3 * n * NB * sizeof(__nv_bfloat16);
+  return ((tbytes + 255) & ~size_t(255)) + sbytes;
 }
 
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
@@ -161,29 +227,33 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
     zero_info_kernel<<<1, 1, 0, s>>>(info);
     KQ_LAUNCH_CHECK("zero_info_kernel");
   }
+  if (n <= 0) return KRONQ_OK;
+  const size_t tbytes = (size_t)((n * n) / 4 + n + 64) * sizeof(float);
+  __nv_bfloat16* splits = reinterpret_cast<__nv_bfloat16*>(
+      static_cast<uint8_t*>(ws) + ((tbytes + 255) & ~size_t(255)));
+  SchurMaps maps;
+  if (n > NB) {
+    kronq_status r = schur_maps(&maps, splits, H, n);
+    if (r != KRONQ_OK) return r;
+  }
   // Blocks are aligned from the top (0, NB, 2 NB, ...); the last may be short.
   const int64_t nblk = ceil_div(n, NB);
+  const int64_t pmax = sm_count();
   for (int64_t bj = nblk - 1; bj >= 0; --bj) {
     const int64_t j0 = bj * NB;
     const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
-    diag_kernel<<<1, 256, 0, s>>>(H, n, j0, nb, info);
-    KQ_LAUNCH_CHECK("diag_kernel");
+    // One CTA per SM at most (each CTA factors the block itself), at least
+    // four panel rows per warp.
+    int64_t pg = j0 > 0 ? ceil_div(j0, 32) : 1;
+    if (pg > pmax) pg = pmax;
+    diag_panel_kernel<<<(unsigned)pg, 256, 0, s>>>(H, n, j0, nb, info, splits);
+    KQ_LAUNCH_CHECK("diag_panel_kernel");
     if (j0 == 0) break;
-    int64_t pg = ceil_div(j0, 8);
-    if (pg > 148 * 16) pg = 148 * 16;
-    panel_kernel<<<(unsigned)pg, 256, 0, s>>>(H, n, j0, nb, info);
-    KQ_LAUNCH_CHECK("panel_kernel");
-    GemmDesc g;
-    g.M = j0; g.N = j0; g.K = nb;
-    g.A = H + j0; g.lda = n; g.transA = false;
-    g.B = H + j0; g.ldb = n; g.transB = true;
-    g.C = H; g.ldc = n;
-    g.alpha = -1.f; g.beta = 1.f;
-    g.c_mode = 1;
-    g.info = info;
-    cudaError_t e = gemm_f32(g, s);
-    if (e != cudaSuccess) return cuda_fail(e, "gemm(schur)");
+    kronq_status r = schur_update_tc(&maps, H, n, j0, info, s);
+    if (r != KRONQ_OK) return r;
   }
+  diag_inverse_kernel<<<(unsigned)nblk, 256, 0, s>>>(H, n, info);
+  KQ_LAUNCH_CHECK("diag_inverse_kernel");
   // Recursive inverse of the off-diagonal blocks.
   float* Tbuf = reinterpret_cast<float*>(ws);
   for (int64_t S = NB; S < n; S *= 2) {

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include "../../include/kronq.h"
@@ -74,6 +75,16 @@ kronq_status rescale_vector(const float* H, int64_t ldh, const float* nrm, int64
                             float* d, cudaStream_t s);
 
 // ------------------------------------------------------------ factorisation
+// TMA descriptors of the tensor-core Schur update (the three panel splits,
+// 128-row boxes, and the fp32 matrix in 32-column boxes).
+struct alignas(64) SchurMaps {
+  unsigned char raw[4 * 128];
+  int tma_c = 0;   // tile of A staged by TMA (needs a 16-byte row stride)
+};
+kronq_status schur_maps(SchurMaps* sm, const __nv_bfloat16* splits, float* H, int64_t n);
+kronq_status schur_update_tc(const SchurMaps* sm, float* H, int64_t n, int64_t j0, const int* info,
+                             cudaStream_t s);
+cudaError_t status_fetch_schur(int* out, cudaStream_t s);
 // In: H (n x n) full symmetric.  Out: U (upper) with U^T U = (H + lambda I)^-1,
 // dead-column flags, info.  ws: see chol_workspace_bytes.
 size_t chol_workspace_bytes(int64_t n);
@@ -81,6 +92,18 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
                                 uint8_t* dead, int* info, void* ws, cudaStream_t s);
 
 // ------------------------------------------------------------ sweep
+// Storage for the four TMA descriptors of the tensor-core trailing update
+// (E hi/lo, U-block hi/lo); filled by trailing_maps on the host.
+struct alignas(64) TrailingMaps {
+  unsigned char raw[5 * 128];
+  int tma_c = 0;   // W tile staged by TMA (needs a 16-byte row stride)
+};
+kronq_status trailing_maps(TrailingMaps* tm, const void* Eh, const void* El, int64_t m,
+                           const void* Uh, const void* Ul, int64_t ldu, float* W, int64_t n);
+kronq_status trailing_update_tc(const TrailingMaps* tm, float* W, int64_t m, int64_t n, int64_t j1,
+                                int bw, const int* info, cudaStream_t s);
+cudaError_t status_fetch_trailing(int* out, cudaStream_t s);
+
 struct SweepDesc {
   float* W = nullptr;  // m x n, row stride n
   const float* U = nullptr;  // n x n upper
@@ -96,6 +119,14 @@ struct SweepDesc {
   const uint8_t* dead = nullptr;
   const int* info = nullptr;
   bool ordered = false;
+  // tensor-core trailing update (used unless ordered): bf16 hi/lo splits of
+  // the block's scaled errors (m x 128) and of the block's rows of U
+  // (128 x ldu), rewritten for every block.
+  __nv_bfloat16* Eh = nullptr;
+  __nv_bfloat16* El = nullptr;
+  __nv_bfloat16* Uh = nullptr;
+  __nv_bfloat16* Ul = nullptr;
+  int64_t ldu = 0;
 };
 kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s);
 

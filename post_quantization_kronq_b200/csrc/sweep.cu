@@ -20,16 +20,19 @@ namespace kq {
 namespace {
 
 constexpr int BW = 128;        // block width (columns)
-constexpr int RPW = 2;         // rows per warp
+constexpr int QW = 16;         // columns held by one lane
+constexpr int LPR = BW / QW;   // lanes per row (8)
 constexpr int WARPS = 8;       // warps per CTA
-constexpr int ROWS_PER_CTA = RPW * WARPS;
+constexpr int ROWS_PER_CTA = WARPS * 32 / LPR;   // 32
+constexpr int US_LD = BW + 4 * (BW / QW);        // padded row of the U block (160 floats)
+constexpr int SWEEP_SMEM = BW * US_LD * sizeof(float);
 
 struct BlockArgs {
   SweepDesc d;
   int64_t j0;
   int bw;         // columns in this block
   int wide;       // 1: the grid of this block's first column was computed beforehand
-  float* Eb;      // scaled-error output of this block
+  float* Eb;      // scaled-error output of this block (fp32) or nullptr
   int64_t lde;
 };
 
@@ -49,121 +52,225 @@ __device__ __forceinline__ void grid_from_range(float lo, float hi, int bits, bo
   zero = asym ? rintf(__fdiv_rn(-xmin, scale)) : (float)(1 << (bits - 1));
 }
 
+// Grid of the group starting at column j of this block: the eight lanes of
+// the row reduce over their columns in [j, j + group).
+__device__ __forceinline__ void group_start(const float (&v)[QW], int j, int bw, int q,
+                                            const SweepDesc& d, bool live, int64_t r, int64_t gi,
+                                            float& sc, float& zp) {
+  const int gend = (j + d.group < bw) ? j + d.group : bw;
+  float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+  for (int cc = 0; cc < QW; ++cc) {
+    const int col = q * QW + cc;
+    if (col >= j && col < gend) {
+      lo = fminf(lo, v[cc]);
+      hi = fmaxf(hi, v[cc]);
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < LPR; o <<= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  grid_from_range(lo, hi, d.bits, d.asym, sc, zp);
+  if (q == 0 && live) {
+    d.scales[r * d.ngroups + gi] = sc;
+    d.zeros[r * d.ngroups + gi] = zp;
+  }
+}
+
+// Column c of the block lives at Us[k * US_LD + ucol(c)]: 4 floats of padding
+// per 16 columns put the eight lanes of a row on different banks for the
+// float4 reads of one U row.
+__device__ __forceinline__ int ucol(int c) { return c + 4 * (c >> 4); }
+
+// One block of 128 columns.  Eight lanes per row: lane q holds the row's
+// columns 16q .. 16q+15 in registers (v[]), so every step of the sequential
+// column loop is register arithmetic with static indices (the unrolled
+// 16-step body stays small enough for the instruction cache).  At column j
+// the lane holding it quantizes, forms e = (w - deq) / U_jj and shuffles e
+// to the other seven lanes of the row; every lane then applies
+// v[c] -= e * U[j][c] to its columns c > j (multiply, then subtract: the
+// operation order of the float32 reference).
+template <bool SMALLG>
 __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
   const SweepDesc& d = a.d;
   if (d.info && *d.info != 0) return;
-  extern __shared__ __align__(16) float us_raw[];
-  float (*Us)[BW] = reinterpret_cast<float (*)[BW]>(us_raw);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  extern __shared__ __align__(16) float Us[];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int q = lane & (LPR - 1);
   const int64_t n = d.n, j0 = a.j0;
   const int bw = a.bw;
+  const int64_t r = (int64_t)blockIdx.x * ROWS_PER_CTA + (tid >> 3);
+  const bool live = r < d.m;
 
-  for (int t = tid; t < BW * BW; t += blockDim.x) {
-    const int r = t / BW, c = t % BW;
-    Us[r][c] = (r < bw && c < bw && c >= r) ? d.U[(j0 + r) * n + j0 + c] : 0.f;
+  // U block (rows j0.., columns j0..j0+127, upper part) into shared memory.
+  // float4 loads, eight in flight per thread.
+  const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(d.U) & 15) == 0);
+  if (vec) {
+#pragma unroll 8
+    for (int it = 0; it < (BW * BW / 4) / (WARPS * 32); ++it) {
+      const int idx = it * (WARPS * 32) + tid;
+      const int k = idx >> 5, c = (idx & 31) * 4;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k < bw) x = *reinterpret_cast<const float4*>(d.U + (j0 + k) * n + j0 + c);
+      x.x = (c + 0 >= k && c + 0 < bw) ? x.x : 0.f;
+      x.y = (c + 1 >= k && c + 1 < bw) ? x.y : 0.f;
+      x.z = (c + 2 >= k && c + 2 < bw) ? x.z : 0.f;
+      x.w = (c + 3 >= k && c + 3 < bw) ? x.w : 0.f;
+      *reinterpret_cast<float4*>(Us + k * US_LD + ucol(c)) = x;
+    }
+  } else {
+    for (int t = tid; t < BW * BW; t += blockDim.x) {
+      const int k = t >> 7, c = t & (BW - 1);
+      Us[k * US_LD + ucol(c)] = (k < bw && c < bw && c >= k) ? d.U[(j0 + k) * n + j0 + c] : 0.f;
+    }
+  }
+
+  // bf16 hi/lo copy of this block's rows of U, columns j1.. (operand B of
+  // the tensor-core trailing update); rows are spread over the CTAs.
+  const int64_t j1 = j0 + bw;
+  if (!d.ordered && j1 < n) {
+    for (int64_t k = blockIdx.x; k < bw; k += gridDim.x) {
+      const float* src = d.U + (j0 + k) * n;
+      __nv_bfloat16* dh = d.Uh + k * d.ldu;
+      __nv_bfloat16* dl = d.Ul + k * d.ldu;
+      if (vec) {
+#pragma unroll 4
+        for (int64_t c = j1 + 4 * tid; c < n; c += 4 * blockDim.x) {
+          const float4 x = *reinterpret_cast<const float4*>(src + c);
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(x.x), h1 = __float2bfloat16_rn(x.y);
+          const __nv_bfloat16 h2 = __float2bfloat16_rn(x.z), h3 = __float2bfloat16_rn(x.w);
+          __nv_bfloat162 hh[2] = {__halves2bfloat162(h0, h1), __halves2bfloat162(h2, h3)};
+          __nv_bfloat162 ll[2] = {
+              __halves2bfloat162(__float2bfloat16_rn(x.x - __bfloat162float(h0)),
+                                 __float2bfloat16_rn(x.y - __bfloat162float(h1))),
+              __halves2bfloat162(__float2bfloat16_rn(x.z - __bfloat162float(h2)),
+                                 __float2bfloat16_rn(x.w - __bfloat162float(h3)))};
+          *reinterpret_cast<uint2*>(dh + c) = *reinterpret_cast<uint2*>(hh);
+          *reinterpret_cast<uint2*>(dl + c) = *reinterpret_cast<uint2*>(ll);
+        }
+      } else {
+        for (int64_t c = j1 + tid; c < n; c += blockDim.x) {
+          const float x = src[c];
+          const __nv_bfloat16 h = __float2bfloat16_rn(x);
+          dh[c] = h;
+          dl[c] = __float2bfloat16_rn(x - __bfloat162float(h));
+        }
+      }
+    }
+  }
+
+  float v[QW], ev[QW];
+  uint32_t code[QW / 4];
+  const float* wrow = d.W + r * n + j0 + q * QW;
+  if (live && q * QW + QW <= bw && vec) {
+#pragma unroll
+    for (int c = 0; c < QW; c += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(wrow + c);
+      v[c] = x.x; v[c + 1] = x.y; v[c + 2] = x.z; v[c + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < QW; ++c) v[c] = (live && q * QW + c < bw) ? wrow[c] : 0.f;
+  }
+#pragma unroll
+  for (int c = 0; c < QW; ++c) {
+    if (d.dead && live && q * QW + c < bw && d.dead[j0 + q * QW + c]) v[c] = 0.f;
+    ev[c] = 0.f;
+  }
+#pragma unroll
+  for (int c = 0; c < QW / 4; ++c) code[c] = 0;
+  float sc = 1.f, zp = 0.f;
+  if (a.wide && live) {
+    const int64_t gi = (d.group == -1) ? 0 : j0 / d.group;
+    sc = d.scales[r * d.ngroups + gi];
+    zp = d.zeros[r * d.ngroups + gi];
   }
   __syncthreads();
 
   const float maxq = (float)((1 << d.bits) - 1);
-  const int64_t rbase = ((int64_t)blockIdx.x * WARPS + warp) * RPW;
-
-  float v[RPW][4], ev[RPW][4];
-  uint32_t code[RPW];
-  float sc[RPW], zp[RPW];
+  const int src_base = lane & ~(LPR - 1);
+  // In-block groups divide 128, so they are powers of two starting at j0.
+  const bool inblock_groups = d.group > 0 && d.group <= BW;
+  const int gmask = inblock_groups ? d.group - 1 : 0;
+  int gshift = 0;
+  while (inblock_groups && (1 << gshift) < d.group) ++gshift;
+  const int64_t g0 = inblock_groups ? j0 >> gshift : 0;
+  for (int qo = 0; qo < LPR; ++qo) {
+    const bool all_later = q > qo;     // every column of this lane comes after the current quarter
+    const bool mine = q == qo;
+    // Groups of 16 or more columns can only start at a lane boundary.
+    if (!SMALLG && inblock_groups && qo * QW < bw && ((qo * QW) & gmask) == 0)
+      group_start(v, qo * QW, bw, q, d, live, r, g0 + ((qo * QW) >> gshift), sc, zp);
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int64_t r = rbase + rr;
-    code[rr] = 0;
-    sc[rr] = 1.f;
-    zp[rr] = 0.f;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int c = 4 * lane + s;
-      float x = 0.f;
-      if (r < d.m && c < bw) {
-        x = d.W[r * n + j0 + c];
-        if (d.dead && d.dead[j0 + c]) x = 0.f;
-      }
-      v[rr][s] = x;
-      ev[rr][s] = 0.f;
-    }
-    if (a.wide && r < d.m) {
-      const int64_t gi = (d.group == -1) ? 0 : j0 / d.group;
-      sc[rr] = d.scales[r * d.ngroups + gi];
-      zp[rr] = d.zeros[r * d.ngroups + gi];
-    }
-  }
-
-  for (int j = 0; j < bw; ++j) {
-    const int64_t gc = j0 + j;
-    if (d.group > 0 && d.group <= BW && (gc % d.group) == 0) {
-      const int gend = (j + d.group < bw) ? j + d.group : bw;
-#pragma unroll
-      for (int rr = 0; rr < RPW; ++rr) {
-        float lo = INFINITY, hi = -INFINITY;
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const int c = 4 * lane + s;
-          if (c >= j && c < gend) {
-            lo = fminf(lo, v[rr][s]);
-            hi = fmaxf(hi, v[rr][s]);
-          }
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-          hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        }
-        grid_from_range(lo, hi, d.bits, d.asym, sc[rr], zp[rr]);
-        const int64_t r = rbase + rr;
-        if (lane == 0 && r < d.m) {
-          d.scales[r * d.ngroups + gc / d.group] = sc[rr];
-          d.zeros[r * d.ngroups + gc / d.group] = zp[rr];
-        }
-      }
-    }
-    const int owner = j >> 2, slot = j & 3;
-    const float ujj = Us[j][j];
-#pragma unroll
-    for (int rr = 0; rr < RPW; ++rr) {
+    for (int c = 0; c < QW; ++c) {
+      const int j = qo * QW + c;
+      if (j >= bw) break;
+      if (SMALLG && (j & gmask) == 0) group_start(v, j, bw, q, d, live, r, g0 + (j >> gshift), sc, zp);
       float e = 0.f;
-      if (lane == owner) {
-        float w = v[rr][0];
-#pragma unroll
-        for (int s = 1; s < 4; ++s)
-          if (s == slot) w = v[rr][s];
-        float q = __fadd_rn(rintf(__fdiv_rn(w, sc[rr])), zp[rr]);
-        q = fminf(fmaxf(q, 0.f), maxq);
-        const float deq = __fmul_rn(sc[rr], __fsub_rn(q, zp[rr]));
-        e = __fdiv_rn(__fsub_rn(w, deq), ujj);
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-          if (s == slot) {
-            v[rr][s] = deq;
-            ev[rr][s] = e;
-          }
-        code[rr] |= ((uint32_t)q & 0xFFu) << (8 * slot);
+      if (mine) {
+        const float w = v[c];
+        float qv = __fadd_rn(rintf(__fdiv_rn(w, sc)), zp);
+        qv = fminf(fmaxf(qv, 0.f), maxq);
+        const float deq = __fmul_rn(sc, __fsub_rn(qv, zp));
+        e = __fdiv_rn(__fsub_rn(w, deq), Us[j * US_LD + ucol(j)]);
+        v[c] = deq;
+        ev[c] = e;
+        code[c >> 2] |= ((uint32_t)qv & 0xFFu) << (8 * (c & 3));
       }
-      e = __shfl_sync(0xffffffffu, e, owner);
-      const float4 u4 = *reinterpret_cast<const float4*>(&Us[j][4 * lane]);
-      const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+      e = __shfl_sync(0xffffffffu, e, src_base + qo);
+      const float* urow = Us + j * US_LD + q * (QW + 4);
 #pragma unroll
-      for (int s = 0; s < 4; ++s)
-        if (4 * lane + s > j) v[rr][s] = __fsub_rn(v[rr][s], __fmul_rn(e, uu[s]));
+      for (int c4 = 0; c4 < QW; c4 += 4) {
+        const float4 u4 = *reinterpret_cast<const float4*>(urow + c4);
+        const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int cc = c4 + t;
+          if (all_later || (mine && cc > c)) v[cc] = __fsub_rn(v[cc], __fmul_rn(e, uu[t]));
+        }
+      }
     }
   }
 
+  if (!live) return;
+  const int64_t base = r * n + j0 + q * QW;
+  const bool full = (q * QW + QW <= bw);
+  if (full && ((reinterpret_cast<uintptr_t>(d.W + base) & 15) == 0)) {
+    float4* w4 = reinterpret_cast<float4*>(d.W + base);
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int64_t r = rbase + rr;
-    if (r >= d.m) continue;
+    for (int c = 0; c < QW; c += 4) w4[c >> 2] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+  } else {
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int c = 4 * lane + s;
-      if (c < bw) {
-        d.W[r * n + j0 + c] = v[rr][s];
-        d.codes[r * n + j0 + c] = (uint8_t)((code[rr] >> (8 * s)) & 0xFFu);
-        a.Eb[r * a.lde + c] = ev[rr][s];
-      }
+    for (int c = 0; c < QW; ++c)
+      if (q * QW + c < bw) d.W[base + c] = v[c];
+  }
+  if (full && ((reinterpret_cast<uintptr_t>(d.codes + base) & 15) == 0)) {
+    uint4* c4 = reinterpret_cast<uint4*>(d.codes + base);
+#pragma unroll
+    for (int t = 0; t < QW / 16; ++t)
+      c4[t] = make_uint4(code[4 * t], code[4 * t + 1], code[4 * t + 2], code[4 * t + 3]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < QW; ++c)
+      if (q * QW + c < bw) d.codes[base + c] = (uint8_t)((code[c >> 2] >> (8 * (c & 3))) & 0xFFu);
+  }
+  if (a.Eb) {
+#pragma unroll
+    for (int c = 0; c < QW; ++c)
+      if (q * QW + c < bw) a.Eb[r * a.lde + q * QW + c] = ev[c];
+  }
+  if (!d.ordered) {
+    __nv_bfloat16* eh = d.Eh + r * BW + q * QW;
+    __nv_bfloat16* el = d.El + r * BW + q * QW;
+#pragma unroll
+    for (int c = 0; c < QW; c += 2) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(ev[c]), h1 = __float2bfloat16_rn(ev[c + 1]);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(ev[c] - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(ev[c + 1] - __bfloat162float(h1));
+      *reinterpret_cast<__nv_bfloat162*>(eh + c) = __halves2bfloat162(h0, h1);
+      *reinterpret_cast<__nv_bfloat162*>(el + c) = __halves2bfloat162(l0, l1);
     }
   }
 }
@@ -199,10 +306,15 @@ __global__ void group_params_kernel(SweepDesc d, int64_t j0, int64_t gw, int64_t
 
 kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
   const int64_t n = d.n, m = d.m;
-  constexpr int SWEEP_SMEM = BW * BW * sizeof(float);
-  cudaError_t ea = allow_smem(reinterpret_cast<const void*>(&sweep_block_kernel), SWEEP_SMEM);
+  cudaError_t ea = allow_smem(reinterpret_cast<const void*>(&sweep_block_kernel<false>), SWEEP_SMEM);
+  if (ea == cudaSuccess) ea = allow_smem(reinterpret_cast<const void*>(&sweep_block_kernel<true>), SWEEP_SMEM);
   if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(sweep)");
   const unsigned grid = (unsigned)ceil_div(m, ROWS_PER_CTA);
+  TrailingMaps maps;
+  if (!d.ordered && n > BW) {
+    kronq_status r = trailing_maps(&maps, d.Eh, d.El, m, d.Uh, d.Ul, d.ldu, d.W, n);
+    if (r != KRONQ_OK) return r;
+  }
   for (int64_t j0 = 0; j0 < n; j0 += BW) {
     const int bw = (int)((j0 + BW <= n) ? BW : n - j0);
     BlockArgs a;
@@ -223,14 +335,23 @@ kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
     if (d.E) {
       a.Eb = d.E + j0;
       a.lde = n;
-    } else {
+    } else if (d.ordered) {
       a.Eb = d.Eblk;
       a.lde = BW;
+    } else {
+      a.Eb = nullptr;   // the tensor-core update reads the bf16 hi/lo copies
+      a.lde = BW;
     }
-    sweep_block_kernel<<<grid, WARPS * 32, SWEEP_SMEM, s>>>(a);
+    if (d.group > 0 && d.group < QW)
+      sweep_block_kernel<true><<<grid, WARPS * 32, SWEEP_SMEM, s>>>(a);
+    else
+      sweep_block_kernel<false><<<grid, WARPS * 32, SWEEP_SMEM, s>>>(a);
     KQ_LAUNCH_CHECK("sweep_block_kernel");
     const int64_t j1 = j0 + bw;
-    if (j1 < n) {
+    if (j1 < n && !d.ordered) {
+      kronq_status r = trailing_update_tc(&maps, d.W, m, n, j1, bw, d.info, s);
+      if (r != KRONQ_OK) return r;
+    } else if (j1 < n) {
       GemmDesc g;
       g.M = m; g.N = n - j1; g.K = bw;
       g.A = a.Eb; g.lda = a.lde;

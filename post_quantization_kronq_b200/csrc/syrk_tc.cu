@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + cc * 32, v);
         tmem_wait_ld();
         const int64_t jb = c0 + cc * 32;

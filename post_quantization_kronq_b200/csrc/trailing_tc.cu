@@ -1,0 +1,270 @@
+// Lazy-batch trailing update of the column sweep on the tensor cores:
+//   W[:, j1:] -= E_blk U[blk, j1:]
+// (GPTQ's block error feedback, which KronQ's sweep keeps; KronQ README intro).
+//
+// K = 128 (one block of columns), so the update is a thin GEMM whose cost is
+// the read-modify-write of W.  To keep float32-level accuracy with bf16 MMAs
+// both operands are split, x = hi + lo with hi = bf16(x), lo = bf16(x - hi),
+// and the product is E_hi U_hi + E_hi U_lo + E_lo U_hi (the dropped lo*lo term
+// is ~2^-16 relative), accumulated in fp32 in TMEM.
+//
+// One CTA per 128 x 128 tile of W[:, j1:]: warp 0 issues all TMA loads (the
+// fp32 W tile into shared memory, two 64-wide k chunks of E_hi/E_lo, K-major,
+// and of U_hi/U_lo, MN-major), warp 1 issues 24 tcgen05.mma (M 128, N 128,
+// K 16) into 128 TMEM columns, warps 2-5 subtract the accumulator from the
+// staged tile (128-byte swizzled boxes, conflict-free float4 accesses) and
+// write it back with TMA stores.  Each element is owned by one CTA.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace kq {
+namespace {
+
+constexpr int BM = 128, BN = 128, KC = 64, NKC = 2;
+constexpr int A_BOX = BM * KC * 2;         // 16 KB: 128 rows x 64 k (K-major, 128 B rows)
+constexpr int B_BOX = 64 * KC * 2;         // 8 KB: 64 k rows x 64 columns (MN-major)
+constexpr int B_SPLIT = (BN / 64) * B_BOX; // 16 KB: one split of the B chunk
+constexpr int CHUNK_BYTES = 2 * A_BOX + 2 * B_SPLIT;   // hi+lo of A and B: 64 KB
+constexpr int C_BOX = BM * 32 * 4;         // 16 KB: 128 rows x 32 fp32 (128-byte swizzle)
+constexpr int C_BYTES = (BN / 32) * C_BOX; // 64 KB
+constexpr int SMEM_BYTES = NKC * CHUNK_BYTES + C_BYTES + 1024 + 256;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = BN;
+
+struct TrailArgs {
+  float* W;       // full W~ (row stride n)
+  int64_t m, n;
+  int64_t j1;     // first column to update
+  int nkc;        // k chunks present (bw / 64, rounded up)
+  int tma_c;      // 1: W tile staged through shared memory by TMA
+  const int* info;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    trailing_tc_kernel(const __grid_constant__ CUtensorMap mEh, const __grid_constant__ CUtensorMap mEl,
+                       const __grid_constant__ CUtensorMap mUh, const __grid_constant__ CUtensorMap mUl,
+                       const __grid_constant__ CUtensorMap mW, TrailArgs args) {
+  if (args.info && *args.info != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NKC * CHUNK_BYTES + C_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NKC + 2);
+  const uint32_t full0 = smem_u32(&bars[0]);
+  const uint32_t cbar = smem_u32(&bars[NKC]);
+  const uint32_t accbar = smem_u32(&bars[NKC + 1]);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r0 = (int64_t)blockIdx.y * BM;
+  const int64_t c0 = args.j1 + (int64_t)blockIdx.x * BN;
+
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < NKC; ++c) mbar_init(full0 + 8 * c, 1);
+    mbar_init(cbar, 1);
+    mbar_init(accbar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t cs = base + NKC * CHUNK_BYTES;   // staged W tile
+
+  if (warp == 0) {
+    if (lane == 0) {
+      if (args.tma_c) {
+        mbar_arrive_expect_tx(cbar, C_BYTES);
+#pragma unroll
+        for (int h = 0; h < BN / 32; ++h) tma_load_2d(cs + h * C_BOX, &mW, cbar, (int)(c0 + 32 * h), (int)r0);
+      }
+      for (int c = 0; c < args.nkc; ++c) {
+        const uint32_t full = full0 + 8 * c;
+        const uint32_t s = base + c * CHUNK_BYTES;
+        mbar_arrive_expect_tx(full, CHUNK_BYTES);
+        tma_load_2d(s, &mEh, full, c * KC, (int)r0);
+        tma_load_2d(s + A_BOX, &mEl, full, c * KC, (int)r0);
+#pragma unroll
+        for (int h = 0; h < BN / 64; ++h) {
+          tma_load_2d(s + 2 * A_BOX + h * B_BOX, &mUh, full, (int)(c0 + 64 * h), c * KC);
+          tma_load_2d(s + 2 * A_BOX + B_SPLIT + h * B_BOX, &mUl, full, (int)(c0 + 64 * h), c * KC);
+        }
+      }
+      for (int c = 0; c < args.nkc; ++c) mbar_wait(full0 + 8 * c, 0);
+      if (args.tma_c) mbar_wait(cbar, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, true);
+      uint32_t acc = 0;
+      for (int c = 0; c < args.nkc; ++c) {
+        if (!mbar_wait(full0 + 8 * c, 0)) break;
+        tc_fence_after();
+        const uint32_t s = base + c * CHUNK_BYTES;
+        const uint32_t ah = s, al = s + A_BOX;
+        const uint32_t bh = s + 2 * A_BOX, bl = s + 2 * A_BOX + B_SPLIT;
+#pragma unroll
+        for (int kk = 0; kk < KC / 16; ++kk) {
+          // A K-major: 16 k = 32 bytes along each 128-byte row.  B MN-major:
+          // 16 k rows of 128 bytes = 2048 bytes inside every 64-column box.
+          const uint64_t dah = smem_desc_sw128(ah + kk * 32, 16, 1024);
+          const uint64_t dal = smem_desc_sw128(al + kk * 32, 16, 1024);
+          const uint64_t dbh = smem_desc_sw128(bh + kk * 2048, B_BOX, 1024);
+          const uint64_t dbl = smem_desc_sw128(bl + kk * 2048, B_BOX, 1024);
+          mma_bf16(tmem, dah, dbh, idesc, acc);
+          acc = 1;
+          mma_bf16(tmem, dah, dbl, idesc, 1u);
+          mma_bf16(tmem, dal, dbh, idesc, 1u);
+        }
+      }
+      mma_commit(accbar);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int rl = q * 32 + lane;          // row of the tile
+    bool ok = true;
+    if (lane == 0) {
+      ok = mbar_wait(accbar, 0);
+      if (ok && args.tma_c) ok = mbar_wait(cbar, 0);
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    if (ok) {
+      tc_fence_after();
+      const int64_t i = r0 + rl;
+      const int64_t n = args.n;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + cc * 32, v);
+        tmem_wait_ld();
+        if (args.tma_c) {
+          uint8_t* box = smem + NKC * CHUNK_BYTES + cc * C_BOX;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            float4* p4 = reinterpret_cast<float4*>(box + sw128_f32(rl, 4 * ch));
+            float4 w = *p4;
+            w.x -= __uint_as_float(v[4 * ch]);
+            w.y -= __uint_as_float(v[4 * ch + 1]);
+            w.z -= __uint_as_float(v[4 * ch + 2]);
+            w.w -= __uint_as_float(v[4 * ch + 3]);
+            *p4 = w;
+          }
+        } else {
+          const int64_t jb = c0 + cc * 32;
+          if (i < args.m && jb < n) {
+            float* row = args.W + i * n + jb;
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              if (jb + t < n) row[t] -= __uint_as_float(v[t]);
+          }
+        }
+      }
+      if (args.tma_c) {
+        fence_proxy_async_smem();
+        named_barrier(1, 128);             // the four epilogue warps
+        if (warp == 2 && lane == 0) {
+#pragma unroll
+          for (int h = 0; h < BN / 32; ++h) tma_store_2d(&mW, cs + h * C_BOX, (int)(c0 + 32 * h), (int)r0);
+          tma_store_commit();
+          tma_store_wait_all();
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool map_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, int64_t inner,
+            int64_t outer, int64_t ld, uint32_t box_inner, uint32_t box_outer) {
+  auto encode = encode_fn();
+  if (!encode) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t gstride[1] = {(cuuint64_t)(ld * esize)};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, dt, 2, const_cast<void*>(base), gdim, gstride, box,
+                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t status_fetch_trailing(int* out, cudaStream_t s) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  *out = v;
+  return e;
+}
+
+kronq_status trailing_maps(TrailingMaps* tm, const void* Eh, const void* El, int64_t m,
+                           const void* Uh, const void* Ul, int64_t ldu, float* W, int64_t n) {
+  static_assert(sizeof(tm->raw) == 5 * sizeof(CUtensorMap), "map storage");
+  CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(tm->raw);
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // E hi/lo: m rows x 128 k, K-major boxes of 64 k x 128 rows.
+  // U hi/lo: 128 k rows x n columns (row stride ldu), boxes of 64 columns x 64 k.
+  if (!map_2d(&maps[0], bf, 2, Eh, 128, m, 128, 64, BM) || !map_2d(&maps[1], bf, 2, El, 128, m, 128, 64, BM) ||
+      !map_2d(&maps[2], bf, 2, Uh, n, 128, ldu, 64, KC) || !map_2d(&maps[3], bf, 2, Ul, n, 128, ldu, 64, KC))
+    return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (trailing update)");
+  // W tile staging (fp32, 32-column boxes): needs a 16-byte row stride.
+  tm->tma_c = ((n % 4) == 0 && aligned(W, 16)) ? 1 : 0;
+  if (tm->tma_c && !map_2d(&maps[4], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W, n, m, n, 32, BM))
+    return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (trailing update, W)");
+  return KRONQ_OK;
+}
+
+kronq_status trailing_update_tc(const TrailingMaps* tm, float* W, int64_t m, int64_t n, int64_t j1,
+                                int bw, const int* info, cudaStream_t s) {
+  if (j1 >= n) return KRONQ_OK;
+  const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(tm->raw);
+  TrailArgs a;
+  a.W = W;
+  a.m = m;
+  a.n = n;
+  a.j1 = j1;
+  a.nkc = (bw + KC - 1) / KC;
+  a.tma_c = tm->tma_c;
+  a.info = info;
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(&trailing_tc_kernel), SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(trailing)");
+  dim3 grid((unsigned)ceil_div(n - j1, BN), (unsigned)ceil_div(m, BM));
+  trailing_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], a);
+  KQ_LAUNCH_CHECK("trailing_tc_kernel");
+  return KRONQ_OK;
+}
+
+}  // namespace kq
