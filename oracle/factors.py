@@ -41,3 +41,9 @@ def sensitivity(HX, HG):
     trx = trace_of_factor(HX)
     trg = trace_of_factor(HG)
     return trx, trg, trg * trx
+
+
+def factor_columns(A, cols) -> np.ndarray:
+    """Columns ``cols`` of H = A^T A: A^T a_j for each sampled j (float64)."""
+    A64 = np.asarray(A, dtype=np.float64)
+    return A64.T @ A64[:, list(cols)]

@@ -179,8 +179,12 @@ def gptq_sweep(Wt, U, bits: int, group: int, asym: bool = True, block: int = 1,
 def gptq_sweep_f32(Wt, U, bits: int, group: int, asym: bool = True, block: int = 128):
     """Float32 sweep in a fixed operation order (bit-exact test mode).
 
-    Every operation is one float32 operation, division correctly rounded,
-    multiply and subtract not fused.  In a block the rank-1 updates run in
+    Every operation is one float32 operation, multiply and subtract not
+    fused.  The grid of a group (scale, zero) uses correctly rounded
+    divisions; per column, the divisions by scale and by U_jj are
+    multiplications by the correctly rounded reciprocals 1/scale and 1/U_jj
+    (float32 throughout, so both the library and this mirror take every
+    rounding decision identically).  In a block the rank-1 updates run in
     column order; after the block, acc = sum_k E[:, k] U[k, later] is
     accumulated in ascending k (one rounding per product and per add) and
     then W[:, later] = W[:, later] - acc.
@@ -202,13 +206,17 @@ def gptq_sweep_f32(Wt, U, bits: int, group: int, asym: bool = True, block: int =
             start, g0, g1 = _group_bounds(j, n, group, block)
             if start:
                 scale, zero = grid_params(W[:, g0:g1], bits, asym, dtype=f32)
+                inv_scale = (f32(1) / scale).astype(f32)
                 gi = 0 if group == -1 else j // group
                 scales[:, gi] = scale
                 zeros[:, gi] = zero
-            q, deq = quantize(W[:, j], scale, zero, bits, dtype=f32)
+            maxq = f32(2 ** bits - 1)
+            q = np.clip(np.rint((W[:, j] * inv_scale).astype(f32)) + zero, f32(0), maxq).astype(f32)
+            deq = (scale * (q - zero)).astype(f32)
             codes[:, j] = q.astype(np.int64)
             Q[:, j] = deq
-            e = ((W[:, j] - deq).astype(f32) / U[j, j]).astype(f32)
+            inv_u = f32(1) / U[j, j]
+            e = ((W[:, j] - deq).astype(f32) * inv_u).astype(f32)
             E[:, j] = e
             if j + 1 < b1:
                 prod = (e[:, None] * U[j, j + 1:b1][None, :]).astype(f32)

@@ -7,8 +7,9 @@
 // block, the owner lane of column j quantizes it, forms the scaled error
 // e = (w - deq) / U_jj, broadcasts e with a shuffle and every lane applies the
 // rank-1 update to its later columns.  All arithmetic of the sweep is single
-// float32 operations (division correctly rounded, multiply and subtract not
-// fused), so the result is reproducible bit for bit.
+// float32 operations (multiply and subtract not fused; the per-column
+// divisions by the group scale and by U_jj are multiplications by their
+// correctly rounded reciprocals), so the result is reproducible bit for bit.
 //
 // After each block the later columns get W[:, later] -= E_blk U[blk, later]
 // (the lazy-batch update), either as a fast GEMM or, in the ordered test mode,
@@ -25,7 +26,7 @@ constexpr int LPR = BW / QW;   // lanes per row (8)
 constexpr int WARPS = 8;       // warps per CTA
 constexpr int ROWS_PER_CTA = WARPS * 32 / LPR;   // 32
 constexpr int US_LD = BW + 4 * (BW / QW);        // padded row of the U block (160 floats)
-constexpr int SWEEP_SMEM = BW * US_LD * sizeof(float);
+constexpr int SWEEP_SMEM = BW * US_LD * sizeof(float) + BW * sizeof(float);  // + 1/U_jj
 
 struct BlockArgs {
   SweepDesc d;
@@ -56,7 +57,7 @@ __device__ __forceinline__ void grid_from_range(float lo, float hi, int bits, bo
 // the row reduce over their columns in [j, j + group).
 __device__ __forceinline__ void group_start(const float (&v)[QW], int j, int bw, int q,
                                             const SweepDesc& d, bool live, int64_t r, int64_t gi,
-                                            float& sc, float& zp) {
+                                            float& sc, float& zp, float& isc) {
   const int gend = (j + d.group < bw) ? j + d.group : bw;
   float lo = INFINITY, hi = -INFINITY;
 #pragma unroll
@@ -73,6 +74,7 @@ __device__ __forceinline__ void group_start(const float (&v)[QW], int j, int bw,
     hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
   grid_from_range(lo, hi, d.bits, d.asym, sc, zp);
+  isc = __frcp_rn(sc);
   if (q == 0 && live) {
     d.scales[r * d.ngroups + gi] = sc;
     d.zeros[r * d.ngroups + gi] = zp;
@@ -187,6 +189,10 @@ __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
     sc = d.scales[r * d.ngroups + gi];
     zp = d.zeros[r * d.ngroups + gi];
   }
+  float isc = __frcp_rn(sc);
+  // correctly rounded reciprocals of the block's diagonal of U
+  float* iu = Us + BW * US_LD;
+  if (tid < bw) iu[tid] = __frcp_rn(d.U[(j0 + tid) * n + j0 + tid]);
   __syncthreads();
 
   const float maxq = (float)((1 << d.bits) - 1);
@@ -202,19 +208,21 @@ __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
     const bool mine = q == qo;
     // Groups of 16 or more columns can only start at a lane boundary.
     if (!SMALLG && inblock_groups && qo * QW < bw && ((qo * QW) & gmask) == 0)
-      group_start(v, qo * QW, bw, q, d, live, r, g0 + ((qo * QW) >> gshift), sc, zp);
+      group_start(v, qo * QW, bw, q, d, live, r, g0 + ((qo * QW) >> gshift), sc, zp, isc);
 #pragma unroll
     for (int c = 0; c < QW; ++c) {
       const int j = qo * QW + c;
       if (j >= bw) break;
-      if (SMALLG && (j & gmask) == 0) group_start(v, j, bw, q, d, live, r, g0 + (j >> gshift), sc, zp);
+      if (SMALLG && (j & gmask) == 0) group_start(v, j, bw, q, d, live, r, g0 + (j >> gshift), sc, zp, isc);
       float e = 0.f;
       if (mine) {
         const float w = v[c];
-        float qv = __fadd_rn(rintf(__fdiv_rn(w, sc)), zp);
+        // division by scale and by U_jj as multiplication by the correctly
+        // rounded reciprocals (the float32 schedule of this library)
+        float qv = __fadd_rn(rintf(__fmul_rn(w, isc)), zp);
         qv = fminf(fmaxf(qv, 0.f), maxq);
         const float deq = __fmul_rn(sc, __fsub_rn(qv, zp));
-        e = __fdiv_rn(__fsub_rn(w, deq), Us[j * US_LD + ucol(j)]);
+        e = __fmul_rn(__fsub_rn(w, deq), iu[j]);
         v[c] = deq;
         ev[c] = e;
         code[c >> 2] |= ((uint32_t)qv & 0xFFu) << (8 * (c & 3));
