@@ -7,11 +7,13 @@
 // U = R^-1, since A^-1 = R^-T R^-1 = U^T U.  That is 2 n^3 / 3 flops in total.
 //
 // Blocked with nb = 64, bottom-right first.  For each diagonal block J:
-//   diag_panel_kernel  factor A_JJ = R_JJ R_JJ^T and solve R[0:j0, J] R_JJ^T
-//                      = A[0:j0, J] (every CTA factors the small block itself)
+//   diag_panel_kernel  factor A_JJ = R_JJ R_JJ^T (itself blocked by 16),
+//                      invert it, U_JJ = R_JJ^-1, and form the panel
+//                      R[0:j0, J] = A[0:j0, J] U_JJ^T (every CTA factors the
+//                      small block itself)
 //   schur_tc_kernel    A[0:j0, 0:j0] -= R[0:j0, J] R[0:j0, J]^T on the tensor
 //                      cores (upper triangle only, fp32-level split products)
-// Then every diagonal block is inverted at once (U_JJ = R_JJ^-1), and the
+// Then the diagonal blocks U_JJ are stored, and the
 // off-diagonal blocks of U come from the recursive formula
 //   inv([[R11, R12], [0, R22]]) = [[U11, -U11 R12 U22], [0, U22]]
 // evaluated level by level (block sizes nb, 2 nb, 4 nb, ...), each level one
@@ -57,20 +59,123 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* H, int64_t n, float d
 
 __global__ void zero_info_kernel(int* info) { *info = 0; }
 
-// Factor the diagonal block A_JJ = R_JJ R_JJ^T (reverse order) in shared
-// memory and solve the panel rows above it, R[i, J] R_JJ^T = A[i, J].
-// Every CTA factors the (small) block itself, so no extra launch sits on the
-// sequential path; CTA 0 writes R_JJ back.  A short block (nb < 64) is padded
-// with the identity.  The panel rows are also written as bf16 hi/mid/lo
-// splits for the tensor-core Schur update.
+// ---------------------------------------------------------------------------
+// Diagonal step of the blocked factorisation: one 64 x 64 block A_JJ,
+// factored and inverted in shared memory by 256 threads, then the panel
+// rows above it.  The block is handled as four 16 x 16 leaves (bottom-right
+// first); each leaf is factored and inverted by one warp in registers (lane
+// c holds column c of the symmetric leaf, pivots are shuffled), the rows
+// above the leaf are multiplied by U_leaf^T, and a rank-16 update follows.
+// U_JJ is assembled from the leaf inverses with the recursive formula.
+
+constexpr int LF = 16;                       // leaf width
+constexpr int PR = 32;                       // panel rows per chunk
+constexpr unsigned FULL = 0xffffffffu;
+
+struct alignas(16) DiagSmem {
+  union {
+    float a[NB][NB + 1];      // A_JJ (upper) -> R_JJ
+    float ut[NB][NB + 4];     // afterwards: U_JJ^T (16-byte aligned rows)
+  } x;
+  float u[NB][NB + 1];        // U_JJ (upper, zero below)
+  union {
+    float ulT[LF][LF];        // U_leaf^T of the current leaf
+    float tb[32][33];         // products R12 U22 while U_JJ is assembled
+    float ach[PR][NB + 1];    // a chunk of panel rows
+  } y;
+  float rinv[NB];
+  int bad;
+};
+
+// Factor and invert the leaf at offset o (one warp).  Writes R_leaf into a,
+// U_leaf into u and its transpose into ulT, and 1 / R_kk into rinv.
+__device__ __forceinline__ void leaf_factor_invert(DiagSmem& S, int o, int lane) {
+  const int c = lane & (LF - 1);
+  float col[LF];
+#pragma unroll
+  for (int i = 0; i < LF; ++i) col[i] = (i <= c) ? S.x.a[o + i][o + c] : S.x.a[o + c][o + i];
+  float mypiv = 1.f;
+  bool badp = false;
+  int badk = -1;
+#pragma unroll
+  for (int K = LF - 1; K >= 0; --K) {
+    const float piv = __shfl_sync(FULL, col[K], K);
+    if (!(piv > 0.f) || !isfinite(piv)) {
+      if (!badp) badk = K;
+      badp = true;
+    }
+    if (c == K) mypiv = piv;
+    const float f = col[K] / piv;  // a[c][K] / pivot
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      const float aik = __shfl_sync(FULL, col[i], K);
+      if (c < K) col[i] = fmaf(-aik, f, col[i]);
+    }
+  }
+  if (lane == 0 && badp && S.bad == 0) S.bad = o + badk + 1;
+  // R[c][c] = sqrt(pivot), R[i][c] = a[i][c] / R[c][c] (values at pivot time)
+  const float rk = sqrtf(mypiv);
+  const float rin = 1.f / rk;
+#pragma unroll
+  for (int i = 0; i < LF; ++i) col[i] = (i < c) ? col[i] * rin : (i == c ? rk : 0.f);
+  // U_leaf = R_leaf^-1 by rows: lane i forms row i from U R = I.
+  const int i = c;
+  float urow[LF];
+#pragma unroll
+  for (int cc = 0; cc < LF; ++cc) {
+    const float rcc = __shfl_sync(FULL, rin, cc);
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < cc; ++k) {
+      const float rkc = __shfl_sync(FULL, col[k], cc);
+      if (k & 1) s1 = fmaf(urow[k], rkc, s1);
+      else s0 = fmaf(urow[k], rkc, s0);
+    }
+    urow[cc] = (cc < i) ? 0.f : (cc == i ? rcc : -(s0 + s1) * rcc);
+  }
+  if (lane < LF) {
+#pragma unroll
+    for (int k = 0; k < LF; ++k) {
+      if (k <= c) S.x.a[o + k][o + c] = col[k];
+      S.u[o + i][o + k] = urow[k];
+      S.y.ulT[k][i] = urow[k];
+    }
+    S.rinv[o + c] = rin;
+  }
+}
+
+// Loads PR panel rows [r0, r0 + PR) of columns J into registers (8 per thread).
+__device__ __forceinline__ void load_chunk(const float* H, int64_t n, int64_t j0, int nb,
+                                           int64_t r0, bool vec4, float (&v)[8]) {
+  const int t = threadIdx.x;
+  const int r = t >> 3, seg = (t & 7) * 8;
+  const int64_t i = r0 + r;
+  const float* src = H + i * n + j0 + seg;
+  if (i < j0 && vec4 && seg + 8 <= nb) {
+    const float4 p = *reinterpret_cast<const float4*>(src);
+    const float4 q = *reinterpret_cast<const float4*>(src + 4);
+    v[0] = p.x; v[1] = p.y; v[2] = p.z; v[3] = p.w;
+    v[4] = q.x; v[5] = q.y; v[6] = q.z; v[7] = q.w;
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = (i < j0 && seg + q < nb) ? src[q] : 0.f;
+  }
+}
+
+// Factor the diagonal block A_JJ = R_JJ R_JJ^T (reverse order), invert it,
+// and form the panel above it, R[i, J] = A[i, J] U_JJ^T.  Every CTA factors
+// the (small) block itself, so no extra launch sits on the sequential path;
+// CTA 0 stages U_JJ (64 x 64, row-major) at stage[j0 * 64].  A short block
+// (nb < 64) is padded with the identity.  The panel rows are also written
+// as bf16 hi/mid/lo splits for the tensor-core Schur update.
 __global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, int64_t j0, int nb,
-                                                         int* info, __nv_bfloat16* splits) {
+                                                         int* info, __nv_bfloat16* splits,
+                                                         float* stage, int vec4) {
   if (*info != 0) return;
-  __shared__ float a[NB][NB + 1];
-  __shared__ float rdiag[NB], rinv[NB];
-  const int tid = threadIdx.x;
-  const int tx = tid & 63, ty = tid >> 6;
+  __shared__ DiagSmem S;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   {
+    const int tx = tid & 63, ty = tid >> 6;
     float x[NB / 4];
 #pragma unroll
     for (int sl = 0; sl < NB / 4; ++sl) {  // all sixteen loads in flight
@@ -80,142 +185,213 @@ __global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, in
 #pragma unroll
     for (int sl = 0; sl < NB / 4; ++sl) {
       const int r = 4 * sl + ty;
-      a[r][tx] = (tx < nb) ? x[sl] : (r == tx ? 1.f : 0.f);
+      S.x.a[r][tx] = (tx < nb) ? x[sl] : (r == tx ? 1.f : 0.f);
+      S.u[r][tx] = 0.f;
     }
   }
-  // One barrier per pivot: the update of column c < k uses
-  // r_ik r_ck = a_ik a_ck / pivot, so column k itself is left unscaled until
-  // the end (it is never written again once its pivot is done).
-  for (int k = NB - 1; k >= 0; --k) {
+  // the first chunk of panel rows is fetched while the block is factored
+  float pv[8];
+  const int64_t chunk0 = (int64_t)blockIdx.x * PR;
+  load_chunk(H, n, j0, nb, chunk0, vec4 != 0, pv);
+  if (tid == 0) S.bad = 0;
+  __syncthreads();
+
+  for (int o = NB - LF; o >= 0; o -= LF) {
+    if (warp == 0) leaf_factor_invert(S, o, lane);
     __syncthreads();
-    const float piv = a[k][k];
-    if (!(piv > 0.f) || !isfinite(piv)) {
-      if (tid == 0 && blockIdx.x == 0) *info = (int)(j0 + k + 1);
-      return;  // uniform: every thread read the same pivot
+    if (S.bad) {
+      if (tid == 0 && blockIdx.x == 0) *info = (int)(j0 + S.bad);
+      return;  // uniform: read after the barrier
     }
-    if (tid == 0) {
-      const float rk = sqrtf(piv);
-      rdiag[k] = rk;
-      rinv[k] = 1.f / rk;
-    }
-    if (tx < k) {
-      // all loads first: stores to column tx cannot be proven not to alias
-      // column k, so interleaving would serialise the sixteen updates
-      const float act = a[tx][k] * (1.f / piv);
-      float ck[NB / 4], ct[NB / 4];
+    if (o == 0) break;
+    // rows i < o of the leaf's columns: R[i, leaf] = A[i, leaf] U_leaf^T
+    {
+      const int i = tid >> 2, g = (tid & 3) * 4;
+      float o4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (i < o) {
 #pragma unroll
-      for (int sl = 0; sl < NB / 4; ++sl) {
-        ck[sl] = a[4 * sl + ty][k];
-        ct[sl] = a[4 * sl + ty][tx];
+        for (int l = 0; l < LF; ++l) {
+          const float al = S.x.a[i][o + l];
+          const float4 w = *reinterpret_cast<const float4*>(&S.y.ulT[l][g]);
+          o4[0] = fmaf(al, w.x, o4[0]);
+          o4[1] = fmaf(al, w.y, o4[1]);
+          o4[2] = fmaf(al, w.z, o4[2]);
+          o4[3] = fmaf(al, w.w, o4[3]);
+        }
       }
+      __syncthreads();
+      if (i < o) {
 #pragma unroll
-      for (int sl = 0; sl < NB / 4; ++sl) {
-        const int i = 4 * sl + ty;
-        if (i <= tx) a[i][tx] = ct[sl] - ck[sl] * act;
+        for (int q = 0; q < 4; ++q) S.x.a[i][o + g + q] = o4[q];
       }
     }
-  }
-  __syncthreads();
-  // scale every column k of R above the diagonal by 1 / r_kk
+    __syncthreads();
+    // rank-16 update of the leading o x o upper triangle
+    {
+      const int cc = tid & 63, ty = tid >> 6;
+      if (cc < o) {
+        float rc[LF];
 #pragma unroll
-  for (int sl = 0; sl < NB / 4; ++sl) {
-    const int i = 4 * sl + ty;
-    if (i < tx) a[i][tx] *= rinv[tx];
+        for (int k = 0; k < LF; ++k) rc[k] = S.x.a[cc][o + k];
+        for (int i = ty; i <= cc; i += 4) {
+          float acc = 0.f;
+#pragma unroll
+          for (int k = 0; k < LF; ++k) acc = fmaf(S.x.a[i][o + k], rc[k], acc);
+          S.x.a[i][cc] -= acc;
+        }
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
+
+  // U_JJ from the leaf inverses: for pairs of diagonal blocks of size s,
+  // U12 = -U11 (R12 U22).  s = 16: two pairs, two outputs per thread.
+  {
+    const int p = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
+    const int b0 = 32 * p;
+    float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float rk = S.x.a[b0 + r][b0 + 16 + k];
+      t0 = fmaf(rk, S.u[b0 + 16 + k][b0 + 16 + c], t0);
+      t1 = fmaf(rk, S.u[b0 + 16 + k][b0 + 16 + c + 1], t1);
+    }
+    S.y.tb[16 * p + r][c] = t0;
+    S.y.tb[16 * p + r][c + 1] = t1;
+    __syncthreads();
+    float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float uk = S.u[b0 + r][b0 + k];
+      v0 = fmaf(uk, S.y.tb[16 * p + k][c], v0);
+      v1 = fmaf(uk, S.y.tb[16 * p + k][c + 1], v1);
+    }
+    S.u[b0 + r][b0 + 16 + c] = -v0;
+    S.u[b0 + r][b0 + 16 + c + 1] = -v1;
+    __syncthreads();
+  }
+  // s = 32: one pair, four outputs per thread.
+  {
+    const int r = tid >> 3, c = (tid & 7) * 4;
+    float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float rk = S.x.a[r][32 + k];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) t[q] = fmaf(rk, S.u[32 + k][32 + c + q], t[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) S.y.tb[r][c + q] = t[q];
+    __syncthreads();
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float uk = S.u[r][k];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] = fmaf(uk, S.y.tb[k][c + q], v[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) S.u[r][32 + c + q] = -v[q];
+    __syncthreads();
+  }
+  // U_JJ^T (over R_JJ, no longer needed); CTA 0 stages U_JJ.
+  for (int t = tid; t < NB * NB; t += blockDim.x) {
+    const int r = t >> 6, c = t & 63;
+    S.x.ut[c][r] = S.u[r][c];
+  }
   if (blockIdx.x == 0) {
-    for (int t = tid; t < nb * NB; t += blockDim.x) {
-      const int r = t >> 6, c = t & 63;
-      if (c < nb) H[(j0 + r) * n + j0 + c] = (r < c) ? a[r][c] : (r == c ? rdiag[r] : 0.f);
-    }
+    float* dst = stage + j0 * NB;
+    for (int t = tid; t < nb * NB; t += blockDim.x) dst[t] = S.u[t >> 6][t & 63];
   }
-  // Panel rows: x R_JJ^T = a, back substitution from the last column; one
-  // warp per row, lane l holds columns l and l + 32.
-  const int warp = tid >> 5, lane = tid & 31;
+  // Panel rows, chunks of PR rows: R[i][c] = sum_k A[i][k] U[c][k].
   const int64_t plane = (int64_t)n * NB;
-  for (int64_t i = (int64_t)blockIdx.x * 8 + warp; i < j0; i += (int64_t)gridDim.x * 8) {
-    float* row = H + i * n + j0;
-    float acc0 = (lane < nb) ? row[lane] : 0.f;
-    float acc1 = (lane + 32 < nb) ? row[lane + 32] : 0.f;
-    float x0 = 0.f, x1 = 0.f;
-    for (int k = NB - 1; k >= 0; --k) {
-      const bool upper_half = k >= 32;
-      const int owner = k & 31;
-      float xk = (upper_half ? acc1 : acc0) * rinv[k];
-      xk = __shfl_sync(0xffffffffu, xk, owner);
-      if (lane == owner) {
-        if (upper_half) x1 = xk;
-        else x0 = xk;
-      }
-      if (lane < k) acc0 -= a[lane][k] * xk;
-      if (lane + 32 < k) acc1 -= a[lane + 32][k] * xk;
+  const int rp = tid >> 4, c0 = (tid & 15) * 4;
+  for (int64_t r0 = chunk0; r0 < j0; r0 += (int64_t)gridDim.x * PR) {
+    if (r0 != chunk0) load_chunk(H, n, j0, nb, r0, vec4 != 0, pv);
+    {
+      const int r = tid >> 3, seg = (tid & 7) * 8;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) S.y.ach[r][seg + q] = pv[q];
     }
-    if (lane < nb) row[lane] = x0;
-    if (lane + 32 < nb) row[lane + 32] = x1;
-    const float xs[2] = {x0, x1};
+    __syncthreads();
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 16
+    for (int k = 0; k < NB; ++k) {
+      const float a0 = S.y.ach[2 * rp][k], a1 = S.y.ach[2 * rp + 1][k];
+      const float4 w = *reinterpret_cast<const float4*>(&S.x.ut[k][c0]);
+      acc[0][0] = fmaf(a0, w.x, acc[0][0]);
+      acc[0][1] = fmaf(a0, w.y, acc[0][1]);
+      acc[0][2] = fmaf(a0, w.z, acc[0][2]);
+      acc[0][3] = fmaf(a0, w.w, acc[0][3]);
+      acc[1][0] = fmaf(a1, w.x, acc[1][0]);
+      acc[1][1] = fmaf(a1, w.y, acc[1][1]);
+      acc[1][2] = fmaf(a1, w.z, acc[1][2]);
+      acc[1][3] = fmaf(a1, w.w, acc[1][3]);
+    }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const float x = xs[h];
-      const __nv_bfloat16 bh = __float2bfloat16_rn(x);
-      const float r1 = x - __bfloat162float(bh);
-      const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
-      const __nv_bfloat16 bl = __float2bfloat16_rn(r1 - __bfloat162float(bm));
-      const int64_t o = i * NB + lane + 32 * h;
-      splits[o] = bh;
-      splits[plane + o] = bm;
-      splits[2 * plane + o] = bl;
+      const int64_t i = r0 + 2 * rp + h;
+      if (i >= j0) continue;
+      float* row = H + i * n + j0 + c0;
+      if (vec4 && c0 + 4 <= nb) {
+        *reinterpret_cast<float4*>(row) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (c0 + q < nb) row[q] = acc[h][q];
+      }
+      uint32_t wh[2] = {0u, 0u}, wm[2] = {0u, 0u}, wl[2] = {0u, 0u};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float x = acc[h][q];
+        const __nv_bfloat16 bh = __float2bfloat16_rn(x);
+        const float r1 = x - __bfloat162float(bh);
+        const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 bl = __float2bfloat16_rn(r1 - __bfloat162float(bm));
+        const int sh = 16 * (q & 1);
+        wh[q >> 1] |= (uint32_t)__bfloat16_as_ushort(bh) << sh;
+        wm[q >> 1] |= (uint32_t)__bfloat16_as_ushort(bm) << sh;
+        wl[q >> 1] |= (uint32_t)__bfloat16_as_ushort(bl) << sh;
+      }
+      const int64_t off = i * NB + c0;
+      *reinterpret_cast<uint2*>(splits + off) = make_uint2(wh[0], wh[1]);
+      *reinterpret_cast<uint2*>(splits + plane + off) = make_uint2(wm[0], wm[1]);
+      *reinterpret_cast<uint2*>(splits + 2 * plane + off) = make_uint2(wl[0], wl[1]);
     }
+    __syncthreads();  // ach is rewritten by the next chunk
   }
 }
 
-// U_JJ = R_JJ^-1 for every diagonal block at once (one CTA per block).
-// Entry (i, i + dd) depends only on entries of smaller distance dd, so the
-// diagonals are computed one after the other, four adjacent lanes per entry.
-__global__ void __launch_bounds__(256) diag_inverse_kernel(float* H, int64_t n, const int* info) {
+// Copy the staged diagonal blocks U_JJ into H (one CTA per block).  They are
+// staged because other CTAs of a diag_panel launch still read A_JJ from H.
+__global__ void __launch_bounds__(256) diag_store_kernel(float* H, int64_t n, const float* stage,
+                                                         const int* info) {
   if (*info != 0) return;
-  __shared__ float a[NB][NB + 1];
-  __shared__ float u[NB][NB + 1];
-  __shared__ float rinv[NB];
   const int64_t j0 = (int64_t)blockIdx.x * NB;
   const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
-  const int tid = threadIdx.x;
-  for (int t = tid; t < NB * NB; t += blockDim.x) {
+  const float* src = stage + j0 * NB;
+  for (int t = threadIdx.x; t < nb * NB; t += blockDim.x) {
     const int r = t >> 6, c = t & 63;
-    float x = 0.f;
-    if (r <= c) x = (c < nb) ? H[(j0 + r) * n + j0 + c] : (r == c ? 1.f : 0.f);
-    a[r][c] = x;
-    u[r][c] = 0.f;
-  }
-  __syncthreads();
-  if (tid < NB) rinv[tid] = 1.f / a[tid][tid];
-  __syncthreads();
-  const int ii = tid >> 2, part = tid & 3;
-  if (part == 0) u[ii][ii] = rinv[ii];
-  __syncthreads();
-  for (int dd = 1; dd < NB; ++dd) {
-    const int jj = ii + dd;
-    float acc = 0.f;
-    if (jj < NB)
-      for (int k = ii + 1 + part; k <= jj; k += 4) acc = fmaf(a[ii][k], u[k][jj], acc);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (jj < NB && part == 0) u[ii][jj] = -acc * rinv[ii];
-    __syncthreads();
-  }
-  for (int t = tid; t < nb * NB; t += blockDim.x) {
-    const int r = t >> 6, c = t & 63;
-    if (c < nb) H[(j0 + r) * n + j0 + c] = (r <= c) ? u[r][c] : 0.f;
+    if (c < nb) H[(j0 + r) * n + j0 + c] = src[t];
   }
 }
 
 }  // namespace
 
-size_t chol_workspace_bytes(int64_t n) {
+static size_t tbuf_bytes(int64_t n) {
   // recursive inverse: products T of the pairs of one level (at most n*n/4
-  // floats); bf16 hi/mid/lo splits of the current panel (3 x n x 64)
-  const size_t tbytes = (size_t)((n * n) / 4 + n + 64) * sizeof(float);
+  // floats); before it, the staged diagonal blocks U_JJ (n x 64 floats)
+  int64_t f = (n * n) / 4 + n + 64;
+  if (f < n * NB + NB * NB) f = n * NB + NB * NB;
+  return (((size_t)f * sizeof(float)) + 255) & ~size_t(255);
+}
+
+size_t chol_workspace_bytes(int64_t n) {
+  // T / staging buffer, then the bf16 hi/mid/lo splits of the current panel
+  // (3 x n x 64)
+  const size_t tbytes = tbuf_bytes(n);
   const size_t sbytes = (size_t)3 * n * NB * sizeof(__nv_bfloat16);
-  return ((tbytes + 255) & ~size_t(255)) + sbytes;
+  return tbytes + sbytes;
 }
 
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
@@ -228,9 +404,9 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
     KQ_LAUNCH_CHECK("zero_info_kernel");
   }
   if (n <= 0) return KRONQ_OK;
-  const size_t tbytes = (size_t)((n * n) / 4 + n + 64) * sizeof(float);
-  __nv_bfloat16* splits = reinterpret_cast<__nv_bfloat16*>(
-      static_cast<uint8_t*>(ws) + ((tbytes + 255) & ~size_t(255)));
+  float* Tbuf = reinterpret_cast<float*>(ws);
+  __nv_bfloat16* splits =
+      reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + tbuf_bytes(n));
   SchurMaps maps;
   if (n > NB) {
     kronq_status r = schur_maps(&maps, splits, H, n);
@@ -239,23 +415,23 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
   // Blocks are aligned from the top (0, NB, 2 NB, ...); the last may be short.
   const int64_t nblk = ceil_div(n, NB);
   const int64_t pmax = sm_count();
+  const int vec4 = ((n % 4) == 0 && aligned(H, 16)) ? 1 : 0;
   for (int64_t bj = nblk - 1; bj >= 0; --bj) {
     const int64_t j0 = bj * NB;
     const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
-    // One CTA per SM at most (each CTA factors the block itself), at least
-    // four panel rows per warp.
-    int64_t pg = j0 > 0 ? ceil_div(j0, 32) : 1;
+    // One CTA per SM at most (each CTA factors the block itself), one chunk
+    // of panel rows per CTA where that suffices.
+    int64_t pg = j0 > 0 ? ceil_div(j0, PR) : 1;
     if (pg > pmax) pg = pmax;
-    diag_panel_kernel<<<(unsigned)pg, 256, 0, s>>>(H, n, j0, nb, info, splits);
+    diag_panel_kernel<<<(unsigned)pg, 256, 0, s>>>(H, n, j0, nb, info, splits, Tbuf, vec4);
     KQ_LAUNCH_CHECK("diag_panel_kernel");
     if (j0 == 0) break;
     kronq_status r = schur_update_tc(&maps, H, n, j0, info, s);
     if (r != KRONQ_OK) return r;
   }
-  diag_inverse_kernel<<<(unsigned)nblk, 256, 0, s>>>(H, n, info);
-  KQ_LAUNCH_CHECK("diag_inverse_kernel");
+  diag_store_kernel<<<(unsigned)nblk, 256, 0, s>>>(H, n, Tbuf, info);
+  KQ_LAUNCH_CHECK("diag_store_kernel");
   // Recursive inverse of the off-diagonal blocks.
-  float* Tbuf = reinterpret_cast<float*>(ws);
   for (int64_t S = NB; S < n; S *= 2) {
     const int64_t npairs_full = n / (2 * S);  // pairs whose R22 has full size S
     struct Pair { int64_t p0, cnt, s2; };
