@@ -17,7 +17,7 @@
 // off-diagonal blocks of U come from the recursive formula
 //   inv([[R11, R12], [0, R22]]) = [[U11, -U11 R12 U22], [0, U22]]
 // evaluated level by level (block sizes nb, 2 nb, 4 nb, ...), each level one
-// batched pair of GEMMs.  A non-positive pivot stops the chain and records
+// batched pair of tensor-core products with a triangular factor.  A non-positive pivot stops the chain and records
 // info = 1 + its index (LAPACK convention); every later kernel then returns.
 #include <math.h>
 
@@ -443,29 +443,29 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
       const int64_t base = gp.p0 * 2 * S;  // R11 origin of the first pair
       const int64_t s2 = gp.s2;
       // T = R12 * U22   (S x s2) = (S x s2)(s2 x s2, upper)
-      GemmDesc t;
+      TriGemm t;
       t.M = S; t.N = s2; t.K = s2;
       t.A = H + base * n + base + S; t.lda = n;
       t.B = H + (base + S) * n + base + S; t.ldb = n; t.b_upper = true;
       t.C = Tbuf; t.ldc = s2;
-      t.alpha = 1.f; t.beta = 0.f;
+      t.alpha = 1.f;
       t.batch = (int)gp.cnt;
       t.strideA = 2 * S * n + 2 * S; t.strideB = 2 * S * n + 2 * S; t.strideC = S * s2;
       t.info = info;
-      cudaError_t e = gemm_f32(t, s);
-      if (e != cudaSuccess) return cuda_fail(e, "gemm(inverse T)");
+      kronq_status r = trigemm_tc(t, s);
+      if (r != KRONQ_OK) return r;
       // U12 = -U11 * T  (S x s2) = (S x S, upper)(S x s2)
-      GemmDesc u;
+      TriGemm u;
       u.M = S; u.N = s2; u.K = S;
       u.A = H + base * n + base; u.lda = n; u.a_upper = true;
       u.B = Tbuf; u.ldb = s2;
       u.C = H + base * n + base + S; u.ldc = n;
-      u.alpha = -1.f; u.beta = 0.f;
+      u.alpha = -1.f;
       u.batch = (int)gp.cnt;
       u.strideA = 2 * S * n + 2 * S; u.strideB = S * s2; u.strideC = 2 * S * n + 2 * S;
       u.info = info;
-      e = gemm_f32(u, s);
-      if (e != cudaSuccess) return cuda_fail(e, "gemm(inverse U12)");
+      r = trigemm_tc(u, s);
+      if (r != KRONQ_OK) return r;
     }
   }
   return KRONQ_OK;

@@ -39,6 +39,29 @@ struct GemmDesc {
 };
 cudaError_t gemm_f32(const GemmDesc& g, cudaStream_t s);
 
+// ------------------------------------------------------------ tensor-core triangular GEMM
+// C = alpha * A B (row-major fp32, optional batch with element strides) with
+// exactly one triangular operand: a_upper (A[i][k] = 0 for k < i) or
+// b_upper (B[k][j] = 0 for k > j); the other triangle of its storage is
+// never used.  fp32-level accuracy (six bf16 split products).  No-op when
+// info != nullptr and *info != 0.
+struct TriGemm {
+  int64_t M = 0, N = 0, K = 0;
+  const float* A = nullptr;
+  int64_t lda = 0;
+  const float* B = nullptr;
+  int64_t ldb = 0;
+  float* C = nullptr;
+  int64_t ldc = 0;
+  float alpha = 1.f;
+  bool a_upper = false, b_upper = false;
+  int batch = 1;
+  int64_t strideA = 0, strideB = 0, strideC = 0;
+  const int* info = nullptr;
+};
+kronq_status trigemm_tc(const TriGemm& t, cudaStream_t s);
+cudaError_t status_fetch_trigemm(int* out, cudaStream_t s);
+
 // ------------------------------------------------------------ factors
 kronq_status syrk_bf16_tc(const void* A, int64_t T, int64_t d, int64_t lda, float* H,
                           bool zero_first, cudaStream_t s);

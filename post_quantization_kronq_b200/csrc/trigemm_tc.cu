@@ -1,0 +1,357 @@
+// Float32 products with a triangular factor, on the tensor cores:
+//   C = alpha * A B,  A (M x K) row-major, B (K x N) row-major, C row-major,
+// with A upper triangular (A[i][k] = 0 for k < i) or B upper triangular
+// (B[k][j] = 0 for k > j) as the recursive triangular inverse needs them
+// (T = R12 U22, then U12 = -U11 T).  The triangle is masked on the fly, so
+// the other triangle of the storage may hold anything; a tile only walks
+// the k range its triangle leaves non-zero.
+//
+// Float32-level accuracy from bf16 MMAs: every operand element is split as
+// x = hi + mid + lo (bf16 roundings of the remainders) and the six products
+// hh + hm + mh + hl + lh + mm are accumulated in fp32 in TMEM (the dropped
+// terms are below 2^-24 relative).  There is no pre-pass and no workspace:
+// eight warps load the fp32 operands from global memory (one chunk ahead, in
+// registers), write the splits into shared memory in the UMMA 128-byte
+// swizzled layouts (A K-major, B MN-major), and arrive on the stage's
+// barrier; thread 0 then issues the chunk's tcgen05.mma (M 128, N 128,
+// K 16; 24 per 64-deep chunk) and commits the stage back.  Two stages of 96 KB.  The
+// epilogue stages the accumulator through shared memory and writes C with
+// coalesced stores.
+#include "common.cuh"
+#include "internal.h"
+
+namespace kq {
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int A_SPLIT = BM * BK * 2;            // 16 KB: 128 rows x 64 k, K-major
+constexpr int B_BOX = 64 * BK * 2;              // 8 KB: 64 k rows x 64 columns, MN-major
+constexpr int B_SPLIT = (BN / 64) * B_BOX;      // 16 KB
+constexpr int STAGE = 3 * A_SPLIT + 3 * B_SPLIT;  // 96 KB
+constexpr int NSTAGE = 2;
+constexpr int CV_THREADS = 256;                 // warps 0-7: convert, MMA issue, epilogue
+constexpr int THREADS = CV_THREADS;
+constexpr int SMEM_BYTES = NSTAGE * STAGE + 1024 + 256;
+constexpr int C_LD = BN + 4;                    // staged C row stride (floats)
+constexpr uint32_t TMEM_COLS = BN;
+static_assert(BM * C_LD * 4 <= NSTAGE * STAGE, "C staging fits the stages");
+
+struct TriArgs {
+  const float* A;
+  const float* B;
+  float* C;
+  int64_t lda, ldb, ldc, strideA, strideB, strideC;
+  int M, N, K;
+  float alpha;
+  int a_upper, b_upper;
+  int tiles_m, tiles_n;
+  int vecA, vecB, vecC;   // float4 access allowed
+  const int* info;
+};
+
+// Up to four consecutive floats p[0..valid-1], zero beyond.
+__device__ __forceinline__ float4 ld4(const float* p, int valid, bool vec) {
+  if (valid >= 4 && vec) return __ldg(reinterpret_cast<const float4*>(p));
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (valid > 0) r.x = __ldg(p);
+  if (valid > 1) r.y = __ldg(p + 1);
+  if (valid > 2) r.z = __ldg(p + 2);
+  if (valid > 3) r.w = __ldg(p + 3);
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 a, __nv_bfloat16 b) {
+  return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+}
+
+// Splits four floats into hi / mid / lo bf16 and stores each as 8 bytes.
+__device__ __forceinline__ void split_store4(uint8_t* smem, uint32_t off, uint32_t split_bytes,
+                                             float4 v) {
+  const float x[4] = {v.x, v.y, v.z, v.w};
+  __nv_bfloat16 h[4], m[4], l[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    h[q] = __float2bfloat16_rn(x[q]);
+    const float r1 = x[q] - __bfloat162float(h[q]);
+    m[q] = __float2bfloat16_rn(r1);
+    l[q] = __float2bfloat16_rn(r1 - __bfloat162float(m[q]));
+  }
+  *reinterpret_cast<uint2*>(smem + off) = make_uint2(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]));
+  *reinterpret_cast<uint2*>(smem + off + split_bytes) =
+      make_uint2(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]));
+  *reinterpret_cast<uint2*>(smem + off + 2 * split_bytes) =
+      make_uint2(pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]));
+}
+
+struct Chunk {
+  float4 a[8];
+  float4 b[8];
+};
+
+// Loads chunk kc (64 k) of A's tile rows and B's tile columns.
+//   A: load j covers rows 16 j + 2 w + (lane / 16), k = kc + 4 (lane % 16) .. +3
+//   B: load j covers k row kc + 8 j + w, columns 4 lane .. +3
+__device__ __forceinline__ void load_chunk(const TriArgs& g, const float* A, const float* B,
+                                           int m0, int n0, int kc, int warp, int lane, Chunk& c) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int r = 16 * j + 2 * warp + (lane >> 4);
+    const int row = m0 + r;
+    const int k = kc + 4 * (lane & 15);
+    int valid = (row < g.M) ? g.K - k : 0;
+    valid = valid < 0 ? 0 : valid;
+    float4 v = ld4(A + (int64_t)row * g.lda + k, valid, g.vecA != 0);
+    if (g.a_upper) {  // A[row][k] = 0 for k < row
+      if (k + 0 < row) v.x = 0.f;
+      if (k + 1 < row) v.y = 0.f;
+      if (k + 2 < row) v.z = 0.f;
+      if (k + 3 < row) v.w = 0.f;
+    }
+    c.a[j] = v;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int k = kc + 8 * j + warp;
+    const int col = n0 + 4 * lane;
+    int valid = (k < g.K) ? g.N - col : 0;
+    valid = valid < 0 ? 0 : valid;
+    float4 v = ld4(B + (int64_t)k * g.ldb + col, valid, g.vecB != 0);
+    if (g.b_upper) {  // B[k][col] = 0 for k > col
+      if (k > col + 0) v.x = 0.f;
+      if (k > col + 1) v.y = 0.f;
+      if (k > col + 2) v.z = 0.f;
+      if (k > col + 3) v.w = 0.f;
+    }
+    c.b[j] = v;
+  }
+}
+
+// Writes the splits of a loaded chunk into stage memory st.
+__device__ __forceinline__ void store_chunk(uint8_t* st, int warp, int lane, const Chunk& c) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int r = 16 * j + 2 * warp + (lane >> 4);
+    const int k = 4 * (lane & 15);
+    const uint32_t off = r * 128 + ((((k >> 3) ^ (r & 7))) << 4) + (k & 7) * 2;
+    split_store4(st, off, A_SPLIT, c.a[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int k = 8 * j + warp;
+    const int nn = 4 * lane;
+    const uint32_t off = 3 * A_SPLIT + (nn >> 6) * B_BOX + k * 128 +
+                         (((((nn & 63) >> 3) ^ (k & 7))) << 4) + (nn & 7) * 2;
+    split_store4(st, off, B_SPLIT, c.b[j]);
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1) trigemm_tc_kernel(TriArgs g) {
+  if (g.info && *g.info != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NSTAGE * STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NSTAGE + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Tile order: the tiles with the longest k range first.
+  const int bid = blockIdx.x;
+  int tm, tn;
+  if (g.b_upper) {
+    tn = g.tiles_n - 1 - bid / g.tiles_m;
+    tm = bid % g.tiles_m;
+  } else {
+    tm = bid / g.tiles_n;
+    tn = bid % g.tiles_n;
+  }
+  const int m0 = tm * BM, n0 = tn * BN;
+  int kbeg = g.a_upper ? m0 : 0;
+  int kend = g.K;
+  if (g.b_upper && n0 + BN < kend) kend = n0 + BN;
+  const int nchunks = kend > kbeg ? (kend - kbeg + BK - 1) / BK : 0;
+  const float* A = g.A + (int64_t)blockIdx.y * g.strideA;
+  const float* B = g.B + (int64_t)blockIdx.y * g.strideB;
+  float* C = g.C + (int64_t)blockIdx.y * g.strideC;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(smem_u32(&bars[s]), CV_THREADS);         // full: every converter thread
+      mbar_init(smem_u32(&bars[NSTAGE + s]), 1);         // empty: tcgen05.commit
+    }
+    mbar_init(smem_u32(&bars[2 * NSTAGE]), 1);           // accumulator ready
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t accbar = smem_u32(&bars[2 * NSTAGE]);
+
+  // Thread 0 also issues the MMAs of a chunk once every thread has stored
+  // its part (the instructions run asynchronously; issuing takes little).
+  auto issue = [&](int s) -> bool {
+    const int st = s & 1, use = s >> 1;
+    if (!mbar_wait(smem_u32(&bars[st]), use & 1)) return false;
+    tc_fence_after();
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, true);
+    const uint32_t sa = base + st * STAGE, sb = sa + 3 * A_SPLIT;
+#pragma unroll
+    for (int kk = 0; kk < BK / 16; ++kk) {
+#pragma unroll
+      for (int t = 0; t < 6; ++t) {
+        // split pairs (a, b) with a + b <= 2: hh, hm, mh, hl, lh, mm
+        const int pa = (t == 2 || t == 5) ? 1 : (t == 4 ? 2 : 0);
+        const int pb = (t == 1 || t == 5) ? 1 : (t == 3 ? 2 : 0);
+        const uint64_t da = smem_desc_sw128(sa + pa * A_SPLIT + kk * 32, 16, 1024);
+        const uint64_t db = smem_desc_sw128(sb + pb * B_SPLIT + kk * 2048, B_BOX, 1024);
+        mma_bf16(tmem, da, db, idesc, (s > 0 || kk > 0 || t > 0) ? 1u : 0u);
+      }
+    }
+    mma_commit(smem_u32(&bars[NSTAGE + st]));
+    return true;
+  };
+
+  {
+    bool ok = true;
+    Chunk c0, c1;
+    if (nchunks > 0) load_chunk(g, A, B, m0, n0, kbeg, warp, lane, c0);
+    for (int s = 0; s < nchunks && ok; s += 2) {
+      // chunk s from c0 (prefetch s + 1 into c1), then chunk s + 1 from c1
+      if (s + 1 < nchunks) load_chunk(g, A, B, m0, n0, kbeg + (s + 1) * BK, warp, lane, c1);
+      {
+        const int st = s & 1, use = s >> 1;
+        if (use > 0) ok = mbar_wait(smem_u32(&bars[NSTAGE + st]), (use - 1) & 1);
+        if (!ok) break;
+        store_chunk(smem + st * STAGE, warp, lane, c0);
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&bars[st]));
+        if (threadIdx.x == 0) ok = issue(s);
+        if (!ok) break;
+      }
+      if (s + 1 >= nchunks) break;
+      if (s + 2 < nchunks) load_chunk(g, A, B, m0, n0, kbeg + (s + 2) * BK, warp, lane, c0);
+      {
+        const int st = (s + 1) & 1, use = (s + 1) >> 1;
+        if (use > 0) ok = mbar_wait(smem_u32(&bars[NSTAGE + st]), (use - 1) & 1);
+        if (!ok) break;
+        store_chunk(smem + st * STAGE, warp, lane, c1);
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&bars[st]));
+        if (threadIdx.x == 0) ok = issue(s + 1);
+        if (!ok) break;
+      }
+    }
+    if (threadIdx.x == 0 && nchunks > 0) mma_commit(accbar);
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) .., columns 64 (w / 4) ..
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && nchunks > 0) {
+      int got = 1;
+      if (lane == 0) got = mbar_wait(accbar, 0) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+    }
+    const int q = warp & 3, hc = warp >> 2;
+    const int r = 32 * q + lane;
+    float* cst = reinterpret_cast<float*>(smem);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
+        if (nchunks > 0) {
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 64 * hc + 32 * cc, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = 0u;
+        }
+        float* dst = cst + r * C_LD + 64 * hc + 32 * cc;
+#pragma unroll
+        for (int t = 0; t < 32; t += 4)
+          *reinterpret_cast<float4*>(dst + t) =
+              make_float4(g.alpha * __uint_as_float(v[t]), g.alpha * __uint_as_float(v[t + 1]),
+                          g.alpha * __uint_as_float(v[t + 2]), g.alpha * __uint_as_float(v[t + 3]));
+      }
+    }
+    named_barrier(1, CV_THREADS);
+    if (ok) {
+      // rows warp, warp + 8, ...: lane covers columns 4 lane .. +3
+      const int col = n0 + 4 * lane;
+      const int valid = g.N - col;
+#pragma unroll 4
+      for (int rr = warp; rr < BM; rr += 8) {
+        const int row = m0 + rr;
+        if (row >= g.M || valid <= 0) continue;
+        const float4 x = *reinterpret_cast<const float4*>(cst + rr * C_LD + 4 * lane);
+        float* out = C + (int64_t)row * g.ldc + col;
+        if (valid >= 4 && g.vecC) {
+          *reinterpret_cast<float4*>(out) = x;
+        } else {
+          out[0] = x.x;
+          if (valid > 1) out[1] = x.y;
+          if (valid > 2) out[2] = x.z;
+          if (valid > 3) out[3] = x.w;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t status_fetch_trigemm(int* out, cudaStream_t s) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  *out = v;
+  return e;
+}
+
+kronq_status trigemm_tc(const TriGemm& t, cudaStream_t s) {
+  if (t.M <= 0 || t.N <= 0) return KRONQ_OK;
+  if (t.a_upper == t.b_upper) return fail(KRONQ_ERR_INVALID_ARG, "trigemm_tc: exactly one triangular operand");
+  if (t.M > (int64_t)1 << 30 || t.N > (int64_t)1 << 30 || t.K > (int64_t)1 << 30)
+    return fail(KRONQ_ERR_INVALID_ARG, "trigemm_tc: size out of range");
+  TriArgs g;
+  g.A = t.A; g.B = t.B; g.C = t.C;
+  g.lda = t.lda; g.ldb = t.ldb; g.ldc = t.ldc;
+  g.strideA = t.strideA; g.strideB = t.strideB; g.strideC = t.strideC;
+  g.M = (int)t.M; g.N = (int)t.N; g.K = (int)t.K;
+  g.alpha = t.alpha;
+  g.a_upper = t.a_upper ? 1 : 0;
+  g.b_upper = t.b_upper ? 1 : 0;
+  g.tiles_m = (int)ceil_div(t.M, BM);
+  g.tiles_n = (int)ceil_div(t.N, BN);
+  auto vec_ok = [&](const float* p, int64_t ld, int64_t stride) {
+    return aligned(p, 16) && (ld % 4) == 0 && (t.batch <= 1 || (stride % 4) == 0);
+  };
+  g.vecA = vec_ok(t.A, t.lda, t.strideA) ? 1 : 0;
+  g.vecB = vec_ok(t.B, t.ldb, t.strideB) ? 1 : 0;
+  g.vecC = vec_ok(t.C, t.ldc, t.strideC) ? 1 : 0;
+  g.info = t.info;
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(&trigemm_tc_kernel), SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(trigemm)");
+  dim3 grid((unsigned)(g.tiles_m * g.tiles_n), (unsigned)t.batch);
+  trigemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(g);
+  KQ_LAUNCH_CHECK("trigemm_tc_kernel");
+  return KRONQ_OK;
+}
+
+}  // namespace kq

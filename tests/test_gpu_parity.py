@@ -155,7 +155,7 @@ def _spd(n, seed, T=None):
     return (X.astype(np.float64).T @ X.astype(np.float64)).astype(np.float32)
 
 
-@pytest.mark.parametrize("n", [256, 200, 640, 1000])
+@pytest.mark.parametrize("n", [256, 200, 640, 1000, 1030, 2304])
 def test_cholesky_of_damped_inverse(n):
     H = _spd(n, seed=n)
     m = 32
