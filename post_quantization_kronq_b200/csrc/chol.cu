@@ -452,6 +452,8 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
       t.batch = (int)gp.cnt;
       t.strideA = 2 * S * n + 2 * S; t.strideB = 2 * S * n + 2 * S; t.strideC = S * s2;
       t.info = info;
+      t.holdA = H; t.holdA_rows = n; t.holdA_cols = n;
+      t.holdB = H; t.holdB_rows = n; t.holdB_cols = n;
       kronq_status r = trigemm_tc(t, s);
       if (r != KRONQ_OK) return r;
       // U12 = -U11 * T  (S x s2) = (S x S, upper)(S x s2)
@@ -464,6 +466,8 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
       u.batch = (int)gp.cnt;
       u.strideA = 2 * S * n + 2 * S; u.strideB = S * s2; u.strideC = 2 * S * n + 2 * S;
       u.info = info;
+      u.holdA = H; u.holdA_rows = n; u.holdA_cols = n;
+      u.holdB = Tbuf; u.holdB_rows = gp.cnt * S; u.holdB_cols = s2;
       r = trigemm_tc(u, s);
       if (r != KRONQ_OK) return r;
     }

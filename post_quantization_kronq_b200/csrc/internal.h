@@ -2,6 +2,8 @@
 // launcher assumes its arguments were validated by the C ABI layer.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -9,6 +11,14 @@
 #include "../../include/kronq.h"
 
 namespace kq {
+
+// ------------------------------------------------------------ TMA maps (host)
+// The driver's cuTensorMapEncodeTiled (nullptr when unavailable) and a 2-D
+// tiled map with the 128-byte swizzle: inner x outer elements, row stride
+// ld elements, box box_inner x box_outer, zero fill out of bounds.
+PFN_cuTensorMapEncodeTiled_v12000 tma_encode_fn();
+bool tma_map_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, int64_t inner,
+                int64_t outer, int64_t ld, uint32_t box_inner, uint32_t box_outer);
 
 // ------------------------------------------------------------ SIMT GEMM
 // C = beta * C + alpha * op(A) op(B), float32, one launch, optional batch.
@@ -58,6 +68,12 @@ struct TriGemm {
   int batch = 1;
   int64_t strideA = 0, strideB = 0, strideC = 0;
   const int* info = nullptr;
+  // Optional: the whole matrices that hold A and B (row strides lda, ldb),
+  // for TMA maps; A and B point inside them.  nullptr: plain loads only.
+  const float* holdA = nullptr;
+  int64_t holdA_rows = 0, holdA_cols = 0;
+  const float* holdB = nullptr;
+  int64_t holdB_rows = 0, holdB_cols = 0;
 };
 kronq_status trigemm_tc(const TriGemm& t, cudaStream_t s);
 cudaError_t status_fetch_trigemm(int* out, cudaStream_t s);

@@ -190,31 +190,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-bool map_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, int64_t inner,
-            int64_t outer, int64_t ld, uint32_t box_inner, uint32_t box_outer) {
-  auto encode = encode_fn();
-  if (!encode) return false;
-  cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-  cuuint64_t gstride[1] = {(cuuint64_t)(ld * esize)};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  return encode(map, dt, 2, const_cast<void*>(base), gdim, gstride, box,
-                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 }  // namespace
 
@@ -237,11 +212,11 @@ kronq_status schur_maps(SchurMaps* sm, const __nv_bfloat16* splits, float* H, in
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(sm->raw);
   for (int t = 0; t < 3; ++t) {
     const __nv_bfloat16* p = splits + (int64_t)t * n * KP;
-    if (!map_2d(&maps[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, KP, n, KP, KP, BM))
+    if (!tma_map_2d(&maps[t], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, KP, n, KP, KP, BM))
       return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (Schur update)");
   }
   sm->tma_c = ((n % 4) == 0 && aligned(H, 16)) ? 1 : 0;
-  if (sm->tma_c && !map_2d(&maps[3], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, n, n, n, 32, BM))
+  if (sm->tma_c && !tma_map_2d(&maps[3], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, n, n, n, 32, BM))
     return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (Schur update, H)");
   return KRONQ_OK;
 }

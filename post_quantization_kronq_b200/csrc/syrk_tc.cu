@@ -206,18 +206,6 @@ __global__ void fill_kernel(float* p, int64_t count, float v) {
     p[i] = v;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
 
 }  // namespace
 
@@ -247,7 +235,7 @@ cudaError_t status_fetch_syrk(int* out, cudaStream_t s) {
 
 kronq_status syrk_bf16_tc(const void* A, int64_t T, int64_t d, int64_t lda, float* H,
                           bool zero_first, cudaStream_t s) {
-  auto encode = encode_fn();
+  auto encode = tma_encode_fn();
   if (!encode) return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   CUtensorMap map;
   cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)T};

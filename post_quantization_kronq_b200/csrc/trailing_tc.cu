@@ -188,31 +188,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-bool map_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, int64_t inner,
-            int64_t outer, int64_t ld, uint32_t box_inner, uint32_t box_outer) {
-  auto encode = encode_fn();
-  if (!encode) return false;
-  cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-  cuuint64_t gstride[1] = {(cuuint64_t)(ld * esize)};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  return encode(map, dt, 2, const_cast<void*>(base), gdim, gstride, box,
-                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 }  // namespace
 
@@ -237,12 +212,12 @@ kronq_status trailing_maps(TrailingMaps* tm, const void* Eh, const void* El, int
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   // E hi/lo: m rows x 128 k, K-major boxes of 64 k x 128 rows.
   // U hi/lo: 128 k rows x n columns (row stride ldu), boxes of 64 columns x 64 k.
-  if (!map_2d(&maps[0], bf, 2, Eh, 128, m, 128, 64, BM) || !map_2d(&maps[1], bf, 2, El, 128, m, 128, 64, BM) ||
-      !map_2d(&maps[2], bf, 2, Uh, n, 128, ldu, 64, KC) || !map_2d(&maps[3], bf, 2, Ul, n, 128, ldu, 64, KC))
+  if (!tma_map_2d(&maps[0], bf, 2, Eh, 128, m, 128, 64, BM) || !tma_map_2d(&maps[1], bf, 2, El, 128, m, 128, 64, BM) ||
+      !tma_map_2d(&maps[2], bf, 2, Uh, n, 128, ldu, 64, KC) || !tma_map_2d(&maps[3], bf, 2, Ul, n, 128, ldu, 64, KC))
     return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (trailing update)");
   // W tile staging (fp32, 32-column boxes): needs a 16-byte row stride.
   tm->tma_c = ((n % 4) == 0 && aligned(W, 16)) ? 1 : 0;
-  if (tm->tma_c && !map_2d(&maps[4], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W, n, m, n, 32, BM))
+  if (tm->tma_c && !tma_map_2d(&maps[4], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W, n, m, n, 32, BM))
     return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (trailing update, W)");
   return KRONQ_OK;
 }

@@ -60,27 +60,22 @@ __device__ __forceinline__ float4 ld4(const float* p, int valid, bool vec) {
   return r;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 a, __nv_bfloat16 b) {
-  return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
-}
-
-// Splits four floats into hi / mid / lo bf16 and stores each as 8 bytes.
+// Splits four floats into hi / mid / lo bf16 (each the bf16 rounding of the
+// remainder so far) and stores each split as 8 bytes.
 __device__ __forceinline__ void split_store4(uint8_t* smem, uint32_t off, uint32_t split_bytes,
                                              float4 v) {
-  const float x[4] = {v.x, v.y, v.z, v.w};
-  __nv_bfloat16 h[4], m[4], l[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    h[q] = __float2bfloat16_rn(x[q]);
-    const float r1 = x[q] - __bfloat162float(h[q]);
-    m[q] = __float2bfloat16_rn(r1);
-    l[q] = __float2bfloat16_rn(r1 - __bfloat162float(m[q]));
-  }
-  *reinterpret_cast<uint2*>(smem + off) = make_uint2(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]));
-  *reinterpret_cast<uint2*>(smem + off + split_bytes) =
-      make_uint2(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]));
-  *reinterpret_cast<uint2*>(smem + off + 2 * split_bytes) =
-      make_uint2(pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]));
+  const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y);
+  const __nv_bfloat162 h23 = __floats2bfloat162_rn(v.z, v.w);
+  const float r0 = v.x - __low2float(h01), r1 = v.y - __high2float(h01);
+  const float r2 = v.z - __low2float(h23), r3 = v.w - __high2float(h23);
+  const __nv_bfloat162 m01 = __floats2bfloat162_rn(r0, r1);
+  const __nv_bfloat162 m23 = __floats2bfloat162_rn(r2, r3);
+  const __nv_bfloat162 l01 = __floats2bfloat162_rn(r0 - __low2float(m01), r1 - __high2float(m01));
+  const __nv_bfloat162 l23 = __floats2bfloat162_rn(r2 - __low2float(m23), r3 - __high2float(m23));
+  auto bits = [](__nv_bfloat162 x) { return *reinterpret_cast<const uint32_t*>(&x); };
+  *reinterpret_cast<uint2*>(smem + off) = make_uint2(bits(h01), bits(h23));
+  *reinterpret_cast<uint2*>(smem + off + split_bytes) = make_uint2(bits(m01), bits(m23));
+  *reinterpret_cast<uint2*>(smem + off + 2 * split_bytes) = make_uint2(bits(l01), bits(l23));
 }
 
 struct Chunk {
@@ -308,6 +303,249 @@ __global__ void __launch_bounds__(THREADS, 1) trigemm_tc_kernel(TriArgs g) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// TMA variant (16-byte aligned rows and origins): the fp32 operand tiles
+// arrive by TMA in a three-deep ring of 32-deep chunks; eight warps convert
+// each chunk into the bf16 splits (both operands MN-major, 128-byte
+// swizzle) in a two-deep ring; warp 8 lane 0 issues the TMA loads, warp 9
+// lane 0 the 12 MMAs per chunk.
+constexpr int TBK = 32;
+constexpr int TF_A = BM * TBK * 4;                // 16 KB: fp32 A box, 32 k x 128 m
+constexpr int TF_BBOX = TBK * 32 * 4;             // 4 KB: fp32 B box, 32 n x 32 k
+constexpr int TF_STAGE = TF_A + (BN / 32) * TF_BBOX;  // 32 KB
+constexpr int TNF = 3;
+constexpr int TS_BOX = 64 * TBK * 2;              // 4 KB: 64 m (or n) x 32 k, MN-major
+constexpr int TS_SPLIT = 2 * TS_BOX;              // 8 KB
+constexpr int TS_STAGE = 6 * TS_SPLIT;            // 48 KB: A hi/mid/lo, B hi/mid/lo
+constexpr int TNS = 2;
+constexpr int T_THREADS = CV_THREADS + 64;        // + producer warp + MMA warp
+constexpr int T_SMEM = TNF * TF_STAGE + TNS * TS_STAGE + 1024 + 256;
+static_assert(BM * C_LD * 4 <= TNF * TF_STAGE + TNS * TS_STAGE, "C staging fits");
+
+struct TriTma {
+  int ax0, ay0, adx, ady;   // map coordinates of A(0, 0) of batch 0, and the batch step
+  int bx0, by0, bdx, bdy;   // the same for B(0, 0)
+};
+
+// MN-major 128-byte-swizzled offset of (mn, k) in one split (64-wide boxes).
+__device__ __forceinline__ uint32_t mn_off(int mn, int k) {
+  return (uint32_t)((mn >> 6) * TS_BOX + (k >> 3) * 1024 + (k & 7) * 128 +
+                    ((((mn & 63) >> 3) ^ (k & 7)) << 4) + (mn & 7) * 2);
+}
+
+__global__ void __launch_bounds__(T_THREADS, 1)
+    trigemm_tma_kernel(const __grid_constant__ CUtensorMap mapA,
+                       const __grid_constant__ CUtensorMap mapB, TriArgs g, TriTma tt) {
+  if (g.info && *g.info != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* fst = smem;                              // fp32 ring
+  uint8_t* bst = smem + TNF * TF_STAGE;             // bf16 ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TNF * TF_STAGE + TNS * TS_STAGE);
+  // ffull[3] fempty[3] bfull[2] bempty[2] acc
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TNF + 2 * TNS + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto ffull = [&](int i) { return smem_u32(&bars[i]); };
+  auto fempty = [&](int i) { return smem_u32(&bars[TNF + i]); };
+  auto bfull = [&](int i) { return smem_u32(&bars[2 * TNF + i]); };
+  auto bempty = [&](int i) { return smem_u32(&bars[2 * TNF + TNS + i]); };
+  const uint32_t accbar = smem_u32(&bars[2 * TNF + 2 * TNS]);
+
+  const int bid = blockIdx.x;
+  int tm, tn;
+  if (g.b_upper) {
+    tn = g.tiles_n - 1 - bid / g.tiles_m;
+    tm = bid % g.tiles_m;
+  } else {
+    tm = bid / g.tiles_n;
+    tn = bid % g.tiles_n;
+  }
+  const int m0 = tm * BM, n0 = tn * BN;
+  const int kbeg = g.a_upper ? m0 : 0;
+  int kend = g.K;
+  if (g.b_upper && n0 + BN < kend) kend = n0 + BN;
+  const int nchunks = kend > kbeg ? (kend - kbeg + TBK - 1) / TBK : 0;
+  const int pair = blockIdx.y;
+  float* C = g.C + (int64_t)pair * g.strideC;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < TNF; ++i) {
+      mbar_init(ffull(i), 1);
+      mbar_init(fempty(i), 8);
+    }
+    for (int i = 0; i < TNS; ++i) {
+      mbar_init(bfull(i), 8);
+      mbar_init(bempty(i), 1);
+    }
+    mbar_init(accbar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 8) {
+    bool ok = true;
+    for (int s = 0; s < nchunks; ++s) {
+      const int fs = s % TNF, fu = s / TNF, bs = s & 1, bu = s >> 1;
+      const int kc = kbeg + s * TBK;
+      if (!mbar_wait(ffull(fs), fu & 1)) { ok = false; break; }
+      const uint8_t* F = fst + fs * TF_STAGE;
+      // A: m groups 4 (4 warp + t), k = lane
+      float av[4][4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          av[t][i] = *reinterpret_cast<const float*>(F + sw128_f32(16 * warp + 4 * t + i, lane));
+      // B: k rows warp + 8 t, n = 4 lane .. +3
+      float4 bv[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int k = warp + 8 * t, nn = 4 * lane;
+        bv[t] = *reinterpret_cast<const float4*>(F + TF_A + (nn >> 5) * TF_BBOX + sw128_f32(k, nn & 31));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(fempty(fs));
+      if (bu > 0 && !mbar_wait(bempty(bs), (bu - 1) & 1)) { ok = false; break; }
+      uint8_t* Sb = bst + bs * TS_STAGE;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int mm = 16 * warp + 4 * t;           // tile-local m of av[t][0]
+        const int k = kc + lane;                     // global k
+        float4 v = make_float4(av[t][0], av[t][1], av[t][2], av[t][3]);
+        const int row = m0 + mm;
+        const bool kin = k < g.K;
+        if (!(kin && row + 0 < g.M && (!g.a_upper || k >= row + 0))) v.x = 0.f;
+        if (!(kin && row + 1 < g.M && (!g.a_upper || k >= row + 1))) v.y = 0.f;
+        if (!(kin && row + 2 < g.M && (!g.a_upper || k >= row + 2))) v.z = 0.f;
+        if (!(kin && row + 3 < g.M && (!g.a_upper || k >= row + 3))) v.w = 0.f;
+        split_store4(Sb, mn_off(mm, lane), TS_SPLIT, v);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int kl = warp + 8 * t, nn = 4 * lane;
+        const int k = kc + kl, col = n0 + nn;
+        float4 v = bv[t];
+        const bool kin = k < g.K;
+        if (!(kin && col + 0 < g.N && (!g.b_upper || k <= col + 0))) v.x = 0.f;
+        if (!(kin && col + 1 < g.N && (!g.b_upper || k <= col + 1))) v.y = 0.f;
+        if (!(kin && col + 2 < g.N && (!g.b_upper || k <= col + 2))) v.z = 0.f;
+        if (!(kin && col + 3 < g.N && (!g.b_upper || k <= col + 3))) v.w = 0.f;
+        split_store4(Sb + 3 * TS_SPLIT, mn_off(nn, kl), TS_SPLIT, v);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bfull(bs));
+    }
+    // epilogue (as in the generic kernel)
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && nchunks > 0) {
+      int got = 1;
+      if (lane == 0) got = mbar_wait(accbar, 0) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+    }
+    const int q = warp & 3, hc = warp >> 2;
+    const int r = 32 * q + lane;
+    float* cst = reinterpret_cast<float*>(smem);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
+        if (nchunks > 0) {
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 64 * hc + 32 * cc, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = 0u;
+        }
+        float* dst = cst + r * C_LD + 64 * hc + 32 * cc;
+#pragma unroll
+        for (int t = 0; t < 32; t += 4)
+          *reinterpret_cast<float4*>(dst + t) =
+              make_float4(g.alpha * __uint_as_float(v[t]), g.alpha * __uint_as_float(v[t + 1]),
+                          g.alpha * __uint_as_float(v[t + 2]), g.alpha * __uint_as_float(v[t + 3]));
+      }
+    }
+    named_barrier(1, CV_THREADS);
+    if (ok) {
+      const int col = n0 + 4 * lane;
+      const int valid = g.N - col;
+#pragma unroll 4
+      for (int rr = warp; rr < BM; rr += 8) {
+        const int row = m0 + rr;
+        if (row >= g.M || valid <= 0) continue;
+        const float4 x = *reinterpret_cast<const float4*>(cst + rr * C_LD + 4 * lane);
+        float* out = C + (int64_t)row * g.ldc + col;
+        if (valid >= 4 && g.vecC) {
+          *reinterpret_cast<float4*>(out) = x;
+        } else {
+          out[0] = x.x;
+          if (valid > 1) out[1] = x.y;
+          if (valid > 2) out[2] = x.z;
+          if (valid > 3) out[3] = x.w;
+        }
+      }
+    }
+  } else if (warp == 8) {
+    if (lane == 0) {
+      const int ax = tt.ax0 + pair * tt.adx, ay = tt.ay0 + pair * tt.ady;
+      const int bx = tt.bx0 + pair * tt.bdx, by = tt.by0 + pair * tt.bdy;
+      for (int s = 0; s < nchunks; ++s) {
+        const int fs = s % TNF, fu = s / TNF;
+        if (fu > 0 && !mbar_wait(fempty(fs), (fu - 1) & 1)) break;
+        const int kc = kbeg + s * TBK;
+        const uint32_t F = smem_u32(fst + fs * TF_STAGE);
+        mbar_arrive_expect_tx(ffull(fs), TF_STAGE);
+        tma_load_2d(F, &mapA, ffull(fs), ax + kc, ay + m0);
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j)
+          tma_load_2d(F + TF_A + j * TF_BBOX, &mapB, ffull(fs), bx + n0 + 32 * j, by + kc);
+      }
+    }
+    __syncwarp();
+  } else {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, true, true);
+      for (int s = 0; s < nchunks; ++s) {
+        const int bs = s & 1, bu = s >> 1;
+        if (!mbar_wait(bfull(bs), bu & 1)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(bst + bs * TS_STAGE), sb = sa + 3 * TS_SPLIT;
+#pragma unroll
+        for (int kk = 0; kk < TBK / 16; ++kk) {
+#pragma unroll
+          for (int t = 0; t < 6; ++t) {
+            // split pairs (a, b) with a + b <= 2: hh, hm, mh, hl, lh, mm
+            const int pa = (t == 2 || t == 5) ? 1 : (t == 4 ? 2 : 0);
+            const int pb = (t == 1 || t == 5) ? 1 : (t == 3 ? 2 : 0);
+            const uint64_t da = smem_desc_sw128(sa + pa * TS_SPLIT + kk * 2048, TS_BOX, 1024);
+            const uint64_t db = smem_desc_sw128(sb + pb * TS_SPLIT + kk * 2048, TS_BOX, 1024);
+            mma_bf16(tmem, da, db, idesc, (s > 0 || kk > 0 || t > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(bempty(bs));
+      }
+      if (nchunks > 0) mma_commit(accbar);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 }  // namespace
 
 cudaError_t status_fetch_trigemm(int* out, cudaStream_t s) {
@@ -346,9 +584,39 @@ kronq_status trigemm_tc(const TriGemm& t, cudaStream_t s) {
   g.vecB = vec_ok(t.B, t.ldb, t.strideB) ? 1 : 0;
   g.vecC = vec_ok(t.C, t.ldc, t.strideC) ? 1 : 0;
   g.info = t.info;
+  dim3 grid((unsigned)(g.tiles_m * g.tiles_n), (unsigned)t.batch);
+  // TMA path: 16-byte row strides and origins, x coordinates on 4 floats.
+  TriTma tt;
+  CUtensorMap mA, mB;
+  auto origin = [](const float* hold, int64_t ld, const float* p, int64_t stride, int& x0, int& y0,
+                   int& dx, int& dy) {
+    const int64_t off = p - hold;
+    if (off < 0 || ld <= 0) return false;
+    x0 = (int)(off % ld);
+    y0 = (int)(off / ld);
+    dx = (int)(stride % ld);
+    dy = (int)(stride / ld);
+    return (x0 % 4) == 0 && (dx % 4) == 0 && stride >= 0;
+  };
+  bool use_tma = t.holdA && t.holdB && (t.lda % 4) == 0 && (t.ldb % 4) == 0 &&
+                 aligned(t.holdA, 16) && aligned(t.holdB, 16) &&
+                 origin(t.holdA, t.lda, t.A, t.batch > 1 ? t.strideA : 0, tt.ax0, tt.ay0, tt.adx, tt.ady) &&
+                 origin(t.holdB, t.ldb, t.B, t.batch > 1 ? t.strideB : 0, tt.bx0, tt.by0, tt.bdx, tt.bdy);
+  if (use_tma) {
+    use_tma = tma_map_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, t.holdA, t.holdA_cols, t.holdA_rows,
+                         t.lda, 32, BM) &&
+              tma_map_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, t.holdB, t.holdB_cols, t.holdB_rows,
+                         t.ldb, 32, TBK);
+  }
+  if (use_tma) {
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(&trigemm_tma_kernel), T_SMEM);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(trigemm tma)");
+    trigemm_tma_kernel<<<grid, T_THREADS, T_SMEM, s>>>(mA, mB, g, tt);
+    KQ_LAUNCH_CHECK("trigemm_tma_kernel");
+    return KRONQ_OK;
+  }
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(&trigemm_tc_kernel), SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(trigemm)");
-  dim3 grid((unsigned)(g.tiles_m * g.tiles_n), (unsigned)t.batch);
   trigemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(g);
   KQ_LAUNCH_CHECK("trigemm_tc_kernel");
   return KRONQ_OK;
