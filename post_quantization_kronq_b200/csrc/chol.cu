@@ -63,14 +63,13 @@ __global__ void zero_info_kernel(int* info) { *info = 0; }
 // Diagonal step of the blocked factorisation: one 64 x 64 block A_JJ,
 // factored and inverted in shared memory by 256 threads, then the panel
 // rows above it.  The block is handled as four 16 x 16 leaves (bottom-right
-// first); each leaf is factored and inverted by one warp in registers (lane
-// c holds column c of the symmetric leaf, pivots are shuffled), the rows
-// above the leaf are multiplied by U_leaf^T, and a rank-16 update follows.
-// U_JJ is assembled from the leaf inverses with the recursive formula.
+// first); each leaf is factored in the registers of one thread, the rows
+// above the leaf are solved against R_leaf, and a rank-16 update follows.
+// Then four threads invert the leaves at once and U_JJ is assembled from
+// them with the recursive two-block formula.
 
 constexpr int LF = 16;                       // leaf width
 constexpr int PR = 32;                       // panel rows per chunk
-constexpr unsigned FULL = 0xffffffffu;
 
 struct alignas(16) DiagSmem {
   union {
@@ -79,7 +78,6 @@ struct alignas(16) DiagSmem {
   } x;
   float u[NB][NB + 1];        // U_JJ (upper, zero below)
   union {
-    float ulT[LF][LF];        // U_leaf^T of the current leaf
     float tb[32][33];         // products R12 U22 while U_JJ is assembled
     float ach[PR][NB + 1];    // a chunk of panel rows
   } y;
@@ -87,61 +85,67 @@ struct alignas(16) DiagSmem {
   int bad;
 };
 
-// Factor and invert the leaf at offset o (one warp).  Writes R_leaf into a,
-// U_leaf into u and its transpose into ulT, and 1 / R_kk into rinv.
-__device__ __forceinline__ void leaf_factor_invert(DiagSmem& S, int o, int lane) {
-  const int c = lane & (LF - 1);
-  float col[LF];
+// Factor the leaf at offset o in the registers of one thread (its upper
+// triangle, 136 values; the last pivot first, each pivot scaled by rsqrt).
+// Writes R_leaf into a and 1 / R_kk into rinv; records the first
+// non-positive pivot in S.bad.  One thread keeps the whole dependency chain
+// in registers, which is several times faster than sharing it across a warp.
+__device__ __forceinline__ void leaf_factor(DiagSmem& S, int o) {
+  float r[LF][LF];
 #pragma unroll
-  for (int i = 0; i < LF; ++i) col[i] = (i <= c) ? S.x.a[o + i][o + c] : S.x.a[o + c][o + i];
-  float mypiv = 1.f;
-  bool badp = false;
+  for (int i = 0; i < LF; ++i)
+#pragma unroll
+    for (int j = i; j < LF; ++j) r[i][j] = S.x.a[o + i][o + j];
   int badk = -1;
 #pragma unroll
   for (int K = LF - 1; K >= 0; --K) {
-    const float piv = __shfl_sync(FULL, col[K], K);
-    if (!(piv > 0.f) || !isfinite(piv)) {
-      if (!badp) badk = K;
-      badp = true;
-    }
-    if (c == K) mypiv = piv;
-    const float f = col[K] / piv;  // a[c][K] / pivot
+    const float piv = r[K][K];
+    if ((!(piv > 0.f) || !isfinite(piv)) && badk < 0) badk = K;
+    const float rs = rsqrtf(piv);
+    S.rinv[o + K] = rs;
+    r[K][K] = piv * rs;
 #pragma unroll
-    for (int i = 0; i < K; ++i) {
-      const float aik = __shfl_sync(FULL, col[i], K);
-      if (c < K) col[i] = fmaf(-aik, f, col[i]);
-    }
+    for (int i = 0; i < K; ++i) r[i][K] *= rs;
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+#pragma unroll
+      for (int i = 0; i <= j; ++i) r[i][j] = fmaf(-r[i][K], r[j][K], r[i][j]);
   }
-  if (lane == 0 && badp && S.bad == 0) S.bad = o + badk + 1;
-  // R[c][c] = sqrt(pivot), R[i][c] = a[i][c] / R[c][c] (values at pivot time)
-  const float rk = sqrtf(mypiv);
-  const float rin = 1.f / rk;
+  if (badk >= 0 && S.bad == 0) S.bad = o + badk + 1;
 #pragma unroll
-  for (int i = 0; i < LF; ++i) col[i] = (i < c) ? col[i] * rin : (i == c ? rk : 0.f);
-  // U_leaf = R_leaf^-1 by rows: lane i forms row i from U R = I.
-  const int i = c;
-  float urow[LF];
+  for (int i = 0; i < LF; ++i)
 #pragma unroll
-  for (int cc = 0; cc < LF; ++cc) {
-    const float rcc = __shfl_sync(FULL, rin, cc);
-    float s0 = 0.f, s1 = 0.f;
+    for (int j = i; j < LF; ++j) S.x.a[o + i][o + j] = r[i][j];
+}
+
+// U_leaf = R_leaf^-1 for the leaf at offset o, in place in the registers of
+// one thread: column j of U is -U[0:j, 0:j] R[0:j, j] / R_jj, the leading
+// block already inverted.  Reads R from a and 1 / R_kk from rinv, writes u.
+__device__ __forceinline__ void leaf_invert(DiagSmem& S, int o) {
+  float r[LF][LF];
 #pragma unroll
-    for (int k = 0; k < cc; ++k) {
-      const float rkc = __shfl_sync(FULL, col[k], cc);
-      if (k & 1) s1 = fmaf(urow[k], rkc, s1);
-      else s0 = fmaf(urow[k], rkc, s0);
+  for (int i = 0; i < LF; ++i)
+#pragma unroll
+    for (int j = i; j < LF; ++j) r[i][j] = S.x.a[o + i][o + j];
+#pragma unroll
+  for (int j = 0; j < LF; ++j) {
+    const float ujj = S.rinv[o + j];
+    float t[LF];
+#pragma unroll
+    for (int i = 0; i < j; ++i) {
+      float acc = 0.f;
+#pragma unroll
+      for (int k = i; k < j; ++k) acc = fmaf(r[i][k], r[k][j], acc);
+      t[i] = acc;
     }
-    urow[cc] = (cc < i) ? 0.f : (cc == i ? rcc : -(s0 + s1) * rcc);
-  }
-  if (lane < LF) {
 #pragma unroll
-    for (int k = 0; k < LF; ++k) {
-      if (k <= c) S.x.a[o + k][o + c] = col[k];
-      S.u[o + i][o + k] = urow[k];
-      S.y.ulT[k][i] = urow[k];
-    }
-    S.rinv[o + c] = rin;
+    for (int i = 0; i < j; ++i) r[i][j] = -t[i] * ujj;
+    r[j][j] = ujj;
   }
+#pragma unroll
+  for (int i = 0; i < LF; ++i)
+#pragma unroll
+    for (int j = i; j < LF; ++j) S.u[o + i][o + j] = r[i][j];
 }
 
 // Loads PR panel rows [r0, r0 + PR) of columns J into registers (8 per thread).
@@ -197,33 +201,32 @@ __global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, in
   __syncthreads();
 
   for (int o = NB - LF; o >= 0; o -= LF) {
-    if (warp == 0) leaf_factor_invert(S, o, lane);
+    if (tid == 0) leaf_factor(S, o);
     __syncthreads();
     if (S.bad) {
       if (tid == 0 && blockIdx.x == 0) *info = (int)(j0 + S.bad);
       return;  // uniform: read after the barrier
     }
     if (o == 0) break;
-    // rows i < o of the leaf's columns: R[i, leaf] = A[i, leaf] U_leaf^T
-    {
-      const int i = tid >> 2, g = (tid & 3) * 4;
-      float o4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (i < o) {
+    // rows i < o of the leaf's columns: solve x R_leaf^T = A[i, leaf], last
+    // column first (one thread per row)
+    if (tid < o) {
+      const int i = tid;
+      float x[LF];
 #pragma unroll
-        for (int l = 0; l < LF; ++l) {
-          const float al = S.x.a[i][o + l];
-          const float4 w = *reinterpret_cast<const float4*>(&S.y.ulT[l][g]);
-          o4[0] = fmaf(al, w.x, o4[0]);
-          o4[1] = fmaf(al, w.y, o4[1]);
-          o4[2] = fmaf(al, w.z, o4[2]);
-          o4[3] = fmaf(al, w.w, o4[3]);
+      for (int k = 0; k < LF; ++k) x[k] = S.x.a[i][o + k];
+#pragma unroll
+      for (int k = LF - 1; k >= 0; --k) {
+        float s0 = x[k], s1 = 0.f;
+#pragma unroll
+        for (int l = k + 1; l < LF; ++l) {
+          if ((l - k) & 1) s0 = fmaf(-S.x.a[o + k][o + l], x[l], s0);
+          else s1 = fmaf(-S.x.a[o + k][o + l], x[l], s1);
         }
+        x[k] = (s0 + s1) * S.rinv[o + k];
       }
-      __syncthreads();
-      if (i < o) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) S.x.a[i][o + g + q] = o4[q];
-      }
+      for (int k = 0; k < LF; ++k) S.x.a[i][o + k] = x[k];
     }
     __syncthreads();
     // rank-16 update of the leading o x o upper triangle
@@ -244,6 +247,8 @@ __global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, in
     __syncthreads();
   }
 
+  if (lane == 0 && warp < NB / LF) leaf_invert(S, warp * LF);
+  __syncthreads();
   // U_JJ from the leaf inverses: for pairs of diagonal blocks of size s,
   // U12 = -U11 (R12 U22).  s = 16: two pairs, two outputs per thread.
   {
