@@ -3,10 +3,12 @@
 // KronQ README intro (extends GPTQ/GPTAQ) and "Reproduce from scratch"
 // (--w_bits --w_groupsize --w_asym).  Rows of W~ are independent once U is
 // known, so the in-block sweep runs one warp per pair of rows with no
-// block-wide synchronisation: lane l holds columns 4l..4l+3 of the 128-column
-// block, the owner lane of column j quantizes it, forms the scaled error
-// e = (w - deq) / U_jj, broadcasts e with a shuffle and every lane applies the
-// rank-1 update to its later columns.  All arithmetic of the sweep is single
+// block-wide synchronisation: eight lanes per row, lane q holds columns
+// 16q..16q+15 of the 128-column block.  The owner lane of a 16-column quarter
+// quantizes its columns one after the other, forming the scaled errors
+// e = (w - deq) / U_jj and updating its own later columns; then the sixteen
+// errors are shuffled to the row's other lanes, which apply them to their
+// (later) columns in column order.  All arithmetic of the sweep is single
 // float32 operations (multiply and subtract not fused; the per-column
 // divisions by the group scale and by U_jj are multiplications by their
 // correctly rounded reciprocals), so the result is reproducible bit for bit.
@@ -89,11 +91,13 @@ __device__ __forceinline__ int ucol(int c) { return c + 4 * (c >> 4); }
 // One block of 128 columns.  Eight lanes per row: lane q holds the row's
 // columns 16q .. 16q+15 in registers (v[]), so every step of the sequential
 // column loop is register arithmetic with static indices (the unrolled
-// 16-step body stays small enough for the instruction cache).  At column j
-// the lane holding it quantizes, forms e = (w - deq) / U_jj and shuffles e
-// to the other seven lanes of the row; every lane then applies
-// v[c] -= e * U[j][c] to its columns c > j (multiply, then subtract: the
-// operation order of the float32 reference).
+// 16-step body stays small enough for the instruction cache).  For each
+// quarter, the lane holding it quantizes its columns in order (forming
+// e = (w - deq) / U_jj and applying v[c] -= e * U[j][c] to its own later
+// columns), with no shuffle inside that dependency chain; the sixteen
+// errors are then shuffled to the later lanes at once.  Every update is a
+// multiply followed by a subtract, in ascending j per element: the
+// operation order of the float32 reference.
 template <bool SMALLG>
 __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
   const SweepDesc& d = a.d;
@@ -209,34 +213,73 @@ __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
     // Groups of 16 or more columns can only start at a lane boundary.
     if (!SMALLG && inblock_groups && qo * QW < bw && ((qo * QW) & gmask) == 0)
       group_start(v, qo * QW, bw, q, d, live, r, g0 + ((qo * QW) >> gshift), sc, zp, isc);
+    // The owner lane sweeps its sixteen columns alone (no cross-lane step
+    // inside the sequential chain) ...
+    if (mine) {
+      const float* urow0 = Us + q * (QW + 4);
 #pragma unroll
-    for (int c = 0; c < QW; ++c) {
-      const int j = qo * QW + c;
-      if (j >= bw) break;
-      if (SMALLG && (j & gmask) == 0) group_start(v, j, bw, q, d, live, r, g0 + (j >> gshift), sc, zp, isc);
-      float e = 0.f;
-      if (mine) {
+      for (int c = 0; c < QW; ++c) {
+        const int j = qo * QW + c;
+        if (j >= bw) break;
+        if (SMALLG && (j & gmask) == 0) {
+          // a group of fewer than 16 columns lies inside this lane
+          float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+          for (int cc = c; cc < QW; ++cc)
+            if (cc < c + d.group && qo * QW + cc < bw) {
+              lo = fminf(lo, v[cc]);
+              hi = fmaxf(hi, v[cc]);
+            }
+          grid_from_range(lo, hi, d.bits, d.asym, sc, zp);
+          isc = __frcp_rn(sc);
+          if (live) {
+            const int64_t gi = g0 + (j >> gshift);
+            d.scales[r * d.ngroups + gi] = sc;
+            d.zeros[r * d.ngroups + gi] = zp;
+          }
+        }
         const float w = v[c];
         // division by scale and by U_jj as multiplication by the correctly
         // rounded reciprocals (the float32 schedule of this library)
         float qv = __fadd_rn(rintf(__fmul_rn(w, isc)), zp);
         qv = fminf(fmaxf(qv, 0.f), maxq);
         const float deq = __fmul_rn(sc, __fsub_rn(qv, zp));
-        e = __fmul_rn(__fsub_rn(w, deq), iu[j]);
+        const float e = __fmul_rn(__fsub_rn(w, deq), iu[j]);
         v[c] = deq;
         ev[c] = e;
         code[c >> 2] |= ((uint32_t)qv & 0xFFu) << (8 * (c & 3));
+        const float* urow = urow0 + j * US_LD;
+#pragma unroll
+        for (int c4 = 0; c4 < QW; c4 += 4) {
+          if (c4 + 3 <= c) continue;
+          const float4 u4 = *reinterpret_cast<const float4*>(urow + c4);
+          const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            if (c4 + t > c) v[c4 + t] = __fsub_rn(v[c4 + t], __fmul_rn(e, uu[t]));
+        }
       }
-      e = __shfl_sync(0xffffffffu, e, src_base + qo);
-      const float* urow = Us + j * US_LD + q * (QW + 4);
+    }
+    // ... then its sixteen errors go to the other lanes of the row, which
+    // apply them to their columns in ascending column order (the same
+    // operation sequence per element as a column-by-column update).
+    float eq[QW];
 #pragma unroll
-      for (int c4 = 0; c4 < QW; c4 += 4) {
-        const float4 u4 = *reinterpret_cast<const float4*>(urow + c4);
-        const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+    for (int c = 0; c < QW; ++c) eq[c] = __shfl_sync(0xffffffffu, ev[c], src_base + qo);
+    if (all_later) {
+      const float* urow0 = Us + q * (QW + 4);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int cc = c4 + t;
-          if (all_later || (mine && cc > c)) v[cc] = __fsub_rn(v[cc], __fmul_rn(e, uu[t]));
+      for (int c = 0; c < QW; ++c) {
+        const int j = qo * QW + c;
+        if (j >= bw) break;
+        const float* urow = urow0 + j * US_LD;
+#pragma unroll
+        for (int c4 = 0; c4 < QW; c4 += 4) {
+          const float4 u4 = *reinterpret_cast<const float4*>(urow + c4);
+          v[c4 + 0] = __fsub_rn(v[c4 + 0], __fmul_rn(eq[c], u4.x));
+          v[c4 + 1] = __fsub_rn(v[c4 + 1], __fmul_rn(eq[c], u4.y));
+          v[c4 + 2] = __fsub_rn(v[c4 + 2], __fmul_rn(eq[c], u4.z));
+          v[c4 + 3] = __fsub_rn(v[c4 + 3], __fmul_rn(eq[c], u4.w));
         }
       }
     }
