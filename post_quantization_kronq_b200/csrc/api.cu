@@ -419,14 +419,15 @@ kronq_status kronq_unpack(const uint32_t* in, int64_t m, int64_t n, int bits, ui
 
 kronq_status kronq_device_status(int* out, kronq_stream_t s) {
   if (!out) return fail(KRONQ_ERR_INVALID_ARG, "device_status: out is NULL");
-  int v[4] = {0, 0, 0, 0};
+  int v[5] = {0, 0, 0, 0, 0};
   cudaError_t e = status_fetch_syrk(&v[0], as_stream(s));
   if (e == cudaSuccess) e = status_fetch_trailing(&v[1], as_stream(s));
   if (e == cudaSuccess) e = status_fetch_schur(&v[2], as_stream(s));
   if (e == cudaSuccess) e = status_fetch_trigemm(&v[3], as_stream(s));
+  if (e == cudaSuccess) e = status_fetch_chol(&v[4], as_stream(s));
   if (e != cudaSuccess) return cuda_fail(e, "device_status");
   *out = 0;
-  for (int i = 0; i < 4 && *out == 0; ++i) *out = v[i];
+  for (int i = 0; i < 5 && *out == 0; ++i) *out = v[i];
   return KRONQ_OK;
 }
 

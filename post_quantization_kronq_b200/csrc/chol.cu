@@ -6,7 +6,9 @@
 // R upper triangular (eliminating from the last index down), and then
 // U = R^-1, since A^-1 = R^-T R^-1 = U^T U.  That is 2 n^3 / 3 flops in total.
 //
-// Blocked with nb = 64, bottom-right first.  For each diagonal block J:
+// Blocked with nb = 64, bottom-right first.  For n > 256 with 16-byte rows
+// the whole chain is one persistent kernel (chol_persistent_kernel below,
+// with a one-step look-ahead); otherwise, for each diagonal block J:
 //   diag_panel_kernel  factor A_JJ = R_JJ R_JJ^T (itself blocked by 16),
 //                      invert it, U_JJ = R_JJ^-1, and form the panel
 //                      R[0:j0, J] = A[0:j0, J] U_JJ^T (every CTA factors the
@@ -23,6 +25,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "schur_tile.cuh"
 
 namespace kq {
 namespace {
@@ -90,7 +93,8 @@ struct alignas(16) DiagSmem {
 // Writes R_leaf into a and 1 / R_kk into rinv; records the first
 // non-positive pivot in S.bad.  One thread keeps the whole dependency chain
 // in registers, which is several times faster than sharing it across a warp.
-__device__ __forceinline__ void leaf_factor(DiagSmem& S, int o) {
+template <class SM>
+__device__ __forceinline__ void leaf_factor(SM& S, int o) {
   float r[LF][LF];
 #pragma unroll
   for (int i = 0; i < LF; ++i)
@@ -121,7 +125,8 @@ __device__ __forceinline__ void leaf_factor(DiagSmem& S, int o) {
 // U_leaf = R_leaf^-1 for the leaf at offset o, in place in the registers of
 // one thread: column j of U is -U[0:j, 0:j] R[0:j, j] / R_jj, the leading
 // block already inverted.  Reads R from a and 1 / R_kk from rinv, writes u.
-__device__ __forceinline__ void leaf_invert(DiagSmem& S, int o) {
+template <class SM>
+__device__ __forceinline__ void leaf_invert(SM& S, int o) {
   float r[LF][LF];
 #pragma unroll
   for (int i = 0; i < LF; ++i)
@@ -148,65 +153,16 @@ __device__ __forceinline__ void leaf_invert(DiagSmem& S, int o) {
     for (int j = i; j < LF; ++j) S.u[o + i][o + j] = r[i][j];
 }
 
-// Loads PR panel rows [r0, r0 + PR) of columns J into registers (8 per thread).
-__device__ __forceinline__ void load_chunk(const float* H, int64_t n, int64_t j0, int nb,
-                                           int64_t r0, bool vec4, float (&v)[8]) {
-  const int t = threadIdx.x;
-  const int r = t >> 3, seg = (t & 7) * 8;
-  const int64_t i = r0 + r;
-  const float* src = H + i * n + j0 + seg;
-  if (i < j0 && vec4 && seg + 8 <= nb) {
-    const float4 p = *reinterpret_cast<const float4*>(src);
-    const float4 q = *reinterpret_cast<const float4*>(src + 4);
-    v[0] = p.x; v[1] = p.y; v[2] = p.z; v[3] = p.w;
-    v[4] = q.x; v[5] = q.y; v[6] = q.z; v[7] = q.w;
-  } else {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) v[q] = (i < j0 && seg + q < nb) ? src[q] : 0.f;
-  }
-}
-
-// Factor the diagonal block A_JJ = R_JJ R_JJ^T (reverse order), invert it,
-// and form the panel above it, R[i, J] = A[i, J] U_JJ^T.  Every CTA factors
-// the (small) block itself, so no extra launch sits on the sequential path;
-// CTA 0 stages U_JJ (64 x 64, row-major) at stage[j0 * 64].  A short block
-// (nb < 64) is padded with the identity.  The panel rows are also written
-// as bf16 hi/mid/lo splits for the tensor-core Schur update.
-__global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, int64_t j0, int nb,
-                                                         int* info, __nv_bfloat16* splits,
-                                                         float* stage, int vec4) {
-  if (*info != 0) return;
-  __shared__ DiagSmem S;
+// Factors the 64 x 64 block in S.x.a (upper triangle; S.u zero, S.bad zero)
+// into R_JJ (in S.x.a) and U_JJ = R_JJ^-1 (in S.u).  Returns false
+// (uniformly) at a non-positive pivot, S.bad = its index + 1.  256 threads.
+template <class SM>
+__device__ bool factor_invert_block(SM& S) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  {
-    const int tx = tid & 63, ty = tid >> 6;
-    float x[NB / 4];
-#pragma unroll
-    for (int sl = 0; sl < NB / 4; ++sl) {  // all sixteen loads in flight
-      const int r = 4 * sl + ty;
-      x[sl] = (r <= tx && tx < nb) ? H[(j0 + r) * n + j0 + tx] : 0.f;
-    }
-#pragma unroll
-    for (int sl = 0; sl < NB / 4; ++sl) {
-      const int r = 4 * sl + ty;
-      S.x.a[r][tx] = (tx < nb) ? x[sl] : (r == tx ? 1.f : 0.f);
-      S.u[r][tx] = 0.f;
-    }
-  }
-  // the first chunk of panel rows is fetched while the block is factored
-  float pv[8];
-  const int64_t chunk0 = (int64_t)blockIdx.x * PR;
-  load_chunk(H, n, j0, nb, chunk0, vec4 != 0, pv);
-  if (tid == 0) S.bad = 0;
-  __syncthreads();
-
   for (int o = NB - LF; o >= 0; o -= LF) {
     if (tid == 0) leaf_factor(S, o);
     __syncthreads();
-    if (S.bad) {
-      if (tid == 0 && blockIdx.x == 0) *info = (int)(j0 + S.bad);
-      return;  // uniform: read after the barrier
-    }
+    if (S.bad) return false;  // uniform: read after the barrier
     if (o == 0) break;
     // rows i < o of the leaf's columns: solve x R_leaf^T = A[i, leaf], last
     // column first (one thread per row)
@@ -299,26 +255,85 @@ __global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, in
     for (int q = 0; q < 4; ++q) S.u[r][32 + c + q] = -v[q];
     __syncthreads();
   }
+  return true;
+}
+
+// Loads PR panel rows [r0, r0 + PR) of columns J into registers (8 per thread).
+__device__ __forceinline__ void load_chunk(const float* H, int64_t n, int64_t j0, int nb,
+                                           int64_t r0, bool vec4, float (&v)[8]) {
+  const int t = threadIdx.x;
+  const int r = t >> 3, seg = (t & 7) * 8;
+  const int64_t i = r0 + r;
+  const float* src = H + i * n + j0 + seg;
+  if (i < j0 && vec4 && seg + 8 <= nb) {
+    const float4 p = *reinterpret_cast<const float4*>(src);
+    const float4 q = *reinterpret_cast<const float4*>(src + 4);
+    v[0] = p.x; v[1] = p.y; v[2] = p.z; v[3] = p.w;
+    v[4] = q.x; v[5] = q.y; v[6] = q.z; v[7] = q.w;
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = (i < j0 && seg + q < nb) ? src[q] : 0.f;
+  }
+}
+
+// Factor the diagonal block A_JJ = R_JJ R_JJ^T (reverse order), invert it,
+// and form the panel above it, R[i, J] = A[i, J] U_JJ^T.  Every CTA factors
+// the (small) block itself, so no extra launch sits on the sequential path;
+// CTA 0 stages U_JJ (64 x 64, row-major) at stage[j0 * 64].  A short block
+// (nb < 64) is padded with the identity.  The panel rows are also written
+// as bf16 hi/mid/lo splits for the tensor-core Schur update.
+// The diagonal step of block J (rows/columns j0 .. j0 + nb) by CTA cta of
+// ncta: returns false (uniformly over the CTA) when a pivot is not
+// positive, after CTA 0 has recorded info.  256 threads.
+__device__ bool diag_step(DiagSmem& S, float* H, int64_t n, int64_t j0, int nb, int* info,
+                          __nv_bfloat16* splits, float* stage, int vec4, int cta, int ncta) {
+  const int tid = threadIdx.x;
+  {
+    const int tx = tid & 63, ty = tid >> 6;
+    float x[NB / 4];
+#pragma unroll
+    for (int sl = 0; sl < NB / 4; ++sl) {  // all sixteen loads in flight
+      const int r = 4 * sl + ty;
+      x[sl] = (r <= tx && tx < nb) ? H[(j0 + r) * n + j0 + tx] : 0.f;
+    }
+#pragma unroll
+    for (int sl = 0; sl < NB / 4; ++sl) {
+      const int r = 4 * sl + ty;
+      S.x.a[r][tx] = (tx < nb) ? x[sl] : (r == tx ? 1.f : 0.f);
+      S.u[r][tx] = 0.f;
+    }
+  }
+  // the first chunk of panel rows is fetched while the block is factored
+  float pv[8];
+  const int64_t chunk0 = (int64_t)cta * PR;
+  load_chunk(H, n, j0, nb, chunk0, vec4 != 0, pv);
+  if (tid == 0) S.bad = 0;
+  __syncthreads();
+  if (!factor_invert_block(S)) {
+    if (tid == 0 && cta == 0) *info = (int)(j0 + S.bad);
+    return false;  // uniform: read after the barrier
+  }
   // U_JJ^T (over R_JJ, no longer needed); CTA 0 stages U_JJ.
   for (int t = tid; t < NB * NB; t += blockDim.x) {
     const int r = t >> 6, c = t & 63;
     S.x.ut[c][r] = S.u[r][c];
   }
-  if (blockIdx.x == 0) {
+  if (cta == 0) {
     float* dst = stage + j0 * NB;
     for (int t = tid; t < nb * NB; t += blockDim.x) dst[t] = S.u[t >> 6][t & 63];
   }
   // Panel rows, chunks of PR rows: R[i][c] = sum_k A[i][k] U[c][k].
   const int64_t plane = (int64_t)n * NB;
   const int rp = tid >> 4, c0 = (tid & 15) * 4;
-  for (int64_t r0 = chunk0; r0 < j0; r0 += (int64_t)gridDim.x * PR) {
-    if (r0 != chunk0) load_chunk(H, n, j0, nb, r0, vec4 != 0, pv);
+  for (int64_t r0 = chunk0; r0 < j0; r0 += (int64_t)ncta * PR) {
     {
       const int r = tid >> 3, seg = (tid & 7) * 8;
 #pragma unroll
       for (int q = 0; q < 8; ++q) S.y.ach[r][seg + q] = pv[q];
     }
     __syncthreads();
+    // the next chunk of this CTA is fetched while this one is multiplied
+    if (r0 + (int64_t)ncta * PR < j0) load_chunk(H, n, j0, nb, r0 + (int64_t)ncta * PR, vec4 != 0, pv);
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll 16
     for (int k = 0; k < NB; ++k) {
@@ -365,6 +380,177 @@ __global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, in
     }
     __syncthreads();  // ach is rewritten by the next chunk
   }
+  return true;
+}
+
+__global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, int64_t j0, int nb,
+                                                         int* info, __nv_bfloat16* splits,
+                                                         float* stage, int vec4) {
+  if (*info != 0) return;
+  __shared__ DiagSmem S;
+  diag_step(S, H, n, j0, nb, info, splits, stage, vec4, blockIdx.x, gridDim.x);
+}
+
+// ---------------------------------------------------------------------------
+// The diagonal step of the persistent kernel: as diag_step, but each
+// diagonal CTA handles its panel rows in chunks of 128 that arrive by
+// cp.async while the block is factored, and multiplies them by U_JJ^T with
+// 4 x 8 register tiles.
+constexpr int PRF = 128;   // panel rows per chunk
+
+struct alignas(16) DiagSmemP {
+  union {
+    float a[NB][NB + 1];      // A_JJ (upper) -> R_JJ
+  } x;
+  float u[NB][NB + 1];        // U_JJ (upper, zero below)
+  union {
+    float tb[32][33];         // products R12 U22 while U_JJ is assembled
+    float wk[NB][NB + 4];     // then U_JJ^T
+  } y;
+  float ach[PRF][NB + 4];     // panel rows A[i, J]
+  float rinv[NB];
+  int bad;
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Starts the copies of A[i, J] (columns j0 .. j0 + nb) of rows r0 .. r0 + PRF - 1
+// (zero beyond nb and in the rows from rend on).
+__device__ __forceinline__ void fetch_rows(DiagSmemP& S, const float* H, int64_t n, int64_t j0, int nb,
+                                           int64_t r0, int64_t rend) {
+  const int tid = threadIdx.x;
+#pragma unroll 4
+  for (int q = 0; q < PRF * 16 / 256; ++q) {
+    const int t = tid + 256 * q;
+    const int row = t >> 4, seg = t & 15;
+    const int64_t i = r0 + row;
+    const int c = 4 * seg;
+    int valid = nb - c;
+    valid = valid < 0 ? 0 : (valid > 4 ? 4 : valid);
+    if (i >= rend) valid = 0;
+    const float* src = (valid > 0) ? H + i * n + j0 + c : H;
+    cp_async16(&S.ach[row][c], src, 4 * valid);
+  }
+  cp_async_commit();
+}
+
+// acc[j][q] = sum_k ach[rg + 32 j][k] wk[k][8 cg + q] for the first NSL
+// 32-row slices.
+template <int NSL>
+__device__ __forceinline__ void panel_product(const DiagSmemP& S, int rg, int cg, float (&acc)[4][8]) {
+#pragma unroll 4
+  for (int k = 0; k < NB; ++k) {
+    const float4 w0 = *reinterpret_cast<const float4*>(&S.y.wk[k][8 * cg]);
+    const float4 w1 = *reinterpret_cast<const float4*>(&S.y.wk[k][8 * cg + 4]);
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int j = 0; j < NSL; ++j) {
+      const float av = S.ach[rg + 32 * j][k];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[j][q] = fmaf(av, wv[q], acc[j][q]);
+    }
+  }
+}
+
+__device__ bool diag_step_p(DiagSmemP& S, float* H, int64_t n, int64_t j0, int nb, int* info,
+                            __nv_bfloat16* splits, float* stage, int cta, int ncta) {
+  const int tid = threadIdx.x;
+  // this CTA's rows: an even share of 0 .. j0, in multiples of 32
+  const int64_t per = (((j0 + ncta - 1) / ncta + 31) / 32) * 32;
+  const int64_t rbeg = (int64_t)cta * per;
+  const int64_t rend = (rbeg + per < j0) ? rbeg + per : j0;
+  if (rbeg < rend) fetch_rows(S, H, n, j0, nb, rbeg, rend);
+  {
+    const int tx = tid & 63, ty = tid >> 6;
+    float x[NB / 4];
+#pragma unroll
+    for (int sl = 0; sl < NB / 4; ++sl) {  // all loads in flight
+      const int r = 4 * sl + ty;
+      x[sl] = (r <= tx && tx < nb) ? H[(j0 + r) * n + j0 + tx] : 0.f;
+    }
+#pragma unroll
+    for (int sl = 0; sl < NB / 4; ++sl) {
+      const int r = 4 * sl + ty;
+      S.x.a[r][tx] = (tx < nb) ? x[sl] : (r == tx ? 1.f : 0.f);
+      S.u[r][tx] = 0.f;
+    }
+  }
+  if (tid == 0) S.bad = 0;
+  __syncthreads();
+  if (!factor_invert_block(S)) {
+    if (tid == 0 && cta == 0) *info = (int)(j0 + S.bad);
+    return false;  // uniform: read after the barrier
+  }
+  // U^T and the staged U_JJ
+  for (int t = tid; t < NB * NB; t += blockDim.x) {
+    const int k = t >> 6, c = t & 63;
+    S.y.wk[k][c] = S.u[c][k];
+  }
+  if (cta == 0) {
+    float* dst = stage + j0 * NB;
+    for (int t = tid; t < nb * NB; t += blockDim.x) dst[t] = S.u[t >> 6][t & 63];
+  }
+  // Panel rows: R[i][c] = sum_k A[i][k] U[c][k]; thread: rows rg + 32 j
+  // (j < 4), columns 8 cg .. 8 cg + 7.
+  const int64_t plane = (int64_t)n * NB;
+  const int rg = tid >> 3, cg = tid & 7;
+  for (int64_t r0 = rbeg; r0 < rend; r0 += PRF) {
+    cp_async_wait_all();
+    __syncthreads();
+    float acc[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[j][q] = 0.f;
+    const int rows = (int)((rend - r0 < PRF) ? (rend - r0) : PRF);
+    // only the 32-row slices that hold rows of the panel (uniform branch)
+    const int nsl = (rows + 31) >> 5;
+    if (nsl == 4) panel_product<4>(S, rg, cg, acc);
+    else if (nsl == 3) panel_product<3>(S, rg, cg, acc);
+    else if (nsl == 2) panel_product<2>(S, rg, cg, acc);
+    else panel_product<1>(S, rg, cg, acc);
+    __syncthreads();                          // the rows are consumed
+    if (r0 + PRF < rend) fetch_rows(S, H, n, j0, nb, r0 + PRF, rend);
+    auto bits = [](__nv_bfloat162 v) { return *reinterpret_cast<const uint32_t*>(&v); };
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t i = r0 + rg + 32 * j;
+      if (i >= rend) continue;
+      float* row = H + i * n + j0 + 8 * cg;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c0 = 8 * cg + 4 * h;
+        const float* v = &acc[j][4 * h];
+        if (c0 + 4 <= nb) {
+          *reinterpret_cast<float4*>(row + 4 * h) = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (c0 + q < nb) row[4 * h + q] = v[q];
+        }
+        const __nv_bfloat162 h01 = __floats2bfloat162_rn(v[0], v[1]);
+        const __nv_bfloat162 h23 = __floats2bfloat162_rn(v[2], v[3]);
+        const float e0 = v[0] - __low2float(h01), e1 = v[1] - __high2float(h01);
+        const float e2 = v[2] - __low2float(h23), e3 = v[3] - __high2float(h23);
+        const __nv_bfloat162 m01 = __floats2bfloat162_rn(e0, e1);
+        const __nv_bfloat162 m23 = __floats2bfloat162_rn(e2, e3);
+        const __nv_bfloat162 l01 = __floats2bfloat162_rn(e0 - __low2float(m01), e1 - __high2float(m01));
+        const __nv_bfloat162 l23 = __floats2bfloat162_rn(e2 - __low2float(m23), e3 - __high2float(m23));
+        const int64_t off = i * NB + c0;
+        *reinterpret_cast<uint2*>(splits + off) = make_uint2(bits(h01), bits(h23));
+        *reinterpret_cast<uint2*>(splits + plane + off) = make_uint2(bits(m01), bits(m23));
+        *reinterpret_cast<uint2*>(splits + 2 * plane + off) = make_uint2(bits(l01), bits(l23));
+      }
+    }
+  }
+  cp_async_wait_all();
+  return true;
 }
 
 // Copy the staged diagonal blocks U_JJ into H (one CTA per block).  They are
@@ -381,7 +567,232 @@ __global__ void __launch_bounds__(256) diag_store_kernel(float* H, int64_t n, co
   }
 }
 
+// ---------------------------------------------------------------------------
+// The whole blocked factorisation as one persistent kernel: one CTA per SM
+// (cooperative launch, so every CTA is resident and CTAs may wait for one
+// another), no launch per step.  The first nd CTAs run the diagonal steps
+// (diag_step_p: each factors the block, they share the panel rows), the
+// others the tensor-core Schur tiles, the last tile column of each step
+// first: it holds the next diagonal block, so the next diagonal step starts
+// while the rest of the update is still running (a one-step look-ahead).
+// Tile (r, c) always belongs to the Schur CTA (c (c+1)/2 + r) mod ns, so the
+// updates of one tile follow each other in that CTA's program order.
+// Cross-CTA order goes through counters in global memory:
+//   panel_done[J]  diagonal CTAs that finished D(J)        (step J waits for all)
+//   colready[J-1]  finished last-column tiles of step J    (D(J-1) waits for all)
+//   schur_done[J]  finished tiles of step J                (D(J-2) waits: it reuses
+//                                                           the split buffer of J)
+// Every wait is bounded; a timeout sets the device status and an abort flag
+// that ends every CTA's loop.
+constexpr int PERSIST_THREADS = 256;
+constexpr int PERSIST_BODY = ((size_t)schur::TILE_SMEM > sizeof(DiagSmemP))
+                                 ? (int)schur::TILE_SMEM
+                                 : (int)((sizeof(DiagSmemP) + 1023) & ~(size_t)1023);
+constexpr int PERSIST_SMEM = PERSIST_BODY + 1024 + 256;
+static_assert(sizeof(DiagSmemP) + 2048 + 256 <= 227 * 1024, "diagonal step fits one CTA's shared memory");
+
+struct PersistArgs {
+  float* H;
+  int64_t n;
+  int nblk;
+  __nv_bfloat16* splits[2];
+  float* stage;
+  int* info;
+  int* ctr;     // panel_done[nblk], colready[nblk], schur_done[nblk], abort
+  int vec4;
+  int ndiag;    // CTAs that run the diagonal steps
+};
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Thread 0 waits until *p >= target (bounded, and ended by the abort flag);
+// the result is shared with the whole CTA.  Orders the CTA's later reads
+// (generic and TMA) after the other CTAs' published writes.
+__device__ __forceinline__ bool cta_wait(const int* p, int target, int* abortf) {
+  int ok = 1;
+  if (threadIdx.x == 0 && ld_acquire_gpu(p) < target) {
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (ld_acquire_gpu(p) >= target) break;
+      if (ld_acquire_gpu(abortf) != 0) {
+        ok = 0;
+        break;
+      }
+      if ((it & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+        record_timeout();
+        atomicExch(abortf, 1);
+        ok = 0;
+        break;
+      }
+      __nanosleep(100);
+    }
+  }
+  ok = __syncthreads_and(ok);
+  fence_proxy_async_global();
+  return ok != 0;
+}
+
+// Publishes this CTA's global writes (generic and TMA) and adds 1 to each
+// counter given.
+__device__ __forceinline__ void cta_publish(int* p0, int* p1) {
+  fence_proxy_async_global();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    red_release_gpu_add(p0, 1);
+    if (p1) red_release_gpu_add(p1, 1);
+  }
+}
+
+__device__ __forceinline__ int tri_count(int nt) { return nt * (nt + 1) / 2; }
+
+// Column-major index of the upper triangle -> (r, c), r <= c.
+__device__ __forceinline__ void tri_rc(int idx, int& r, int& c) {
+  c = (int)((sqrtf(8.f * (float)idx + 1.f) - 1.f) * 0.5f);
+  while (tri_count(c) > idx) --c;
+  while (tri_count(c + 1) <= idx) ++c;
+  r = idx - tri_count(c);
+}
+
+__global__ void __launch_bounds__(PERSIST_THREADS, 1)
+    chol_persistent_kernel(const __grid_constant__ CUtensorMap p0h, const __grid_constant__ CUtensorMap p0m,
+                           const __grid_constant__ CUtensorMap p0l, const __grid_constant__ CUtensorMap p1h,
+                           const __grid_constant__ CUtensorMap p1m, const __grid_constant__ CUtensorMap p1l,
+                           const __grid_constant__ CUtensorMap mC, PersistArgs a) {
+  if (*a.info != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PERSIST_BODY);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  const uint32_t full = smem_u32(&bars[0]);
+  const uint32_t cbar = smem_u32(&bars[1]);
+  const uint32_t accbar = smem_u32(&bars[2]);
+  const int warp = threadIdx.x >> 5;
+  const int cta = blockIdx.x, ncta = gridDim.x;
+  const int nblk = a.nblk;
+  const int64_t n = a.n;
+  int* panel_done = a.ctr;
+  int* colready = a.ctr + nblk;
+  int* schur_done = a.ctr + 2 * nblk;
+  int* abortf = a.ctr + 3 * nblk;
+
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(cbar, 1);
+    mbar_init(accbar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), schur::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const schur::TileMaps maps[2] = {{&p0h, &p0m, &p0l, &mC}, {&p1h, &p1m, &p1l, &mC}};
+  uint32_t tcount = 0;
+  // Roles: CTAs 0 .. nd-1 run the diagonal steps (each factors the block,
+  // they share the panel rows), the other ns CTAs the Schur tiles.
+  const int nd = a.ndiag, ns = ncta - nd;
+
+  // nt(J): tiles per side of the update of step J (the upper triangle of j0 x j0)
+  auto nt_of = [](int J) { return (J * NB + 127) / 128; };
+
+  if (cta < nd) {
+    DiagSmemP& F = *reinterpret_cast<DiagSmemP*>(smem);
+    for (int J = nblk - 1; J >= 0; --J) {
+      // block J is final once the last tile column of step J + 1 is done;
+      // its split buffer is free once every tile of step J + 2 is done
+      if (J < nblk - 1 && !cta_wait(&colready[J], nt_of(J + 1), abortf)) break;
+      if (J + 2 <= nblk - 1 && !cta_wait(&schur_done[J + 2], tri_count(nt_of(J + 2)), abortf)) break;
+      const int64_t j0 = (int64_t)J * NB;
+      const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
+      if (!diag_step_p(F, a.H, n, j0, nb, a.info, a.splits[J & 1], a.stage, cta, nd)) {
+        // a non-positive pivot (seen by every diagonal CTA): stop the Schur CTAs too
+        if (threadIdx.x == 0) atomicExch(abortf, 2);
+        break;
+      }
+      cta_publish(&panel_done[J], nullptr);
+    }
+  } else {
+    const int sc = cta - nd;
+    // One tile; a last-column tile is published at once (the next diagonal
+    // step waits for it), the bulk tiles of a step together at its end.
+    auto run_tile = [&](int J, int idx, bool last) -> bool {
+      int r, c;
+      tri_rc(idx, r, c);
+      const bool ok = schur::tile<0, 8>(smem, full, cbar, accbar, tcount & 1u, tmem, maps[J & 1], a.H,
+                                        n, (int64_t)J * NB, (int64_t)r * 128, (int64_t)c * 128, 1,
+                                        last ? 1 : 0);
+      ++tcount;
+      tc_fence_before();
+      if (last) cta_publish(&colready[J - 1], &schur_done[J]);
+      const int all = __syncthreads_and(ok ? 1 : 0);
+      tc_fence_after();
+      if (!all) {
+        if (threadIdx.x == 0) atomicExch(abortf, 1);
+        return false;
+      }
+      return true;
+    };
+    bool ok = true;
+    for (int J = nblk - 1; ok && J >= 1; --J) {
+      const int nt = nt_of(J);
+      const int lo = tri_count(nt - 1), hi = tri_count(nt);
+      if (!cta_wait(&panel_done[J], nd, abortf)) break;
+      // the last tile column (holds block J - 1) first, then the others from
+      // the right, so the next step's last column comes early
+      for (int idx = lo + ((sc - lo % ns) % ns + ns) % ns; ok && idx < hi; idx += ns) ok = run_tile(J, idx, true);
+      const int top = lo - 1 - ((((lo - 1) - sc) % ns) + ns) % ns;   // largest idx < lo owned by sc
+      int nbulk = 0;
+      for (int idx = top; ok && idx >= 0; idx -= ns, ++nbulk) ok = run_tile(J, idx, false);
+      if (!ok) break;
+      if (nbulk > 0) {
+        if (threadIdx.x == 0) tma_store_wait_all();   // the bulk tiles' stores reached memory
+        fence_proxy_async_global();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          __threadfence();
+          red_release_gpu_add(&schur_done[J], nbulk);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, schur::TMEM_COLS);
+  }
+}
+
 }  // namespace
+
+cudaError_t status_fetch_chol(int* out, cudaStream_t s) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(s);
+  *out = v;
+  return e;
+}
 
 static size_t tbuf_bytes(int64_t n) {
   // recursive inverse: products T of the pairs of one level (at most n*n/4
@@ -391,12 +802,15 @@ static size_t tbuf_bytes(int64_t n) {
   return (((size_t)f * sizeof(float)) + 255) & ~size_t(255);
 }
 
+static size_t splits_bytes(int64_t n) {
+  return (((size_t)3 * n * NB * sizeof(__nv_bfloat16)) + 255) & ~size_t(255);
+}
+
 size_t chol_workspace_bytes(int64_t n) {
-  // T / staging buffer, then the bf16 hi/mid/lo splits of the current panel
-  // (3 x n x 64)
-  const size_t tbytes = tbuf_bytes(n);
-  const size_t sbytes = (size_t)3 * n * NB * sizeof(__nv_bfloat16);
-  return tbytes + sbytes;
+  // T / staging buffer, two buffers of bf16 hi/mid/lo panel splits
+  // (3 x n x 64 each), the step counters of the persistent kernel
+  const int64_t nblk = ceil_div(n, NB);
+  return tbuf_bytes(n) + 2 * splits_bytes(n) + (size_t)(3 * nblk + 4) * sizeof(int);
 }
 
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
@@ -410,8 +824,10 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
   }
   if (n <= 0) return KRONQ_OK;
   float* Tbuf = reinterpret_cast<float*>(ws);
-  __nv_bfloat16* splits =
-      reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + tbuf_bytes(n));
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* splits = reinterpret_cast<__nv_bfloat16*>(wsb + tbuf_bytes(n));
+  __nv_bfloat16* splits1 = reinterpret_cast<__nv_bfloat16*>(wsb + tbuf_bytes(n) + splits_bytes(n));
+  int* ctr = reinterpret_cast<int*>(wsb + tbuf_bytes(n) + 2 * splits_bytes(n));
   SchurMaps maps;
   if (n > NB) {
     kronq_status r = schur_maps(&maps, splits, H, n);
@@ -421,7 +837,46 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
   const int64_t nblk = ceil_div(n, NB);
   const int64_t pmax = sm_count();
   const int vec4 = ((n % 4) == 0 && aligned(H, 16)) ? 1 : 0;
-  for (int64_t bj = nblk - 1; bj >= 0; --bj) {
+  // The persistent kernel (one launch for the whole chain) when the tile of
+  // A can be staged by TMA and every CTA can be resident at once.
+  bool persist = n > 4 * NB && maps.tma_c && nblk < (1 << 20);
+  int coop = 0, per_sm = 0;
+  if (persist) {
+    int dev = 0;
+    KQ_CUDA(cudaGetDevice(&dev));
+    KQ_CUDA(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(&chol_persistent_kernel), PERSIST_SMEM);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(persistent factorisation)");
+    KQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &per_sm, reinterpret_cast<const void*>(&chol_persistent_kernel), PERSIST_THREADS, PERSIST_SMEM));
+    persist = coop != 0 && per_sm >= 1;
+  }
+  if (persist) {
+    SchurMaps maps1;
+    kronq_status r = schur_maps(&maps1, splits1, H, n);
+    if (r != KRONQ_OK) return r;
+    KQ_CUDA(cudaMemsetAsync(ctr, 0, (size_t)(3 * nblk + 4) * sizeof(int), s));
+    const CUtensorMap* m0 = reinterpret_cast<const CUtensorMap*>(maps.raw);
+    const CUtensorMap* m1 = reinterpret_cast<const CUtensorMap*>(maps1.raw);
+    CUtensorMap a0 = m0[0], a1 = m0[1], a2 = m0[2], b0 = m1[0], b1 = m1[1], b2 = m1[2], c = m0[3];
+    PersistArgs pa;
+    pa.H = H;
+    pa.n = n;
+    pa.nblk = (int)nblk;
+    pa.splits[0] = splits;
+    pa.splits[1] = splits1;
+    pa.stage = Tbuf;
+    pa.info = info;
+    pa.ctr = ctr;
+    pa.vec4 = vec4;
+    pa.ndiag = (int)(pmax >= 64 ? 32 : pmax / 2);
+    void* args[] = {&a0, &a1, &a2, &b0, &b1, &b2, &c, &pa};
+    KQ_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(&chol_persistent_kernel),
+                                        dim3((unsigned)pmax), dim3(PERSIST_THREADS), args,
+                                        (size_t)PERSIST_SMEM, s));
+    count_launch();
+  }
+  for (int64_t bj = persist ? -1 : nblk - 1; bj >= 0; --bj) {
     const int64_t j0 = bj * NB;
     const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
     // One CTA per SM at most (each CTA factors the block itself), one chunk

@@ -173,17 +173,19 @@ def test_cholesky_of_damped_inverse(n):
     assert rel(got, U) < 2e-4
 
 
-def test_cholesky_not_positive_definite_reports_info():
-    n = 130
+@pytest.mark.parametrize("n,bad", [(130, 37), (640, 301), (1024, 1000)])
+def test_cholesky_not_positive_definite_reports_info(n, bad):
+    # n = 130 runs the per-step kernels, the larger sizes the persistent one
     H = np.eye(n, dtype=np.float32)
-    H[37, 37] = -5.0
+    H[bad, bad] = -5.0
     lp = LayerPass(8, n, bits=4, group=128)
     lp.HX.copy_(torch.from_numpy(H))
     lp.Wt.zero_()
     lp.quantize()
     torch.cuda.synchronize()
     A, _ = sweep.damp(H.astype(np.float64), 0.01)
-    assert int(lp.info.item()) == sweep.reverse_chol_failure(A) == 38
+    assert int(lp.info.item()) == sweep.reverse_chol_failure(A) == bad + 1
+    assert kq.kronq_device_status() == 0
 
 
 # ------------------------------------------------------------------ sweep
