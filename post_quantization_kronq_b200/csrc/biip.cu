@@ -48,6 +48,45 @@ __device__ __forceinline__ float col_factor(const RowPass& p, int j) {
   return f;
 }
 
+// One radix-16 pass of the FWHT over bits LO .. LO+3 of a 4096-long row
+// (rows of stride RS, padded by padx).  Item t of a row: a0 has bits LO ..
+// LO+3 clear; its sixteen elements a0 + (u << LO) sit at padx(a0) + off(u)
+// with off(u) known at compile time (the padding adds one word per 32, and
+// a0 never carries into it: a0 mod 32 is 0 or 16 for LO = 0, below 16 for
+// LO = 4).
+template <int LO>
+__device__ __forceinline__ void radix16_pass(float* cur, int RS, int logR) {
+  constexpr int PER_ROW = 4096 / 16;
+  const int items = PER_ROW << logR;
+  for (int t = threadIdx.x; t < items; t += RP_THREADS) {
+    const int rr = t >> 8;
+    const int rem = t & (PER_ROW - 1);
+    const int a0 = ((rem >> LO) << (LO + 4)) | (rem & ((1 << LO) - 1));
+    float* base = cur + rr * RS + padx(a0);
+    float x[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int off = (LO == 0) ? u : (LO == 4 ? 16 * u + (u >> 1) : (u << LO) + (u << (LO - 5)));
+      x[u] = base[off];
+    }
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if ((u & h) == 0) {
+          const float s0 = x[u], s1 = x[u | h];
+          x[u] = s0 + s1;
+          x[u | h] = s0 - s1;
+        }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int off = (LO == 0) ? u : (LO == 4 ? 16 * u + (u >> 1) : (u << LO) + (u << (LO - 5)));
+      base[off] = x[u];
+    }
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
   extern __shared__ __align__(16) float sm[];
   const RowPass& p = A.p;
@@ -70,8 +109,35 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
 
   // 1. load rows (forward: times sign and scale of the column); the column
   //    factor is computed once per column and reused for the R rows.
-  //    All R loads of a column are issued before any is used.
-  for (int j = tid; j < L; j += RP_THREADS) {
+  //    Rows up to 8 x RP_THREADS long: all of a thread's loads (8 columns x
+  //    R rows) are issued before any is used, one memory latency per CTA.
+  if (L <= 8 * RP_THREADS) {
+    float v[8][8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int j = tid + c * RP_THREADS;
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        v[c][rr] = 0.f;
+        if (j < L && rr < rows_here) {
+          const int64_t idx = (r0 + rr) * p.ld_in + j;
+          v[c][rr] = p.in_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[idx])
+                               : reinterpret_cast<const float*>(p.in)[idx];
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int j = tid + c * RP_THREADS;
+      if (j < L) {
+        const float f = p.inverse ? 1.f : col_factor(p, j);
+        const int pj = padx(j);
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+          if (rr < R) buf0[rr * RS + pj] = v[c][rr] * f;
+      }
+    }
+  } else for (int j = tid; j < L; j += RP_THREADS) {
     const float f = p.inverse ? 1.f : col_factor(p, j);
     const int pj = padx(j);
     float v[8];
@@ -130,7 +196,12 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
     // 3. FWHT along a: radix-16 register passes over 4-bit groups of a.
     //    Item order (b fastest, then the low bits of a, then the high bits)
     //    keeps neighbouring threads on neighbouring shared-memory words.
-    for (int lo = 0; lo < A.logP; lo += 4) {
+    if (K == 1 && A.logP == 12) {
+      // length 4096: three radix-16 passes with compile-time offsets
+      radix16_pass<0>(cur, RS, A.logR);
+      radix16_pass<4>(cur, RS, A.logR);
+      radix16_pass<8>(cur, RS, A.logR);
+    } else for (int lo = 0; lo < A.logP; lo += 4) {
       const int nb = (A.logP - lo) < 4 ? (A.logP - lo) : 4;
       const int G = 1 << nb;
       const int per_row = L >> nb;

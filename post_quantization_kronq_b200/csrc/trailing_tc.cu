@@ -11,9 +11,10 @@
 // One CTA per 128 x 128 tile of W[:, j1:]: warp 0 issues all TMA loads (the
 // fp32 W tile into shared memory, two 64-wide k chunks of E_hi/E_lo, K-major,
 // and of U_hi/U_lo, MN-major), warp 1 issues 24 tcgen05.mma (M 128, N 128,
-// K 16) into 128 TMEM columns, warps 2-5 subtract the accumulator from the
-// staged tile (128-byte swizzled boxes, conflict-free float4 accesses) and
-// write it back with TMA stores.  Each element is owned by one CTA.
+// K 16) into 128 TMEM columns, then all eight warps subtract the accumulator
+// from the staged tile (128-byte swizzled boxes, conflict-free float4
+// accesses) and one thread writes it back with TMA stores.  Each element is
+// owned by one CTA.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -31,7 +32,7 @@ constexpr int CHUNK_BYTES = 2 * A_BOX + 2 * B_SPLIT;   // hi+lo of A and B: 64 K
 constexpr int C_BOX = BM * 32 * 4;         // 16 KB: 128 rows x 32 fp32 (128-byte swizzle)
 constexpr int C_BYTES = (BN / 32) * C_BOX; // 64 KB
 constexpr int SMEM_BYTES = NKC * CHUNK_BYTES + C_BYTES + 1024 + 256;
-constexpr int THREADS = 192;
+constexpr int THREADS = 256;
 constexpr uint32_t TMEM_COLS = BN;
 
 struct TrailArgs {
@@ -77,71 +78,68 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t base = smem_u32(smem);
   const uint32_t cs = base + NKC * CHUNK_BYTES;   // staged W tile
 
-  if (warp == 0) {
-    if (lane == 0) {
-      if (args.tma_c) {
-        mbar_arrive_expect_tx(cbar, C_BYTES);
+  if (warp == 0 && lane == 0) {
+    if (args.tma_c) {
+      mbar_arrive_expect_tx(cbar, C_BYTES);
 #pragma unroll
-        for (int h = 0; h < BN / 32; ++h) tma_load_2d(cs + h * C_BOX, &mW, cbar, (int)(c0 + 32 * h), (int)r0);
-      }
-      for (int c = 0; c < args.nkc; ++c) {
-        const uint32_t full = full0 + 8 * c;
-        const uint32_t s = base + c * CHUNK_BYTES;
-        mbar_arrive_expect_tx(full, CHUNK_BYTES);
-        tma_load_2d(s, &mEh, full, c * KC, (int)r0);
-        tma_load_2d(s + A_BOX, &mEl, full, c * KC, (int)r0);
-#pragma unroll
-        for (int h = 0; h < BN / 64; ++h) {
-          tma_load_2d(s + 2 * A_BOX + h * B_BOX, &mUh, full, (int)(c0 + 64 * h), c * KC);
-          tma_load_2d(s + 2 * A_BOX + B_SPLIT + h * B_BOX, &mUl, full, (int)(c0 + 64 * h), c * KC);
-        }
-      }
-      for (int c = 0; c < args.nkc; ++c) mbar_wait(full0 + 8 * c, 0);
-      if (args.tma_c) mbar_wait(cbar, 0);
+      for (int h = 0; h < BN / 32; ++h) tma_load_2d(cs + h * C_BOX, &mW, cbar, (int)(c0 + 32 * h), (int)r0);
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, true);
-      uint32_t acc = 0;
-      for (int c = 0; c < args.nkc; ++c) {
-        if (!mbar_wait(full0 + 8 * c, 0)) break;
-        tc_fence_after();
-        const uint32_t s = base + c * CHUNK_BYTES;
-        const uint32_t ah = s, al = s + A_BOX;
-        const uint32_t bh = s + 2 * A_BOX, bl = s + 2 * A_BOX + B_SPLIT;
+    for (int c = 0; c < args.nkc; ++c) {
+      const uint32_t full = full0 + 8 * c;
+      const uint32_t s = base + c * CHUNK_BYTES;
+      mbar_arrive_expect_tx(full, CHUNK_BYTES);
+      tma_load_2d(s, &mEh, full, c * KC, (int)r0);
+      tma_load_2d(s + A_BOX, &mEl, full, c * KC, (int)r0);
 #pragma unroll
-        for (int kk = 0; kk < KC / 16; ++kk) {
-          // A K-major: 16 k = 32 bytes along each 128-byte row.  B MN-major:
-          // 16 k rows of 128 bytes = 2048 bytes inside every 64-column box.
-          const uint64_t dah = smem_desc_sw128(ah + kk * 32, 16, 1024);
-          const uint64_t dal = smem_desc_sw128(al + kk * 32, 16, 1024);
-          const uint64_t dbh = smem_desc_sw128(bh + kk * 2048, B_BOX, 1024);
-          const uint64_t dbl = smem_desc_sw128(bl + kk * 2048, B_BOX, 1024);
-          mma_bf16(tmem, dah, dbh, idesc, acc);
-          acc = 1;
-          mma_bf16(tmem, dah, dbl, idesc, 1u);
-          mma_bf16(tmem, dal, dbh, idesc, 1u);
-        }
+      for (int h = 0; h < BN / 64; ++h) {
+        tma_load_2d(s + 2 * A_BOX + h * B_BOX, &mUh, full, (int)(c0 + 64 * h), c * KC);
+        tma_load_2d(s + 2 * A_BOX + B_SPLIT + h * B_BOX, &mUl, full, (int)(c0 + 64 * h), c * KC);
       }
-      mma_commit(accbar);
     }
-    __syncwarp();
-  } else {
-    const int q = warp & 3;
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, true);
+    uint32_t acc = 0;
+    for (int c = 0; c < args.nkc; ++c) {
+      if (!mbar_wait(full0 + 8 * c, 0)) break;
+      tc_fence_after();
+      const uint32_t s = base + c * CHUNK_BYTES;
+      const uint32_t ah = s, al = s + A_BOX;
+      const uint32_t bh = s + 2 * A_BOX, bl = s + 2 * A_BOX + B_SPLIT;
+#pragma unroll
+      for (int kk = 0; kk < KC / 16; ++kk) {
+        // A K-major: 16 k = 32 bytes along each 128-byte row.  B MN-major:
+        // 16 k rows of 128 bytes = 2048 bytes inside every 64-column box.
+        const uint64_t dah = smem_desc_sw128(ah + kk * 32, 16, 1024);
+        const uint64_t dal = smem_desc_sw128(al + kk * 32, 16, 1024);
+        const uint64_t dbh = smem_desc_sw128(bh + kk * 2048, B_BOX, 1024);
+        const uint64_t dbl = smem_desc_sw128(bl + kk * 2048, B_BOX, 1024);
+        mma_bf16(tmem, dah, dbh, idesc, acc);
+        acc = 1;
+        mma_bf16(tmem, dah, dbl, idesc, 1u);
+        mma_bf16(tmem, dal, dbh, idesc, 1u);
+      }
+    }
+    mma_commit(accbar);
+  }
+  __syncwarp();
+  {
+    // epilogue, all eight warps: warp w takes TMEM lanes 32 (w % 4) and the
+    // columns 64 (w / 4) .. +63 of the tile
+    const int q = warp & 3, half = warp >> 2;
     const int rl = q * 32 + lane;          // row of the tile
-    bool ok = true;
+    int good = 1;
     if (lane == 0) {
-      ok = mbar_wait(accbar, 0);
-      if (ok && args.tma_c) ok = mbar_wait(cbar, 0);
+      good = mbar_wait(accbar, 0) ? 1 : 0;
+      if (good && args.tma_c) good = mbar_wait(cbar, 0) ? 1 : 0;
     }
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    good = __shfl_sync(0xffffffffu, good, 0);
     __syncwarp();
-    if (ok) {
+    if (good) {
       tc_fence_after();
       const int64_t i = r0 + rl;
       const int64_t n = args.n;
 #pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
+      for (int cc = 2 * half; cc < 2 * half + 2; ++cc) {
         uint32_t v[32];
         __syncwarp();  // the TMEM load is warp-collective
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + cc * 32, v);
@@ -168,15 +166,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (args.tma_c) {
-        fence_proxy_async_smem();
-        named_barrier(1, 128);             // the four epilogue warps
-        if (warp == 2 && lane == 0) {
+      if (args.tma_c) fence_proxy_async_smem();
+    }
+    if (args.tma_c) {
+      __syncthreads();
+      if (good && warp == 0 && lane == 0) {
 #pragma unroll
-          for (int h = 0; h < BN / 32; ++h) tma_store_2d(&mW, cs + h * C_BOX, (int)(c0 + 32 * h), (int)r0);
-          tma_store_commit();
-          tma_store_wait_all();
-        }
+        for (int h = 0; h < BN / 32; ++h) tma_store_2d(&mW, cs + h * C_BOX, (int)(c0 + 32 * h), (int)r0);
+        tma_store_commit();
+        tma_store_wait_read();  // shared memory read; the writes finish on their own
       }
     }
   }

@@ -114,7 +114,7 @@ def _biip_case(m, n, seed, wdtype=torch.float32):
     return Wg, to_np(Wg), HX, HG
 
 
-@pytest.mark.parametrize("m,n", [(256, 256), (200, 448), (96, 392), (3, 5), (1, 24)])
+@pytest.mark.parametrize("m,n", [(256, 256), (200, 448), (96, 392), (3, 5), (1, 24), (48, 4096), (4096, 40)])
 def test_biip_forward_inverse(m, n):
     Wg, W, HX, HG = _biip_case(m, n, seed=m + n)
     HXg, HGg = torch.from_numpy(HX).to(DEV), torch.from_numpy(HG).to(DEV)
