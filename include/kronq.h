@@ -211,10 +211,10 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
  * exposes no allocator, or a foreign-language caller without a CUDA
  * allocation binding), or run where cudaMalloc is not allowed because it
  * synchronises the device.  Arguments as kronq_quantize_layer, minus the
- * workspace: the scratch is a file-scope static device array of 32 MiB that
+ * workspace: the scratch is a file-scope static device array of 64 MiB that
  * every GPU loading the library holds until the process exits.
- *   - Layers whose kronq_quantize_workspace_bytes(m, n, p) exceeds 32 MiB
- *     (for example n = 4096 with m up to ~28000, or n up to ~5600 with small
+ *   - Layers whose kronq_quantize_workspace_bytes(m, n, p) exceeds 64 MiB
+ *     (for example n = 4096 with m above ~9000, or n above ~7000 with small
  *     m) are rejected with KRONQ_ERR_INVALID_ARG before anything runs.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call

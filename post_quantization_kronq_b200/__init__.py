@@ -155,7 +155,7 @@ def kronq_quantize_layer(Wt, HX, params: QuantParams, codes, scales, zeros, info
 def kronq_quantize_layer_static(Wt, HX, params: QuantParams, codes, scales, zeros, info, E=None,
                                 stream=None):
     """kronq_quantize_layer without a workspace, for callers that cannot
-    allocate device memory: the scratch is the library's 32 MiB static device
+    allocate device memory: the scratch is the library's 64 MiB static device
     array (shared by all calls on a device; overlapping calls race)."""
     m, n = Wt.shape
     for t, name in ((Wt, "Wt"), (HX, "HX"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),

@@ -94,15 +94,22 @@ size_t biip_ws(int64_t m, int64_t n) {
 
 int64_t quant_ldu(int64_t n) { return (n + 7) / 8 * 8; }
 
+// Blocks per group of the two-level trailing update: up to eight (K = 1024).
+int64_t quant_gblocks(int64_t n) {
+  const int64_t nblk = ceil_div(n, 128);
+  return nblk < 8 ? (nblk < 1 ? 1 : nblk) : 8;
+}
+
 size_t quant_ws(int64_t m, int64_t n) {
   Carver c(nullptr);
   c.take<uint8_t>(chol_workspace_bytes(n));
   c.take<uint8_t>((size_t)n);
   c.take<float>((size_t)(m * 128));
-  c.take<__nv_bfloat16>((size_t)(m * 128));
-  c.take<__nv_bfloat16>((size_t)(m * 128));
-  c.take<__nv_bfloat16>((size_t)(128 * quant_ldu(n)));
-  c.take<__nv_bfloat16>((size_t)(128 * quant_ldu(n)));
+  const int64_t kg = 128 * quant_gblocks(n);
+  c.take<__nv_bfloat16>((size_t)(m * kg));
+  c.take<__nv_bfloat16>((size_t)(m * kg));
+  c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
+  c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
   return c.size();
 }
 
@@ -375,10 +382,11 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
   void* cws = c.take<uint8_t>(chol_workspace_bytes(n));
   uint8_t* dead = c.take<uint8_t>((size_t)n);
   float* Eblk = c.take<float>((size_t)(m * 128));
-  __nv_bfloat16* Eh = c.take<__nv_bfloat16>((size_t)(m * 128));
-  __nv_bfloat16* El = c.take<__nv_bfloat16>((size_t)(m * 128));
-  __nv_bfloat16* Uh = c.take<__nv_bfloat16>((size_t)(128 * quant_ldu(n)));
-  __nv_bfloat16* Ul = c.take<__nv_bfloat16>((size_t)(128 * quant_ldu(n)));
+  const int64_t kg = 128 * quant_gblocks(n);
+  __nv_bfloat16* Eh = c.take<__nv_bfloat16>((size_t)(m * kg));
+  __nv_bfloat16* El = c.take<__nv_bfloat16>((size_t)(m * kg));
+  __nv_bfloat16* Uh = c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
+  __nv_bfloat16* Ul = c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
   const bool u_given = (p->flags & KRONQ_U_GIVEN) != 0;
   kronq_status r;
   if (u_given) {
@@ -398,6 +406,8 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
   d.info = info;
   d.ordered = (p->flags & KRONQ_ORDERED_FP32) != 0;
   d.Eh = Eh; d.El = El; d.Uh = Uh; d.Ul = Ul; d.ldu = quant_ldu(n);
+  d.lde = kg;
+  d.gblocks = (int)quant_gblocks(n);
   return gptq_sweep(d, st);
 }
 

@@ -138,10 +138,13 @@ struct alignas(64) TrailingMaps {
   unsigned char raw[5 * 128];
   int tma_c = 0;   // W tile staged by TMA (needs a 16-byte row stride)
 };
-kronq_status trailing_maps(TrailingMaps* tm, const void* Eh, const void* El, int64_t m,
-                           const void* Uh, const void* Ul, int64_t ldu, float* W, int64_t n);
-kronq_status trailing_update_tc(const TrailingMaps* tm, float* W, int64_t m, int64_t n, int64_t j1,
-                                int bw, const int* info, cudaStream_t s);
+// E hi/lo: m x lde bf16 (K-major); U hi/lo: ku x n bf16 (row stride ldu).
+kronq_status trailing_maps(TrailingMaps* tm, const void* Eh, const void* El, int64_t m, int64_t lde,
+                           const void* Uh, const void* Ul, int64_t ku, int64_t ldu, float* W, int64_t n);
+// W[:, c_begin : c_begin + ncols] -= E[:, k0 : k0 + K] U[k0 : k0 + K, same columns]
+// (K rounded up to 64; the E and U entries beyond K must be zero).
+kronq_status trailing_update_tc(const TrailingMaps* tm, float* W, int64_t m, int64_t n, int64_t c_begin,
+                                int64_t ncols, int64_t k0, int64_t K, const int* info, cudaStream_t s);
 cudaError_t status_fetch_trailing(int* out, cudaStream_t s);
 
 struct SweepDesc {
@@ -159,14 +162,19 @@ struct SweepDesc {
   const uint8_t* dead = nullptr;
   const int* info = nullptr;
   bool ordered = false;
-  // tensor-core trailing update (used unless ordered): bf16 hi/lo splits of
-  // the block's scaled errors (m x 128) and of the block's rows of U
-  // (128 x ldu), rewritten for every block.
+  // tensor-core trailing updates (used unless ordered), two-level: bf16
+  // hi/lo splits of the scaled errors (m x lde, lde = 128 gblocks) and of the
+  // rows of U (128 gblocks x ldu) of the blocks of the current group of
+  // gblocks blocks.  After a block, the next block's columns get the update
+  // of every block of the group so far; at the group's end the columns past
+  // it get the whole group's update at once (K = 128 gblocks).
   __nv_bfloat16* Eh = nullptr;
   __nv_bfloat16* El = nullptr;
   __nv_bfloat16* Uh = nullptr;
   __nv_bfloat16* Ul = nullptr;
   int64_t ldu = 0;
+  int64_t lde = 128;
+  int gblocks = 1;
 };
 kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s);
 

@@ -24,7 +24,7 @@
 
 namespace {
 
-constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB per device
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;  // 64 MiB per device
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_quant_scratch[kStaticScratchBytes];
@@ -65,7 +65,7 @@ extern "C" kronq_status kronq_quantize_layer_static(float* Wt, float* HX, int64_
                     "quantize_layer_static: this layer needs " + std::to_string(need) +
                         " bytes of scratch but the static scratch holds " +
                         std::to_string(kStaticScratchBytes) +
-                        " bytes (32 MiB); use kronq_quantize_layer with a caller workspace");
+                        " bytes (64 MiB); use kronq_quantize_layer with a caller workspace");
   void* scratch = nullptr;
   kronq_status r = scratch_address(&scratch);
   if (r != KRONQ_OK) return r;

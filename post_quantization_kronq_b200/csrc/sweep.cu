@@ -37,6 +37,7 @@ struct BlockArgs {
   int wide;       // 1: the grid of this block's first column was computed beforehand
   float* Eb;      // scaled-error output of this block (fp32) or nullptr
   int64_t lde;
+  int slot;       // position of the block in its group (split buffers)
 };
 
 __device__ __forceinline__ void grid_from_range(float lo, float hi, int bits, bool asym, float& scale,
@@ -139,8 +140,8 @@ __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
   if (!d.ordered && j1 < n) {
     for (int64_t k = blockIdx.x; k < bw; k += gridDim.x) {
       const float* src = d.U + (j0 + k) * n;
-      __nv_bfloat16* dh = d.Uh + k * d.ldu;
-      __nv_bfloat16* dl = d.Ul + k * d.ldu;
+      __nv_bfloat16* dh = d.Uh + ((int64_t)a.slot * BW + k) * d.ldu;
+      __nv_bfloat16* dl = d.Ul + ((int64_t)a.slot * BW + k) * d.ldu;
       if (vec) {
 #pragma unroll 4
         for (int64_t c = j1 + 4 * tid; c < n; c += 4 * blockDim.x) {
@@ -313,8 +314,8 @@ __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
       if (q * QW + c < bw) a.Eb[r * a.lde + q * QW + c] = ev[c];
   }
   if (!d.ordered) {
-    __nv_bfloat16* eh = d.Eh + r * BW + q * QW;
-    __nv_bfloat16* el = d.El + r * BW + q * QW;
+    __nv_bfloat16* eh = d.Eh + r * d.lde + (int64_t)a.slot * BW + q * QW;
+    __nv_bfloat16* el = d.El + r * d.lde + (int64_t)a.slot * BW + q * QW;
 #pragma unroll
     for (int c = 0; c < QW; c += 2) {
       const __nv_bfloat16 h0 = __float2bfloat16_rn(ev[c]), h1 = __float2bfloat16_rn(ev[c + 1]);
@@ -363,15 +364,18 @@ kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div(m, ROWS_PER_CTA);
   TrailingMaps maps;
   if (!d.ordered && n > BW) {
-    kronq_status r = trailing_maps(&maps, d.Eh, d.El, m, d.Uh, d.Ul, d.ldu, d.W, n);
+    kronq_status r = trailing_maps(&maps, d.Eh, d.El, m, d.lde, d.Uh, d.Ul, (int64_t)d.gblocks * BW,
+                                   d.ldu, d.W, n);
     if (r != KRONQ_OK) return r;
   }
-  for (int64_t j0 = 0; j0 < n; j0 += BW) {
+  int64_t blk = 0;
+  for (int64_t j0 = 0; j0 < n; j0 += BW, ++blk) {
     const int bw = (int)((j0 + BW <= n) ? BW : n - j0);
     BlockArgs a;
     a.d = d;
     a.j0 = j0;
     a.bw = bw;
+    a.slot = (int)(blk % d.gblocks);
     a.wide = 0;
     if (d.group == -1 && j0 == 0) a.wide = 1;
     if (d.group > BW && (j0 % d.group) == 0) a.wide = 1;
@@ -400,7 +404,11 @@ kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
     KQ_LAUNCH_CHECK("sweep_block_kernel");
     const int64_t j1 = j0 + bw;
     if (j1 < n && !d.ordered) {
-      kronq_status r = trailing_update_tc(&maps, d.W, m, n, j1, bw, d.info, s);
+      // a block followed by columns is a full block, so K is a multiple of 128
+      const int64_t K = (int64_t)(a.slot + 1) * BW;
+      const bool group_end = (a.slot == d.gblocks - 1);
+      const int64_t ncols = group_end ? n - j1 : ((n - j1 < BW) ? n - j1 : BW);
+      kronq_status r = trailing_update_tc(&maps, d.W, m, n, j1, ncols, 0, K, d.info, s);
       if (r != KRONQ_OK) return r;
     } else if (j1 < n) {
       GemmDesc g;
