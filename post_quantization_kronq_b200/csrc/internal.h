@@ -165,9 +165,9 @@ struct SweepDesc {
   // tensor-core trailing updates (used unless ordered), two-level: bf16
   // hi/lo splits of the scaled errors (m x lde, lde = 128 gblocks) and of the
   // rows of U (128 gblocks x ldu) of the blocks of the current group of
-  // gblocks blocks.  After a block, the next block's columns get the update
-  // of every block of the group so far; at the group's end the columns past
-  // it get the whole group's update at once (K = 128 gblocks).
+  // gblocks blocks.  After a block, the group's later columns get its update
+  // (K = 128); at the group's end the columns past it get the whole group's
+  // update at once (K = 128 gblocks).
   __nv_bfloat16* Eh = nullptr;
   __nv_bfloat16* El = nullptr;
   __nv_bfloat16* Uh = nullptr;

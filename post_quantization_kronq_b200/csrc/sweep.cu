@@ -404,11 +404,15 @@ kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
     KQ_LAUNCH_CHECK("sweep_block_kernel");
     const int64_t j1 = j0 + bw;
     if (j1 < n && !d.ordered) {
-      // a block followed by columns is a full block, so K is a multiple of 128
-      const int64_t K = (int64_t)(a.slot + 1) * BW;
+      // Inside a group: this block's errors (K = 128) to the group's later
+      // columns.  At the group's end: the whole group (K = 128 gblocks) to
+      // every column past it.  (A block followed by columns is a full block.)
       const bool group_end = (a.slot == d.gblocks - 1);
-      const int64_t ncols = group_end ? n - j1 : ((n - j1 < BW) ? n - j1 : BW);
-      kronq_status r = trailing_update_tc(&maps, d.W, m, n, j1, ncols, 0, K, d.info, s);
+      const int64_t gend = j0 + (int64_t)(d.gblocks - a.slot) * BW;
+      const int64_t k0 = group_end ? 0 : (int64_t)a.slot * BW;
+      const int64_t K = group_end ? (int64_t)d.gblocks * BW : BW;
+      const int64_t ncols = group_end ? n - j1 : ((gend < n ? gend : n) - j1);
+      kronq_status r = trailing_update_tc(&maps, d.W, m, n, j1, ncols, k0, K, d.info, s);
       if (r != KRONQ_OK) return r;
     } else if (j1 < n) {
       GemmDesc g;
