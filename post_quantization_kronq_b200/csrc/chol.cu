@@ -458,46 +458,133 @@ __device__ __forceinline__ void panel_product(const DiagSmemP& S, int rg, int cg
   }
 }
 
-__device__ bool diag_step_p(DiagSmemP& S, float* H, int64_t n, int64_t j0, int nb, int* info,
-                            __nv_bfloat16* splits, float* stage, int cta, int ncta) {
+// ---- leader CTA: the chain of diagonal blocks -----------------------------
+// On entry S.x.a holds the diagonal block (upper triangle; identity beyond
+// nb), S.u is zero and S.bad is zero.  Factors and inverts it, stages U_JJ
+// (64 x 64 row-major at stage[j0 * 64]) and leaves U_JJ^T in S.y.wk.
+__device__ bool leader_factor(DiagSmemP& S, int64_t j0, int* info, float* stage) {
   const int tid = threadIdx.x;
-  // this CTA's rows: an even share of 0 .. j0, in multiples of 32
-  const int64_t per = (((j0 + ncta - 1) / ncta + 31) / 32) * 32;
-  const int64_t rbeg = (int64_t)cta * per;
-  const int64_t rend = (rbeg + per < j0) ? rbeg + per : j0;
-  if (rbeg < rend) fetch_rows(S, H, n, j0, nb, rbeg, rend);
+  if (!factor_invert_block(S)) {
+    if (tid == 0) *info = (int)(j0 + S.bad);
+    return false;  // uniform: read after the barrier
+  }
+  // all 64 x 64 (a short block's identity padding too: the panel CTAs
+  // multiply by the whole U_JJ; the staging area has room for it)
+  float* dst = stage + j0 * NB;
+  for (int t = tid; t < NB * NB; t += blockDim.x) {
+    const int k = t >> 6, c = t & 63;
+    S.y.wk[k][c] = S.u[c][k];
+    dst[t] = S.u[t >> 6][t & 63];
+  }
+  return true;
+}
+
+// The next diagonal block with this step's update folded in:
+//   P = A[j0 - 64 : j0, J] U_JJ^T   (those 64 rows of the panel; nb = width of J)
+//   S.x.a = A[J-1, J-1] - P P^T      (upper triangle)
+// A[J-1, J-1] must hold every update of the later steps (the Schur CTAs
+// leave this block out of step J's update).  The 64 rows of A are read by
+// leader_rows before the panel CTAs overwrite them with R.
+__device__ void leader_rows(DiagSmemP& S, const float* H, int64_t n, int64_t j0, int nb) {
+  const int tid = threadIdx.x;
+  const int64_t jp = j0 - NB;
+  const int r = tid >> 2, c0 = (tid & 3) * 16;
+  const float* src = H + (jp + r) * n + j0 + c0;
+  float v[16];
+#pragma unroll
+  for (int q = 0; q < 16; q += 4) {
+    if (c0 + q + 4 <= nb) {
+      const float4 x = *reinterpret_cast<const float4*>(src + q);
+      v[q] = x.x; v[q + 1] = x.y; v[q + 2] = x.z; v[q + 3] = x.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[q + e] = (c0 + q + e < nb) ? src[q + e] : 0.f;
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) S.ach[r][c0 + q] = v[q];
+  __syncthreads();
+}
+
+__device__ void leader_next(DiagSmemP& S, const float* H, int64_t n, int64_t j0) {
+  const int tid = threadIdx.x;
+  const int64_t jp = j0 - NB;
+  float acc[4][8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[j][q] = 0.f;
+  const int rg = tid >> 3, cg = tid & 7;
+  panel_product<2>(S, rg, cg, acc);
+  __syncthreads();  // U^T in wk is consumed
+  // P^T into wk: wk[k][r] = P[r][k]
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) S.y.wk[8 * cg + q][rg + 32 * j] = acc[j][q];
   {
     const int tx = tid & 63, ty = tid >> 6;
     float x[NB / 4];
 #pragma unroll
-    for (int sl = 0; sl < NB / 4; ++sl) {  // all loads in flight
+    for (int sl = 0; sl < NB / 4; ++sl) {
       const int r = 4 * sl + ty;
-      x[sl] = (r <= tx && tx < nb) ? H[(j0 + r) * n + j0 + tx] : 0.f;
+      x[sl] = (r <= tx) ? H[(jp + r) * n + jp + tx] : 0.f;
     }
 #pragma unroll
     for (int sl = 0; sl < NB / 4; ++sl) {
-      const int r = 4 * sl + ty;
-      S.x.a[r][tx] = (tx < nb) ? x[sl] : (r == tx ? 1.f : 0.f);
-      S.u[r][tx] = 0.f;
+      S.x.a[4 * sl + ty][tx] = x[sl];
+      S.u[4 * sl + ty][tx] = 0.f;
     }
   }
   if (tid == 0) S.bad = 0;
   __syncthreads();
-  if (!factor_invert_block(S)) {
-    if (tid == 0 && cta == 0) *info = (int)(j0 + S.bad);
-    return false;  // uniform: read after the barrier
+  // S.x.a -= P P^T on the upper triangle, 4 x 4 register tiles
+  {
+    const int tr = tid >> 4, tc = tid & 15;
+    if (tr <= tc) {
+      float t[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) t[i][j] = 0.f;
+#pragma unroll 4
+      for (int k = 0; k < NB; ++k) {
+        const float4 ra = *reinterpret_cast<const float4*>(&S.y.wk[k][4 * tr]);
+        const float4 rb = *reinterpret_cast<const float4*>(&S.y.wk[k][4 * tc]);
+        const float av[4] = {ra.x, ra.y, ra.z, ra.w}, bv[4] = {rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) t[i][j] = fmaf(av[i], bv[j], t[i][j]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (4 * tr + i <= 4 * tc + j) S.x.a[4 * tr + i][4 * tc + j] -= t[i][j];
+    }
   }
-  // U^T and the staged U_JJ
+  __syncthreads();
+}
+
+// ---- panel CTAs: R[i, J] = A[i, J] U_JJ^T for a share of the rows i < j0 ----
+// U_JJ comes from the leader's staging.  Rows arrive by cp.async in chunks
+// of 128 and are multiplied with 4 x 8 register tiles; the result goes to H
+// and, as bf16 hi/mid/lo splits, to the Schur tiles.
+__device__ void panel_rows(DiagSmemP& S, float* H, int64_t n, int64_t j0, int nb,
+                           __nv_bfloat16* splits, const float* stage, int pcta, int npan) {
+  const int tid = threadIdx.x;
+  // this CTA's rows: an even share of 0 .. j0, in multiples of 32
+  const int64_t per = (((j0 + npan - 1) / npan + 31) / 32) * 32;
+  const int64_t rbeg = (int64_t)pcta * per;
+  const int64_t rend = (rbeg + per < j0) ? rbeg + per : j0;
+  if (rbeg >= rend) return;
+  fetch_rows(S, H, n, j0, nb, rbeg, rend);
+  const float* src = stage + j0 * NB;
   for (int t = tid; t < NB * NB; t += blockDim.x) {
-    const int k = t >> 6, c = t & 63;
-    S.y.wk[k][c] = S.u[c][k];
+    const int c = t >> 6, k = t & 63;
+    S.y.wk[k][c] = src[t];  // U[c][k]
   }
-  if (cta == 0) {
-    float* dst = stage + j0 * NB;
-    for (int t = tid; t < nb * NB; t += blockDim.x) dst[t] = S.u[t >> 6][t & 63];
-  }
-  // Panel rows: R[i][c] = sum_k A[i][k] U[c][k]; thread: rows rg + 32 j
-  // (j < 4), columns 8 cg .. 8 cg + 7.
   const int64_t plane = (int64_t)n * NB;
   const int rg = tid >> 3, cg = tid & 7;
   for (int64_t r0 = rbeg; r0 < rend; r0 += PRF) {
@@ -550,7 +637,6 @@ __device__ bool diag_step_p(DiagSmemP& S, float* H, int64_t n, int64_t j0, int n
     }
   }
   cp_async_wait_all();
-  return true;
 }
 
 // Copy the staged diagonal blocks U_JJ into H (one CTA per block).  They are
@@ -598,9 +684,9 @@ struct PersistArgs {
   __nv_bfloat16* splits[2];
   float* stage;
   int* info;
-  int* ctr;     // panel_done[nblk], colready[nblk], schur_done[nblk], abort
+  int* ctr;     // panel_done, colready, schur_done, uready, diagready (nblk each), abort
   int vec4;
-  int ndiag;    // CTAs that run the diagonal steps
+  int npanel;   // CTAs that form the panel rows
 };
 
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
@@ -685,7 +771,9 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
   int* panel_done = a.ctr;
   int* colready = a.ctr + nblk;
   int* schur_done = a.ctr + 2 * nblk;
-  int* abortf = a.ctr + 3 * nblk;
+  int* uready = a.ctr + 3 * nblk;
+  int* diagready = a.ctr + 4 * nblk;
+  int* abortf = a.ctr + 5 * nblk;
 
   if (threadIdx.x == 0) {
     mbar_init(full, 1);
@@ -703,42 +791,79 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const schur::TileMaps maps[2] = {{&p0h, &p0m, &p0l, &mC}, {&p1h, &p1m, &p1l, &mC}};
   uint32_t tcount = 0;
-  // Roles: CTAs 0 .. nd-1 run the diagonal steps (each factors the block,
-  // they share the panel rows), the other ns CTAs the Schur tiles.
-  const int nd = a.ndiag, ns = ncta - nd;
+  // Roles: CTA 0 leads the chain of diagonal blocks, CTAs 1 .. npan form the
+  // panel rows, the rest run the Schur tiles.
+  const int npan = a.npanel, ns = ncta - 1 - npan;
 
   // nt(J): tiles per side of the update of step J (the upper triangle of j0 x j0)
   auto nt_of = [](int J) { return (J * NB + 127) / 128; };
 
-  if (cta < nd) {
+  if (cta == 0) {
+    // ---- leader
     DiagSmemP& F = *reinterpret_cast<DiagSmemP*>(smem);
+    {
+      const int64_t j0 = (int64_t)(nblk - 1) * NB;
+      const int nb = (int)(n - j0);
+      const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+      for (int sl = 0; sl < NB / 4; ++sl) {
+        const int r = 4 * sl + ty;
+        F.x.a[r][tx] = (tx < nb) ? ((r <= tx) ? a.H[(j0 + r) * n + j0 + tx] : 0.f) : (r == tx ? 1.f : 0.f);
+        F.u[r][tx] = 0.f;
+      }
+      if (threadIdx.x == 0) F.bad = 0;
+      __syncthreads();
+    }
     for (int J = nblk - 1; J >= 0; --J) {
-      // block J is final once the last tile column of step J + 1 is done;
-      // its split buffer is free once every tile of step J + 2 is done
-      if (J < nblk - 1 && !cta_wait(&colready[J], nt_of(J + 1), abortf)) break;
+      const int64_t j0 = (int64_t)J * NB;
+      const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
+      if (!leader_factor(F, j0, a.info, a.stage)) {
+        if (threadIdx.x == 0) atomicExch(abortf, 2);  // stop every other CTA
+        break;
+      }
+      if (J > 0) {
+        // the 64 panel rows of block J - 1 need step J + 1's last tile
+        // column; they are read before the panel CTAs may overwrite them
+        if (J + 1 <= nblk - 1 && !cta_wait(&colready[J], nt_of(J + 1), abortf)) break;
+        leader_rows(F, a.H, n, j0, nb);
+      }
+      cta_publish(&uready[J], nullptr);
+      if (J == 0) break;
+      // block J - 1's diagonal needs step J + 1's tile holding it
+      if (J + 1 <= nblk - 1 && !cta_wait(&diagready[J - 1], 1, abortf)) break;
+      leader_next(F, a.H, n, j0);
+    }
+  } else if (cta <= npan) {
+    // ---- panel rows
+    DiagSmemP& F = *reinterpret_cast<DiagSmemP*>(smem);
+    const int pc = cta - 1;
+    for (int J = nblk - 1; J >= 1; --J) {
+      if (!cta_wait(&uready[J], 1, abortf)) break;
+      if (J + 1 <= nblk - 1 && !cta_wait(&colready[J], nt_of(J + 1), abortf)) break;
       if (J + 2 <= nblk - 1 && !cta_wait(&schur_done[J + 2], tri_count(nt_of(J + 2)), abortf)) break;
       const int64_t j0 = (int64_t)J * NB;
       const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
-      if (!diag_step_p(F, a.H, n, j0, nb, a.info, a.splits[J & 1], a.stage, cta, nd)) {
-        // a non-positive pivot (seen by every diagonal CTA): stop the Schur CTAs too
-        if (threadIdx.x == 0) atomicExch(abortf, 2);
-        break;
-      }
+      panel_rows(F, a.H, n, j0, nb, a.splits[J & 1], a.stage, pc, npan);
       cta_publish(&panel_done[J], nullptr);
     }
   } else {
-    const int sc = cta - nd;
-    // One tile; a last-column tile is published at once (the next diagonal
-    // step waits for it), the bulk tiles of a step together at its end.
-    auto run_tile = [&](int J, int idx, bool last) -> bool {
+    // ---- Schur tiles
+    const int sc = cta - 1 - npan;
+    // One tile of step J; the last-column tiles and the tile holding block
+    // J - 2's diagonal are published at once (the panel CTAs and the leader
+    // wait for them), the bulk tiles of a step together at its end.
+    auto run_tile = [&](int J, int idx, bool last, bool diag) -> bool {
       int r, c;
       tri_rc(idx, r, c);
+      const bool urgent = last || diag;
       const bool ok = schur::tile<0, 8>(smem, full, cbar, accbar, tcount & 1u, tmem, maps[J & 1], a.H,
                                         n, (int64_t)J * NB, (int64_t)r * 128, (int64_t)c * 128, 1,
-                                        last ? 1 : 0);
+                                        urgent ? 1 : 0, (int64_t)(J - 1) * NB);
       ++tcount;
       tc_fence_before();
-      if (last) cta_publish(&colready[J - 1], &schur_done[J]);
+      if (urgent) {
+        cta_publish(&schur_done[J], last ? &colready[J - 1] : nullptr);
+        if (diag) cta_publish(&diagready[J - 2], nullptr);
+      }
       const int all = __syncthreads_and(ok ? 1 : 0);
       tc_fence_after();
       if (!all) {
@@ -751,13 +876,25 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
     for (int J = nblk - 1; ok && J >= 1; --J) {
       const int nt = nt_of(J);
       const int lo = tri_count(nt - 1), hi = tri_count(nt);
-      if (!cta_wait(&panel_done[J], nd, abortf)) break;
-      // the last tile column (holds block J - 1) first, then the others from
-      // the right, so the next step's last column comes early
-      for (int idx = lo + ((sc - lo % ns) % ns + ns) % ns; ok && idx < hi; idx += ns) ok = run_tile(J, idx, true);
+      // the tile holding block J - 2's diagonal (the leader needs it next)
+      int idx_d = -1;
+      if (J >= 2) {
+        const int d = ((J - 2) * NB) / 128;
+        idx_d = tri_count(d) + d;
+      }
+      if (!cta_wait(&panel_done[J], npan, abortf)) break;
+      // the last tile column (block J - 1's panel rows) first
+      for (int idx = lo + ((sc - lo % ns) % ns + ns) % ns; ok && idx < hi; idx += ns)
+        ok = run_tile(J, idx, true, idx == idx_d);
+      if (ok && idx_d >= 0 && idx_d < lo && idx_d % ns == sc) ok = run_tile(J, idx_d, false, true);
+      // the rest from the right
       const int top = lo - 1 - ((((lo - 1) - sc) % ns) + ns) % ns;   // largest idx < lo owned by sc
       int nbulk = 0;
-      for (int idx = top; ok && idx >= 0; idx -= ns, ++nbulk) ok = run_tile(J, idx, false);
+      for (int idx = top; ok && idx >= 0; idx -= ns) {
+        if (idx == idx_d) continue;
+        ok = run_tile(J, idx, false, false);
+        ++nbulk;
+      }
       if (!ok) break;
       if (nbulk > 0) {
         if (threadIdx.x == 0) tma_store_wait_all();   // the bulk tiles' stores reached memory
@@ -810,7 +947,7 @@ size_t chol_workspace_bytes(int64_t n) {
   // T / staging buffer, two buffers of bf16 hi/mid/lo panel splits
   // (3 x n x 64 each), the step counters of the persistent kernel
   const int64_t nblk = ceil_div(n, NB);
-  return tbuf_bytes(n) + 2 * splits_bytes(n) + (size_t)(3 * nblk + 4) * sizeof(int);
+  return tbuf_bytes(n) + 2 * splits_bytes(n) + (size_t)(5 * nblk + 4) * sizeof(int);
 }
 
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
@@ -855,7 +992,7 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
     SchurMaps maps1;
     kronq_status r = schur_maps(&maps1, splits1, H, n);
     if (r != KRONQ_OK) return r;
-    KQ_CUDA(cudaMemsetAsync(ctr, 0, (size_t)(3 * nblk + 4) * sizeof(int), s));
+    KQ_CUDA(cudaMemsetAsync(ctr, 0, (size_t)(5 * nblk + 4) * sizeof(int), s));
     const CUtensorMap* m0 = reinterpret_cast<const CUtensorMap*>(maps.raw);
     const CUtensorMap* m1 = reinterpret_cast<const CUtensorMap*>(maps1.raw);
     CUtensorMap a0 = m0[0], a1 = m0[1], a2 = m0[2], b0 = m1[0], b1 = m1[1], b2 = m1[2], c = m0[3];
@@ -869,7 +1006,7 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
     pa.info = info;
     pa.ctr = ctr;
     pa.vec4 = vec4;
-    pa.ndiag = (int)(pmax >= 64 ? 32 : pmax / 2);
+    pa.npanel = (int)(pmax >= 64 ? 31 : pmax / 2);
     void* args[] = {&a0, &a1, &a2, &b0, &b1, &b2, &c, &pa};
     KQ_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(&chol_persistent_kernel),
                                         dim3((unsigned)pmax), dim3(PERSIST_THREADS), args,

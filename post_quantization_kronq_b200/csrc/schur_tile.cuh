@@ -36,7 +36,7 @@ struct TileMaps {
 };
 
 // Processes one tile; every thread of the CTA calls it.  Entries i <= j < j0
-// are updated (j0 a multiple of 32).  Warp 0 lane 0
+// with i < rowlim (default j0) are updated (j0 a multiple of 32).  Warp 0 lane 0
 // issues the TMA loads, warp 1 lane 0 the MMAs; warps EPI_W0 .. EPI_W0+NW-1
 // (NW = 4 or 8; the role warps may be among them) run the epilogue, warp w
 // on TMEM lanes 32 (w % 4) and, with eight warps, on half of the columns.
@@ -50,7 +50,7 @@ template <int EPI_W0, int NW>
 __device__ __forceinline__ bool tile(uint8_t* smem, uint32_t full, uint32_t cbar, uint32_t accbar,
                                      uint32_t parity, uint32_t tmem, const TileMaps& mp, float* H,
                                      int64_t n, int64_t j0, int64_t r0, int64_t c0, int tma_c,
-                                     int store_done = 1) {
+                                     int store_done = 1, int64_t rowlim = -1) {
   static_assert(NW == 4 || NW == 8, "four or eight epilogue warps");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = smem_u32(smem);
@@ -111,8 +111,10 @@ __device__ __forceinline__ bool tile(uint8_t* smem, uint32_t full, uint32_t cbar
       tc_fence_after();
       const int i = (int)(r0 + rl);
       const int j0i = (int)j0;
-      // every entry of a tile strictly above the diagonal and left of j0 is updated
-      const bool interior = (r0 + BM <= c0) && (c0 + BN <= j0);
+      const int rlim = (int)(rowlim < 0 ? j0 : rowlim);
+      // every entry of a tile strictly above the diagonal, left of j0 and
+      // above the row limit is updated
+      const bool interior = (r0 + BM <= c0) && (c0 + BN <= j0) && (r0 + BM <= rlim);
 #pragma unroll 1
       for (int cc = ch0; cc < ch0 + NCH; ++cc) {
         uint32_t v[32];
@@ -134,7 +136,7 @@ __device__ __forceinline__ bool tile(uint8_t* smem, uint32_t full, uint32_t cbar
               *p4 = w;
             }
           } else {
-            const bool rowok = i < j0i;
+            const bool rowok = i < rlim;
 #pragma unroll
             for (int c4 = 0; c4 < 8; ++c4) {
               float4* p4 = reinterpret_cast<float4*>(box + sw128_f32(rl, 4 * c4));
@@ -147,7 +149,7 @@ __device__ __forceinline__ bool tile(uint8_t* smem, uint32_t full, uint32_t cbar
               *p4 = w;
             }
           }
-        } else if (i < j0i && jb < j0i && jb + 31 >= i) {
+        } else if (i < rlim && jb < j0i && jb + 31 >= i) {
           float* row = H + (int64_t)i * n + jb;
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
