@@ -506,22 +506,85 @@ __device__ void leader_rows(DiagSmemP& S, const float* H, int64_t n, int64_t j0,
   __syncthreads();
 }
 
-__device__ void leader_next(DiagSmemP& S, const float* H, int64_t n, int64_t j0) {
-  const int tid = threadIdx.x;
+// Tensor-core form of the two 64^3 products of the leader (P = A_rows U^T,
+// then S.x.a -= P P^T): operands split into bf16 hi/mid/lo in the UMMA
+// 128-byte-swizzled K-major layout (rows of 128 bytes), six split products
+// per 16-deep k step, M = 128 (rows 64 .. 127 of the A operand stay zero),
+// N = 64, accumulators in TMEM columns 0 .. 63 (P) and 64 .. 127 (P P^T).
+constexpr int LSPLIT_A = 128 * 128;            // 16 KB: 128 rows x 64 k bf16
+constexpr int LSPLIT_B = 64 * 128;             // 8 KB: 64 rows x 64 k bf16
+constexpr int LEAD_SPLIT_BYTES = 3 * LSPLIT_A + 3 * LSPLIT_B;   // 72 KB
+
+__device__ __forceinline__ uint32_t kmaj_off(int r, int k) {
+  return (uint32_t)(r * 128 + ((((k >> 3) ^ (r & 7))) << 4) + (k & 7) * 2);
+}
+
+// Splits four consecutive-k floats of row r into three bf16 planes.
+__device__ __forceinline__ void lsplit4(uint8_t* base, uint32_t plane, int r, int k, float4 v) {
+  const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y);
+  const __nv_bfloat162 h23 = __floats2bfloat162_rn(v.z, v.w);
+  const float r0 = v.x - __low2float(h01), r1 = v.y - __high2float(h01);
+  const float r2 = v.z - __low2float(h23), r3 = v.w - __high2float(h23);
+  const __nv_bfloat162 m01 = __floats2bfloat162_rn(r0, r1);
+  const __nv_bfloat162 m23 = __floats2bfloat162_rn(r2, r3);
+  const __nv_bfloat162 l01 = __floats2bfloat162_rn(r0 - __low2float(m01), r1 - __high2float(m01));
+  const __nv_bfloat162 l23 = __floats2bfloat162_rn(r2 - __low2float(m23), r3 - __high2float(m23));
+  auto bits = [](__nv_bfloat162 x) { return *reinterpret_cast<const uint32_t*>(&x); };
+  const uint32_t off = kmaj_off(r, k);
+  *reinterpret_cast<uint2*>(base + off) = make_uint2(bits(h01), bits(h23));
+  *reinterpret_cast<uint2*>(base + plane + off) = make_uint2(bits(m01), bits(m23));
+  *reinterpret_cast<uint2*>(base + 2 * plane + off) = make_uint2(bits(l01), bits(l23));
+}
+
+// One thread: the 24 MMAs of a 64-deep product, D[tmem_col ..] = A B^T.
+__device__ __forceinline__ void lead_mma(uint32_t tmem_d, uint32_t sa, uint32_t sb, uint32_t pb) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, false, false);
+  const int pa_[6] = {0, 0, 1, 0, 2, 1};
+  const int pb_[6] = {0, 1, 0, 2, 0, 1};
+  uint32_t acc = 0;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+    for (int t = 0; t < 6; ++t) {
+      const uint64_t da = smem_desc_sw128(sa + pa_[t] * LSPLIT_A + kk * 32, 16, 1024);
+      const uint64_t db = smem_desc_sw128(sb + pb_[t] * pb + kk * 32, 16, 1024);
+      mma_bf16(tmem_d, da, db, idesc, acc);
+      acc = 1;
+    }
+  }
+}
+
+// The next diagonal block: P = A[j0 - 64 : j0, J] U_JJ^T (rows in S.ach,
+// U_JJ in S.u), then S.x.a = A[J-1, J-1] - P P^T (upper triangle).  sp: the
+// 1024-aligned split area (its A rows 64 .. 127 are zero); bar: an mbarrier
+// of this CTA, par its next phase parity.  256 threads.
+__device__ bool leader_next(DiagSmemP& S, uint8_t* sp, uint32_t tmem, uint32_t bar, uint32_t& par,
+                            const float* H, int64_t n, int64_t j0) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t jp = j0 - NB;
-  float acc[4][8];
+  uint8_t* SA = sp;
+  uint8_t* SB = sp + 3 * LSPLIT_A;
+  const uint32_t sa = smem_u32(SA), sb = smem_u32(SB);
+  {
+    // splits of the 64 A rows and of U's rows (U[c][k]: B K-major)
+    const int r = tid >> 2, k0 = (tid & 3) * 16;
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int q = 0; q < 8; ++q) acc[j][q] = 0.f;
-  const int rg = tid >> 3, cg = tid & 7;
-  panel_product<2>(S, rg, cg, acc);
-  __syncthreads();  // U^T in wk is consumed
-  // P^T into wk: wk[k][r] = P[r][k]
-#pragma unroll
-  for (int j = 0; j < 2; ++j)
-#pragma unroll
-    for (int q = 0; q < 8; ++q) S.y.wk[8 * cg + q][rg + 32 * j] = acc[j][q];
+    for (int q = 0; q < 16; q += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(&S.ach[r][k0 + q]);
+      lsplit4(SA, LSPLIT_A, r, k0 + q, v);
+      const float4 w = make_float4(S.u[r][k0 + q], S.u[r][k0 + q + 1], S.u[r][k0 + q + 2], S.u[r][k0 + q + 3]);
+      lsplit4(SB, LSPLIT_B, r, k0 + q, w);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {
+    tc_fence_after();
+    lead_mma(tmem, sa, sb, LSPLIT_B);
+    mma_commit(bar);
+  }
+  // meanwhile: the diagonal block J - 1 from H, S.u cleared
   {
     const int tx = tid & 63, ty = tid >> 6;
     float x[NB / 4];
@@ -537,34 +600,65 @@ __device__ void leader_next(DiagSmemP& S, const float* H, int64_t n, int64_t j0)
     }
   }
   if (tid == 0) S.bad = 0;
-  __syncthreads();
-  // S.x.a -= P P^T on the upper triangle, 4 x 4 register tiles
-  {
-    const int tr = tid >> 4, tc = tid & 15;
-    if (tr <= tc) {
-      float t[4][4];
+  int good = 1;
+  if (warp < 2) {
+    if (lane == 0) good = mbar_wait(bar, par) ? 1 : 0;
+    good = __shfl_sync(0xffffffffu, good, 0);
+    __syncwarp();
+    if (good) {
+      tc_fence_after();
+      // P rows 32 warp + lane: two loads of 32 columns, then the splits of
+      // the row into SA (rows 0 .. 63; A and B of the second product)
+      const int r = 32 * warp + lane;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * h, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) t[i][j] = 0.f;
-#pragma unroll 4
-      for (int k = 0; k < NB; ++k) {
-        const float4 ra = *reinterpret_cast<const float4*>(&S.y.wk[k][4 * tr]);
-        const float4 rb = *reinterpret_cast<const float4*>(&S.y.wk[k][4 * tc]);
-        const float av[4] = {ra.x, ra.y, ra.z, ra.w}, bv[4] = {rb.x, rb.y, rb.z, rb.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) t[i][j] = fmaf(av[i], bv[j], t[i][j]);
+        for (int q = 0; q < 32; q += 4)
+          lsplit4(SA, LSPLIT_A, r, 32 * h + q,
+                  make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]), __uint_as_float(v[q + 2]),
+                              __uint_as_float(v[q + 3])));
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (4 * tr + i <= 4 * tc + j) S.x.a[4 * tr + i][4 * tc + j] -= t[i][j];
     }
   }
-  __syncthreads();
+  par ^= 1u;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  good = __syncthreads_and(good);
+  if (!good) return false;
+  if (tid == 0) {
+    tc_fence_after();
+    lead_mma(tmem + 64, sa, sa, LSPLIT_A);   // P P^T: B = the first 64 rows of P's splits
+    mma_commit(bar);
+  }
+  if (warp < 2) {
+    if (lane == 0) good = mbar_wait(bar, par) ? 1 : 0;
+    good = __shfl_sync(0xffffffffu, good, 0);
+    __syncwarp();
+    if (good) {
+      tc_fence_after();
+      const int r = 32 * warp + lane;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 64 + 32 * h, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const int c = 32 * h + q;
+          if (c >= r) S.x.a[r][c] -= __uint_as_float(v[q]);
+        }
+      }
+    }
+  }
+  par ^= 1u;
+  tc_fence_before();
+  good = __syncthreads_and(good);
+  return good != 0;
 }
 
 // ---- panel CTAs: R[i, J] = A[i, J] U_JJ^T for a share of the rows i < j0 ----
@@ -671,9 +765,10 @@ __global__ void __launch_bounds__(256) diag_store_kernel(float* H, int64_t n, co
 // Every wait is bounded; a timeout sets the device status and an abort flag
 // that ends every CTA's loop.
 constexpr int PERSIST_THREADS = 256;
-constexpr int PERSIST_BODY = ((size_t)schur::TILE_SMEM > sizeof(DiagSmemP))
-                                 ? (int)schur::TILE_SMEM
-                                 : (int)((sizeof(DiagSmemP) + 1023) & ~(size_t)1023);
+// the leader's split area sits after its DiagSmemP, 1024-aligned
+constexpr int LEAD_SPLIT_OFF = (int)((sizeof(DiagSmemP) + 1023) & ~(size_t)1023);
+constexpr int LEAD_BODY = LEAD_SPLIT_OFF + LEAD_SPLIT_BYTES;
+constexpr int PERSIST_BODY = (schur::TILE_SMEM > LEAD_BODY) ? schur::TILE_SMEM : LEAD_BODY;
 constexpr int PERSIST_SMEM = PERSIST_BODY + 1024 + 256;
 static_assert(sizeof(DiagSmemP) + 2048 + 256 <= 227 * 1024, "diagonal step fits one CTA's shared memory");
 
@@ -801,6 +896,11 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
   if (cta == 0) {
     // ---- leader
     DiagSmemP& F = *reinterpret_cast<DiagSmemP*>(smem);
+    uint8_t* sp = smem + LEAD_SPLIT_OFF;
+    uint32_t par = 0;
+    for (int t = threadIdx.x; t < LEAD_SPLIT_BYTES / 16; t += blockDim.x)
+      reinterpret_cast<uint4*>(sp)[t] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     {
       const int64_t j0 = (int64_t)(nblk - 1) * NB;
       const int nb = (int)(n - j0);
@@ -830,7 +930,10 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
       if (J == 0) break;
       // block J - 1's diagonal needs step J + 1's tile holding it
       if (J + 1 <= nblk - 1 && !cta_wait(&diagready[J - 1], 1, abortf)) break;
-      leader_next(F, a.H, n, j0);
+      if (!leader_next(F, sp, tmem, accbar, par, a.H, n, j0)) {
+        if (threadIdx.x == 0) atomicExch(abortf, 1);
+        break;
+      }
     }
   } else if (cta <= npan) {
     // ---- panel rows
