@@ -42,6 +42,10 @@ METRIC = "weights quantized/sec per layer (incl. H_X/H_G accumulation); % of roo
 UNIT = "weights/s"
 M = N_IN = 4096
 TOKENS = 131072
+# dram__bytes_read.sum / dram__bytes_write.sum of one syrk_bf16_tc_kernel launch
+# at T = 16384, d = 4096 (ncu, B200), used for roofline.traffic
+SYRK_READ_BYTES_T16384 = 225.659136e6
+SYRK_WRITE_BYTES_D4096 = 41.663232e6
 WORKLOAD = "llama2-7b q_proj 4096x4096, T=131072 tokens, W{bits} g{group} asym, BiIP full"
 
 
@@ -283,8 +287,14 @@ def run_kronq(args):
         peak, peak_src = peaks["bf16_tflops_sustained"], "measured (sustained bf16, MEASURED_PEAKS.json)"
     else:
         peak, peak_src = 1400.0, "fallback (sustained)"
+    # DRAM traffic per launch, from one ncu capture of the same kernel at
+    # T = 16384, d = 4096 (dram__bytes_read.sum 225.66 MB, dram__bytes_write.sum
+    # 41.66 MB): the token reads grow in proportion to T, the H write does not.
+    traffic = SYRK_READ_BYTES_T16384 * (TOKENS / 16384) + SYRK_WRITE_BYTES_D4096
     roofline = {"bound": "tensor", "kernel": "syrk_bf16_tc_kernel", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "traffic_source": "ncu capture at T=16384 (d=4096), reads scaled by T/16384",
+                "peak_source": peak_src,
                 "flops_per_launch": flops, "launch_ms": syrk_launch_ms}
 
     # End to end through the public API: inputs copied from pinned host memory
