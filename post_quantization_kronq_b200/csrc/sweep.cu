@@ -2,16 +2,26 @@
 //
 // KronQ README intro (extends GPTQ/GPTAQ) and "Reproduce from scratch"
 // (--w_bits --w_groupsize --w_asym).  Rows of W~ are independent once U is
-// known, so the in-block sweep runs one warp per pair of rows with no
-// block-wide synchronisation: eight lanes per row, lane q holds columns
-// 16q..16q+15 of the 128-column block.  The owner lane of a 16-column quarter
-// quantizes its columns one after the other, forming the scaled errors
-// e = (w - deq) / U_jj and updating its own later columns; then the sixteen
-// errors are shuffled to the row's other lanes, which apply them to their
-// (later) columns in column order.  All arithmetic of the sweep is single
-// float32 operations (multiply and subtract not fused; the per-column
-// divisions by the group scale and by U_jj are multiplications by their
-// correctly rounded reciprocals), so the result is reproducible bit for bit.
+// known, so the in-block sweep runs eight lanes per row and four rows per
+// warp with no block-wide synchronisation.  The 128 columns of a block are
+// dealt out round-robin: lane q holds columns q, q + 8, ..., q + 120 in
+// registers.  For column c, every lane evaluates the quantizer on its
+// register of that column (only the owner lane, q = c mod 8, keeps the
+// result), the owner's scaled error e = (w - deq) / U_cc is broadcast with
+// one shuffle, and every lane applies it to all of its later columns.  Since
+// each lane holds columns spread over the whole block, all eight lanes have
+// update work at every step.  Outside the ordered test mode the updates run
+// two columns at a time as packed float32x2 fused multiply-adds (sm_100).
+// The block is processed in four rounds of 32 columns; after a round the lane's four retired registers are stored and
+// the register file shifts down by four, so the code of one round serves all
+// four with static register indices.
+//
+// Arithmetic: the quantizer and the error are single float32 operations
+// (divisions by the group scale and by U_cc are multiplications by their
+// correctly rounded reciprocals).  In the ordered test mode each update is a
+// scalar product then a difference (one rounding each), in ascending column
+// order per element: bit for bit the float32 mirror.  Otherwise each update
+// is one packed fused multiply-add.
 //
 // After each block the later columns get W[:, later] -= E_blk U[blk, later]
 // (the lazy-batch update), either as a fast GEMM or, in the ordered test mode,
@@ -23,12 +33,20 @@ namespace kq {
 namespace {
 
 constexpr int BW = 128;        // block width (columns)
-constexpr int QW = 16;         // columns held by one lane
-constexpr int LPR = BW / QW;   // lanes per row (8)
+constexpr int LPR = 8;         // lanes per row
+constexpr int NREG = BW / LPR; // registers per lane: register k holds column 8k + q
+constexpr int RC = 32;         // columns per round
+constexpr int NROUND = BW / RC;
 constexpr int WARPS = 8;       // warps per CTA
 constexpr int ROWS_PER_CTA = WARPS * 32 / LPR;   // 32
-constexpr int US_LD = BW + 4 * (BW / QW);        // padded row of the U block (160 floats)
-constexpr int SWEEP_SMEM = BW * US_LD * sizeof(float) + BW * sizeof(float);  // + 1/U_jj
+// U block in shared memory, permuted: Up[c][q][k] = U[c][8k + q] for
+// 8k + q > c (zero on and below the diagonal and past the block), k < 16,
+// and zero for 16 <= k < 28 (the rounds read up to k = 4 R + 15).  A stride
+// of 28 floats puts the eight lanes of a row on distinct banks for the
+// 16-byte reads of one column.
+constexpr int UP_LD = 28;
+constexpr int UP_ROW = LPR * UP_LD;
+constexpr int SWEEP_SMEM = (BW * UP_ROW + BW) * (int)sizeof(float);
 
 struct BlockArgs {
   SweepDesc d;
@@ -56,19 +74,39 @@ __device__ __forceinline__ void grid_from_range(float lo, float hi, int bits, bo
   zero = asym ? rintf(__fdiv_rn(-xmin, scale)) : (float)(1 << (bits - 1));
 }
 
-// Grid of the group starting at column j of this block: the eight lanes of
-// the row reduce over their columns in [j, j + group).
-__device__ __forceinline__ void group_start(const float (&v)[QW], int j, int bw, int q,
+// Quantizer state of the current group.  The clamp of rint(w / scale) + zero
+// to [0, maxq] is applied as the clamp of rint(w / scale) to [-zero,
+// maxq - zero]: zero is an integer below 2^8, so both forms give the same
+// deq = scale (q - zero) and the same code q.
+struct Grid {
+  float sc, zp, isc, lo, hi;
+};
+
+__device__ __forceinline__ Grid make_grid(float sc, float zp, float maxq) {
+  Grid g;
+  g.sc = sc;
+  g.zp = zp;
+  g.isc = __frcp_rn(sc);
+  g.lo = __fsub_rn(0.f, zp);
+  g.hi = __fsub_rn(maxq, zp);
+  return g;
+}
+
+// Grid of the group that starts at block column cs: the eight lanes of the
+// row reduce over their registers in [cs, min(cs + group, bw)).  Register k
+// holds column 32 R + 8 k + q in round R.
+__device__ __forceinline__ Grid group_start(const float2 (&v2)[NREG / 2], int cs, int R, int q, int bw,
                                             const SweepDesc& d, bool live, int64_t r, int64_t gi,
-                                            float& sc, float& zp, float& isc) {
-  const int gend = (j + d.group < bw) ? j + d.group : bw;
+                                            float maxq) {
+  const int ce = min(cs + d.group, bw);
   float lo = INFINITY, hi = -INFINITY;
 #pragma unroll
-  for (int cc = 0; cc < QW; ++cc) {
-    const int col = q * QW + cc;
-    if (col >= j && col < gend) {
-      lo = fminf(lo, v[cc]);
-      hi = fmaxf(hi, v[cc]);
+  for (int k = 0; k < NREG; ++k) {
+    const int col = RC * R + 8 * k + q;
+    const float x = (k & 1) ? v2[k >> 1].y : v2[k >> 1].x;
+    if (col >= cs && col < ce) {
+      lo = fminf(lo, x);
+      hi = fmaxf(hi, x);
     }
   }
 #pragma unroll
@@ -76,34 +114,39 @@ __device__ __forceinline__ void group_start(const float (&v)[QW], int j, int bw,
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
     hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
+  float sc, zp;
   grid_from_range(lo, hi, d.bits, d.asym, sc, zp);
-  isc = __frcp_rn(sc);
   if (q == 0 && live) {
     d.scales[r * d.ngroups + gi] = sc;
     d.zeros[r * d.ngroups + gi] = zp;
   }
+  return make_grid(sc, zp, maxq);
 }
 
-// Column c of the block lives at Us[k * US_LD + ucol(c)]: 4 floats of padding
-// per 16 columns put the eight lanes of a row on different banks for the
-// float4 reads of one U row.
-__device__ __forceinline__ int ucol(int c) { return c + 4 * (c >> 4); }
+// v -= e u on a pair of columns, with ne = -e in both halves.  Ordered
+// mode: product then sum, each rounded (-(e u) rounds like e u), as scalar
+// operations that are never fused; otherwise one packed fused multiply-add.
+template <bool ORD>
+__device__ __forceinline__ void upd2(float2& v, float2 ne, float2 u) {
+  if (ORD) {
+    v.x = __fadd_rn(v.x, __fmul_rn(ne.x, u.x));
+    v.y = __fadd_rn(v.y, __fmul_rn(ne.y, u.y));
+  } else {
+    v = __ffma2_rn(ne, u, v);
+  }
+}
 
-// One block of 128 columns.  Eight lanes per row: lane q holds the row's
-// columns 16q .. 16q+15 in registers (v[]), so every step of the sequential
-// column loop is register arithmetic with static indices (the unrolled
-// 16-step body stays small enough for the instruction cache).  For each
-// quarter, the lane holding it quantizes its columns in order (forming
-// e = (w - deq) / U_jj and applying v[c] -= e * U[j][c] to its own later
-// columns), with no shuffle inside that dependency chain; the sixteen
-// errors are then shuffled to the later lanes at once.  Every update is a
-// multiply followed by a subtract, in ascending j per element: the
-// operation order of the float32 reference.
-template <bool SMALLG>
-__global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
+// One block of up to 128 columns.  GM: group - 1 for in-block groups of 16
+// to 128 columns (group starts known at compile time), -2 for in-block
+// groups of 1 to 8 columns (tested per column), -1 when the block's grid was
+// computed beforehand (one group per row, or groups wider than a block).
+template <bool ORD, int GM>
+__global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a) {
   const SweepDesc& d = a.d;
   if (d.info && *d.info != 0) return;
-  extern __shared__ __align__(16) float Us[];
+  extern __shared__ __align__(16) float smem[];
+  float* Up = smem;
+  float* iu = smem + BW * UP_ROW;
   const int tid = threadIdx.x, lane = tid & 31;
   const int q = lane & (LPR - 1);
   const int64_t n = d.n, j0 = a.j0;
@@ -111,33 +154,42 @@ __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
   const int64_t r = (int64_t)blockIdx.x * ROWS_PER_CTA + (tid >> 3);
   const bool live = r < d.m;
 
-  // U block (rows j0.., columns j0..j0+127, upper part) into shared memory.
-  // float4 loads, eight in flight per thread.
+  // U block (rows j0.., columns j0..j0+127, strictly upper part) into the
+  // permuted layout; 16-byte loads when rows are aligned (bw is then a
+  // multiple of 4, so a load never passes the block's last column).
   const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(d.U) & 15) == 0);
-  if (vec) {
-#pragma unroll 8
-    for (int it = 0; it < (BW * BW / 4) / (WARPS * 32); ++it) {
-      const int idx = it * (WARPS * 32) + tid;
-      const int k = idx >> 5, c = (idx & 31) * 4;
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (k < bw) x = *reinterpret_cast<const float4*>(d.U + (j0 + k) * n + j0 + c);
-      x.x = (c + 0 >= k && c + 0 < bw) ? x.x : 0.f;
-      x.y = (c + 1 >= k && c + 1 < bw) ? x.y : 0.f;
-      x.z = (c + 2 >= k && c + 2 < bw) ? x.z : 0.f;
-      x.w = (c + 3 >= k && c + 3 < bw) ? x.w : 0.f;
-      *reinterpret_cast<float4*>(Us + k * US_LD + ucol(c)) = x;
+#pragma unroll 4
+  for (int it = 0; it < (BW * BW / 4) / (WARPS * 32); ++it) {
+    const int idx = it * (WARPS * 32) + tid;
+    const int k = idx >> 5, c = (idx & 31) * 4;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (k < bw && c < bw) {
+      const float* src = d.U + (j0 + k) * n + j0 + c;
+      if (vec) {
+        const float4 t = *reinterpret_cast<const float4*>(src);
+        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = (c + i < bw) ? src[i] : 0.f;
+      }
     }
-  } else {
-    for (int t = tid; t < BW * BW; t += blockDim.x) {
-      const int k = t >> 7, c = t & (BW - 1);
-      Us[k * US_LD + ucol(c)] = (k < bw && c < bw && c >= k) ? d.U[(j0 + k) * n + j0 + c] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int cc = c + i;
+      Up[(k * LPR + (cc & 7)) * UP_LD + (cc >> 3)] = (cc > k && cc < bw) ? x[i] : 0.f;
     }
   }
+  for (int t = tid; t < BW * LPR * 3; t += WARPS * 32) {
+    const int row = t / 3, p = t - 3 * (t / 3);
+    *reinterpret_cast<float4*>(Up + row * UP_LD + NREG + 4 * p) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // correctly rounded reciprocals of the block's diagonal of U (0 past bw)
+  if (tid < BW) iu[tid] = (tid < bw) ? __frcp_rn(d.U[(j0 + tid) * n + j0 + tid]) : 0.f;
 
   // bf16 hi/lo copy of this block's rows of U, columns j1.. (operand B of
   // the tensor-core trailing update); rows are spread over the CTAs.
   const int64_t j1 = j0 + bw;
-  if (!d.ordered && j1 < n) {
+  if (!ORD && j1 < n) {
     for (int64_t k = blockIdx.x; k < bw; k += gridDim.x) {
       const float* src = d.U + (j0 + k) * n;
       __nv_bfloat16* dh = d.Uh + ((int64_t)a.slot * BW + k) * d.ldu;
@@ -168,162 +220,98 @@ __global__ void __launch_bounds__(WARPS * 32) sweep_block_kernel(BlockArgs a) {
     }
   }
 
-  float v[QW], ev[QW];
-  uint32_t code[QW / 4];
-  const float* wrow = d.W + r * n + j0 + q * QW;
-  if (live && q * QW + QW <= bw && vec) {
+  // The row's columns q, q + 8, ... (zero past bw, for dead columns and for
+  // rows past m).
+  float2 v2[NREG / 2];
+  const float* wrow = d.W + r * n + j0;
 #pragma unroll
-    for (int c = 0; c < QW; c += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(wrow + c);
-      v[c] = x.x; v[c + 1] = x.y; v[c + 2] = x.z; v[c + 3] = x.w;
+  for (int i = 0; i < NREG / 2; ++i) {
+    const int c0 = 16 * i + q, c1 = c0 + 8;
+    float x0 = (live && c0 < bw) ? wrow[c0] : 0.f;
+    float x1 = (live && c1 < bw) ? wrow[c1] : 0.f;
+    if (d.dead) {
+      if (live && c0 < bw && d.dead[j0 + c0]) x0 = 0.f;
+      if (live && c1 < bw && d.dead[j0 + c1]) x1 = 0.f;
     }
-  } else {
-#pragma unroll
-    for (int c = 0; c < QW; ++c) v[c] = (live && q * QW + c < bw) ? wrow[c] : 0.f;
+    v2[i] = make_float2(x0, x1);
   }
-#pragma unroll
-  for (int c = 0; c < QW; ++c) {
-    if (d.dead && live && q * QW + c < bw && d.dead[j0 + q * QW + c]) v[c] = 0.f;
-    ev[c] = 0.f;
-  }
-#pragma unroll
-  for (int c = 0; c < QW / 4; ++c) code[c] = 0;
-  float sc = 1.f, zp = 0.f;
-  if (a.wide && live) {
+  const float maxq = (float)((1 << d.bits) - 1);
+  Grid g = make_grid(1.f, 0.f, maxq);
+  if (GM == -1 && live) {
     const int64_t gi = (d.group == -1) ? 0 : j0 / d.group;
-    sc = d.scales[r * d.ngroups + gi];
-    zp = d.zeros[r * d.ngroups + gi];
+    g = make_grid(d.scales[r * d.ngroups + gi], d.zeros[r * d.ngroups + gi], maxq);
   }
-  float isc = __frcp_rn(sc);
-  // correctly rounded reciprocals of the block's diagonal of U
-  float* iu = Us + BW * US_LD;
-  if (tid < bw) iu[tid] = __frcp_rn(d.U[(j0 + tid) * n + j0 + tid]);
+  int gshift = 0;
+  while (GM != -1 && (1 << gshift) < d.group) ++gshift;
+  const int gmask = (GM == -1) ? 0 : d.group - 1;
+  const int64_t g0 = j0 >> gshift;
   __syncthreads();
 
-  const float maxq = (float)((1 << d.bits) - 1);
   const int src_base = lane & ~(LPR - 1);
-  // In-block groups divide 128, so they are powers of two starting at j0.
-  const bool inblock_groups = d.group > 0 && d.group <= BW;
-  const int gmask = inblock_groups ? d.group - 1 : 0;
-  int gshift = 0;
-  while (inblock_groups && (1 << gshift) < d.group) ++gshift;
-  const int64_t g0 = inblock_groups ? j0 >> gshift : 0;
-  for (int qo = 0; qo < LPR; ++qo) {
-    const bool all_later = q > qo;     // every column of this lane comes after the current quarter
-    const bool mine = q == qo;
-    // Groups of 16 or more columns can only start at a lane boundary.
-    if (!SMALLG && inblock_groups && qo * QW < bw && ((qo * QW) & gmask) == 0)
-      group_start(v, qo * QW, bw, q, d, live, r, g0 + ((qo * QW) >> gshift), sc, zp, isc);
-    // The owner lane sweeps its sixteen columns alone (no cross-lane step
-    // inside the sequential chain) ...
-    if (mine) {
-      const float* urow0 = Us + q * (QW + 4);
+  const int64_t wbase = r * n + j0;
+#pragma unroll 1
+  for (int R = 0; R < NROUND; ++R) {
+    const float* up = Up + (RC * R) * UP_ROW + q * UP_LD + 4 * R;
+    const float* iur = iu + RC * R;
+    float e4[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t code4 = 0;
 #pragma unroll
-      for (int c = 0; c < QW; ++c) {
-        const int j = qo * QW + c;
-        if (j >= bw) break;
-        if (SMALLG && (j & gmask) == 0) {
-          // a group of fewer than 16 columns lies inside this lane
-          float lo = INFINITY, hi = -INFINITY;
+    for (int t = 0; t < RC; ++t) {
+      const int kt = t >> 3, o = t & 7;
+      if (GM >= 0) {
+        if ((t & (GM & (RC - 1))) == 0 && ((RC * R) & GM) == 0 && RC * R + t < bw)
+          g = group_start(v2, RC * R + t, R, q, bw, d, live, r, g0 + ((RC * R + t) >> gshift), maxq);
+      } else if (GM == -2) {
+        if (((RC * R + t) & gmask) == 0 && RC * R + t < bw)
+          g = group_start(v2, RC * R + t, R, q, bw, d, live, r, g0 + ((RC * R + t) >> gshift), maxq);
+      }
+      // every lane evaluates the quantizer on its register of this column;
+      // the owner lane (q == o) keeps the result
+      const float w = (kt & 1) ? v2[kt >> 1].y : v2[kt >> 1].x;
+      const float rr = fminf(fmaxf(rintf(__fmul_rn(w, g.isc)), g.lo), g.hi);
+      const float deq = __fmul_rn(g.sc, rr);
+      const float ne = __fmul_rn(__fsub_rn(deq, w), iur[t]);   // -e, exactly
+      if (q == o) {
+        if (kt & 1) v2[kt >> 1].y = deq;
+        else v2[kt >> 1].x = deq;
+        e4[kt] = -ne;
+        code4 |= ((uint32_t)__fadd_rn(rr, g.zp) & 0xFFu) << (8 * kt);
+      }
+      const float nb = __shfl_sync(0xffffffffu, ne, src_base + o);
+      const float2 ne2 = make_float2(nb, nb);
+      // later columns: registers from kt on (U is zero on and below the
+      // diagonal, so earlier columns in the same pair are left unchanged)
+      const float4* u4 = reinterpret_cast<const float4*>(up + t * UP_ROW);
 #pragma unroll
-          for (int cc = c; cc < QW; ++cc)
-            if (cc < c + d.group && qo * QW + cc < bw) {
-              lo = fminf(lo, v[cc]);
-              hi = fmaxf(hi, v[cc]);
-            }
-          grid_from_range(lo, hi, d.bits, d.asym, sc, zp);
-          isc = __frcp_rn(sc);
-          if (live) {
-            const int64_t gi = g0 + (j >> gshift);
-            d.scales[r * d.ngroups + gi] = sc;
-            d.zeros[r * d.ngroups + gi] = zp;
+      for (int i = kt >> 2; i < NREG / 4; ++i) {
+        const float4 u = u4[i];
+        if (2 * i >= (kt >> 1)) upd2<ORD>(v2[2 * i], ne2, make_float2(u.x, u.y));
+        upd2<ORD>(v2[2 * i + 1], ne2, make_float2(u.z, u.w));
+      }
+    }
+    // retire registers 0..3: columns 32 R + 8 k + q
+    if (live) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int col = RC * R + 8 * k + q;
+        if (col < bw) {
+          const float x = (k & 1) ? v2[k >> 1].y : v2[k >> 1].x;
+          d.W[wbase + col] = x;
+          d.codes[wbase + col] = (uint8_t)((code4 >> (8 * k)) & 0xFFu);
+          if (a.Eb) a.Eb[r * a.lde + col] = e4[k];
+          if (!ORD) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(e4[k]);
+            const int64_t eo = r * d.lde + (int64_t)a.slot * BW + col;
+            d.Eh[eo] = h;
+            d.El[eo] = __float2bfloat16_rn(e4[k] - __bfloat162float(h));
           }
         }
-        const float w = v[c];
-        // division by scale and by U_jj as multiplication by the correctly
-        // rounded reciprocals (the float32 schedule of this library)
-        float qv = __fadd_rn(rintf(__fmul_rn(w, isc)), zp);
-        qv = fminf(fmaxf(qv, 0.f), maxq);
-        const float deq = __fmul_rn(sc, __fsub_rn(qv, zp));
-        const float e = __fmul_rn(__fsub_rn(w, deq), iu[j]);
-        v[c] = deq;
-        ev[c] = e;
-        code[c >> 2] |= ((uint32_t)qv & 0xFFu) << (8 * (c & 3));
-        const float* urow = urow0 + j * US_LD;
-#pragma unroll
-        for (int c4 = 0; c4 < QW; c4 += 4) {
-          if (c4 + 3 <= c) continue;
-          const float4 u4 = *reinterpret_cast<const float4*>(urow + c4);
-          const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t)
-            if (c4 + t > c) v[c4 + t] = __fsub_rn(v[c4 + t], __fmul_rn(e, uu[t]));
-        }
       }
     }
-    // ... then its sixteen errors go to the other lanes of the row, which
-    // apply them to their columns in ascending column order (the same
-    // operation sequence per element as a column-by-column update).
-    float eq[QW];
 #pragma unroll
-    for (int c = 0; c < QW; ++c) eq[c] = __shfl_sync(0xffffffffu, ev[c], src_base + qo);
-    if (all_later) {
-      const float* urow0 = Us + q * (QW + 4);
-#pragma unroll
-      for (int c = 0; c < QW; ++c) {
-        const int j = qo * QW + c;
-        if (j >= bw) break;
-        const float* urow = urow0 + j * US_LD;
-#pragma unroll
-        for (int c4 = 0; c4 < QW; c4 += 4) {
-          const float4 u4 = *reinterpret_cast<const float4*>(urow + c4);
-          v[c4 + 0] = __fsub_rn(v[c4 + 0], __fmul_rn(eq[c], u4.x));
-          v[c4 + 1] = __fsub_rn(v[c4 + 1], __fmul_rn(eq[c], u4.y));
-          v[c4 + 2] = __fsub_rn(v[c4 + 2], __fmul_rn(eq[c], u4.z));
-          v[c4 + 3] = __fsub_rn(v[c4 + 3], __fmul_rn(eq[c], u4.w));
-        }
-      }
-    }
-  }
-
-  if (!live) return;
-  const int64_t base = r * n + j0 + q * QW;
-  const bool full = (q * QW + QW <= bw);
-  if (full && ((reinterpret_cast<uintptr_t>(d.W + base) & 15) == 0)) {
-    float4* w4 = reinterpret_cast<float4*>(d.W + base);
-#pragma unroll
-    for (int c = 0; c < QW; c += 4) w4[c >> 2] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-  } else {
-#pragma unroll
-    for (int c = 0; c < QW; ++c)
-      if (q * QW + c < bw) d.W[base + c] = v[c];
-  }
-  if (full && ((reinterpret_cast<uintptr_t>(d.codes + base) & 15) == 0)) {
-    uint4* c4 = reinterpret_cast<uint4*>(d.codes + base);
-#pragma unroll
-    for (int t = 0; t < QW / 16; ++t)
-      c4[t] = make_uint4(code[4 * t], code[4 * t + 1], code[4 * t + 2], code[4 * t + 3]);
-  } else {
-#pragma unroll
-    for (int c = 0; c < QW; ++c)
-      if (q * QW + c < bw) d.codes[base + c] = (uint8_t)((code[c >> 2] >> (8 * (c & 3))) & 0xFFu);
-  }
-  if (a.Eb) {
-#pragma unroll
-    for (int c = 0; c < QW; ++c)
-      if (q * QW + c < bw) a.Eb[r * a.lde + q * QW + c] = ev[c];
-  }
-  if (!d.ordered) {
-    __nv_bfloat16* eh = d.Eh + r * d.lde + (int64_t)a.slot * BW + q * QW;
-    __nv_bfloat16* el = d.El + r * d.lde + (int64_t)a.slot * BW + q * QW;
-#pragma unroll
-    for (int c = 0; c < QW; c += 2) {
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(ev[c]), h1 = __float2bfloat16_rn(ev[c + 1]);
-      const __nv_bfloat16 l0 = __float2bfloat16_rn(ev[c] - __bfloat162float(h0));
-      const __nv_bfloat16 l1 = __float2bfloat16_rn(ev[c + 1] - __bfloat162float(h1));
-      *reinterpret_cast<__nv_bfloat162*>(eh + c) = __halves2bfloat162(h0, h1);
-      *reinterpret_cast<__nv_bfloat162*>(el + c) = __halves2bfloat162(l0, l1);
-    }
+    for (int i = 0; i < NREG / 2 - 2; ++i) v2[i] = v2[i + 2];
+    v2[NREG / 2 - 2] = make_float2(0.f, 0.f);
+    v2[NREG / 2 - 1] = make_float2(0.f, 0.f);
   }
 }
 
@@ -354,13 +342,33 @@ __global__ void group_params_kernel(SweepDesc d, int64_t j0, int64_t gw, int64_t
   }
 }
 
+template <bool ORD, int GM>
+cudaError_t launch_gm(const BlockArgs& a, unsigned grid, cudaStream_t s) {
+  const void* fn = reinterpret_cast<const void*>(&sweep_block_kernel<ORD, GM>);
+  cudaError_t e = allow_smem(fn, SWEEP_SMEM);
+  if (e != cudaSuccess) return e;
+  sweep_block_kernel<ORD, GM><<<grid, WARPS * 32, SWEEP_SMEM, s>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Picks the instance for the block's group layout.
+template <bool ORD>
+cudaError_t launch_block(const BlockArgs& a, unsigned grid, cudaStream_t s) {
+  if (a.wide) return launch_gm<ORD, -1>(a, grid, s);
+  switch (a.d.group) {
+    case 128: return launch_gm<ORD, 127>(a, grid, s);
+    case 64: return launch_gm<ORD, 63>(a, grid, s);
+    case 32: return launch_gm<ORD, 31>(a, grid, s);
+    case 16: return launch_gm<ORD, 15>(a, grid, s);
+    default: return launch_gm<ORD, -2>(a, grid, s);
+  }
+}
+
 }  // namespace
 
 kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
   const int64_t n = d.n, m = d.m;
-  cudaError_t ea = allow_smem(reinterpret_cast<const void*>(&sweep_block_kernel<false>), SWEEP_SMEM);
-  if (ea == cudaSuccess) ea = allow_smem(reinterpret_cast<const void*>(&sweep_block_kernel<true>), SWEEP_SMEM);
-  if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(sweep)");
   const unsigned grid = (unsigned)ceil_div(m, ROWS_PER_CTA);
   TrailingMaps maps;
   if (!d.ordered && n > BW) {
@@ -397,11 +405,8 @@ kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
       a.Eb = nullptr;   // the tensor-core update reads the bf16 hi/lo copies
       a.lde = BW;
     }
-    if (d.group > 0 && d.group < QW)
-      sweep_block_kernel<true><<<grid, WARPS * 32, SWEEP_SMEM, s>>>(a);
-    else
-      sweep_block_kernel<false><<<grid, WARPS * 32, SWEEP_SMEM, s>>>(a);
-    KQ_LAUNCH_CHECK("sweep_block_kernel");
+    cudaError_t el = d.ordered ? launch_block<true>(a, grid, s) : launch_block<false>(a, grid, s);
+    if (el != cudaSuccess) return cuda_fail(el, "sweep_block_kernel");
     const int64_t j1 = j0 + bw;
     if (j1 < n && !d.ordered) {
       // Inside a group: this block's errors (K = 128) to the group's later
