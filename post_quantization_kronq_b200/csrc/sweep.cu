@@ -80,6 +80,7 @@ __device__ __forceinline__ void grid_from_range(float lo, float hi, int bits, bo
 // deq = scale (q - zero) and the same code q.
 struct Grid {
   float sc, zp, isc, lo, hi;
+  float zp2;   // zero + 2^23: the code q = rr + zero is the low byte of rr + zp2
 };
 
 __device__ __forceinline__ Grid make_grid(float sc, float zp, float maxq) {
@@ -89,6 +90,7 @@ __device__ __forceinline__ Grid make_grid(float sc, float zp, float maxq) {
   g.isc = __frcp_rn(sc);
   g.lo = __fsub_rn(0.f, zp);
   g.hi = __fsub_rn(maxq, zp);
+  g.zp2 = __fadd_rn(zp, 8388608.f);
   return g;
 }
 
@@ -136,14 +138,31 @@ __device__ __forceinline__ void upd2(float2& v, float2 ne, float2 u) {
   }
 }
 
+// rint for the quantizer: adding and removing 1.5 * 2^23 rounds to the
+// nearest integer, ties to even, for |x| < 2^22 (two adds on the FMA pipe).
+// Larger |x| give values beyond any grid, which the clamp that follows maps
+// to the same end point as rint would.
+__device__ __forceinline__ float rint_grid(float x) {
+  return __fsub_rn(__fadd_rn(x, 12582912.f), 12582912.f);
+}
+
 // One block of up to 128 columns.  GM: group - 1 for in-block groups of 16
 // to 128 columns (group starts known at compile time), -2 for in-block
 // groups of 1 to 8 columns (tested per column), -1 when the block's grid was
 // computed beforehand (one group per row, or groups wider than a block).
+//
+// Besides its strided registers, every lane of a row holds a window of the
+// row's next two columns c and c + 1, so all eight lanes evaluate the
+// quantizer of column c on the same value and get the same error without a
+// cross-lane step in the column chain.  After column c the window's column
+// c + 1 takes its update, and the owner of column c + 2 (whose register now
+// has every update up to column c) hands its value to the row's lanes with
+// one shuffle, which is needed only after column c + 1's quantizer.  The
+// window and the owner's register receive the same updates in the same
+// order, so they hold the same value.
 template <bool ORD, int GM>
 __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a) {
   const SweepDesc& d = a.d;
-  if (d.info && *d.info != 0) return;
   extern __shared__ __align__(16) float smem[];
   float* Up = smem;
   float* iu = smem + BW * UP_ROW;
@@ -153,26 +172,55 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
   const int bw = a.bw;
   const int64_t r = (int64_t)blockIdx.x * ROWS_PER_CTA + (tid >> 3);
   const bool live = r < d.m;
-
-  // U block (rows j0.., columns j0..j0+127, strictly upper part) into the
-  // permuted layout; 16-byte loads when rows are aligned (bw is then a
-  // multiple of 4, so a load never passes the block's last column).
   const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(d.U) & 15) == 0);
-#pragma unroll 4
+
+  // Issue every load of the block's inputs first: the U block (16-byte
+  // loads when rows are aligned; bw is then a multiple of 4, so a load never
+  // passes the block's last column), U's diagonal and the row's columns q,
+  // q + 8, ... (zero past bw, for dead columns and for rows past m).
+  float4 ub[(BW * BW / 4) / (WARPS * 32)];
+#pragma unroll
   for (int it = 0; it < (BW * BW / 4) / (WARPS * 32); ++it) {
     const int idx = it * (WARPS * 32) + tid;
     const int k = idx >> 5, c = (idx & 31) * 4;
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    ub[it] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (k < bw && c < bw) {
       const float* src = d.U + (j0 + k) * n + j0 + c;
       if (vec) {
-        const float4 t = *reinterpret_cast<const float4*>(src);
-        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+        ub[it] = *reinterpret_cast<const float4*>(src);
       } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = (c + i < bw) ? src[i] : 0.f;
+        ub[it].x = src[0];
+        ub[it].y = (c + 1 < bw) ? src[1] : 0.f;
+        ub[it].z = (c + 2 < bw) ? src[2] : 0.f;
+        ub[it].w = (c + 3 < bw) ? src[3] : 0.f;
       }
     }
+  }
+  const float udiag = (tid < bw) ? d.U[(j0 + tid) * n + j0 + tid] : 1.f;
+  float2 v2[NREG / 2];
+  const float* wrow = d.W + r * n + j0;
+#pragma unroll
+  for (int i = 0; i < NREG / 2; ++i) {
+    const int c0 = 16 * i + q, c1 = c0 + 8;
+    v2[i] = make_float2((live && c0 < bw) ? wrow[c0] : 0.f, (live && c1 < bw) ? wrow[c1] : 0.f);
+  }
+  if (d.info && *d.info != 0) return;
+  if (d.dead) {
+#pragma unroll
+    for (int i = 0; i < NREG / 2; ++i) {
+      const int c0 = 16 * i + q, c1 = c0 + 8;
+      if (c0 < bw && d.dead[j0 + c0]) v2[i].x = 0.f;
+      if (c1 < bw && d.dead[j0 + c1]) v2[i].y = 0.f;
+    }
+  }
+
+  // U block into the permuted layout (strictly upper part), zero pads, and
+  // the correctly rounded reciprocals of the diagonal (0 past bw).
+#pragma unroll
+  for (int it = 0; it < (BW * BW / 4) / (WARPS * 32); ++it) {
+    const int idx = it * (WARPS * 32) + tid;
+    const int k = idx >> 5, c = (idx & 31) * 4;
+    const float x[4] = {ub[it].x, ub[it].y, ub[it].z, ub[it].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int cc = c + i;
@@ -183,8 +231,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
     const int row = t / 3, p = t - 3 * (t / 3);
     *reinterpret_cast<float4*>(Up + row * UP_LD + NREG + 4 * p) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // correctly rounded reciprocals of the block's diagonal of U (0 past bw)
-  if (tid < BW) iu[tid] = (tid < bw) ? __frcp_rn(d.U[(j0 + tid) * n + j0 + tid]) : 0.f;
+  if (tid < BW) iu[tid] = (tid < bw) ? __frcp_rn(udiag) : 0.f;
 
   // bf16 hi/lo copy of this block's rows of U, columns j1.. (operand B of
   // the tensor-core trailing update); rows are spread over the CTAs.
@@ -220,21 +267,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
     }
   }
 
-  // The row's columns q, q + 8, ... (zero past bw, for dead columns and for
-  // rows past m).
-  float2 v2[NREG / 2];
-  const float* wrow = d.W + r * n + j0;
-#pragma unroll
-  for (int i = 0; i < NREG / 2; ++i) {
-    const int c0 = 16 * i + q, c1 = c0 + 8;
-    float x0 = (live && c0 < bw) ? wrow[c0] : 0.f;
-    float x1 = (live && c1 < bw) ? wrow[c1] : 0.f;
-    if (d.dead) {
-      if (live && c0 < bw && d.dead[j0 + c0]) x0 = 0.f;
-      if (live && c1 < bw && d.dead[j0 + c1]) x1 = 0.f;
-    }
-    v2[i] = make_float2(x0, x1);
-  }
   const float maxq = (float)((1 << d.bits) - 1);
   Grid g = make_grid(1.f, 0.f, maxq);
   if (GM == -1 && live) {
@@ -249,45 +281,60 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
 
   const int src_base = lane & ~(LPR - 1);
   const int64_t wbase = r * n + j0;
+  // the window: columns 0 and 1 (register 0 of lanes 0 and 1)
+  float win[2];
+  win[0] = __shfl_sync(0xffffffffu, v2[0].x, src_base + 0);
+  win[1] = __shfl_sync(0xffffffffu, v2[0].x, src_base + 1);
 #pragma unroll 1
   for (int R = 0; R < NROUND; ++R) {
     const float* up = Up + (RC * R) * UP_ROW + q * UP_LD + 4 * R;
+    const float* upw = Up + (RC * R) * UP_ROW + 4 * R;
     const float* iur = iu + RC * R;
     float e4[4] = {0.f, 0.f, 0.f, 0.f};
     uint32_t code4 = 0;
 #pragma unroll
     for (int t = 0; t < RC; ++t) {
       const int kt = t >> 3, o = t & 7;
+      bool gs = false;
       if (GM >= 0) {
-        if ((t & (GM & (RC - 1))) == 0 && ((RC * R) & GM) == 0 && RC * R + t < bw)
-          g = group_start(v2, RC * R + t, R, q, bw, d, live, r, g0 + ((RC * R + t) >> gshift), maxq);
+        gs = (t & (GM & (RC - 1))) == 0 && ((RC * R) & GM) == 0 && RC * R + t < bw;
       } else if (GM == -2) {
-        if (((RC * R + t) & gmask) == 0 && RC * R + t < bw)
-          g = group_start(v2, RC * R + t, R, q, bw, d, live, r, g0 + ((RC * R + t) >> gshift), maxq);
+        gs = ((RC * R + t) & gmask) == 0 && RC * R + t < bw;
       }
-      // every lane evaluates the quantizer on its register of this column;
-      // the owner lane (q == o) keeps the result
-      const float w = (kt & 1) ? v2[kt >> 1].y : v2[kt >> 1].x;
-      const float rr = fminf(fmaxf(rintf(__fmul_rn(w, g.isc)), g.lo), g.hi);
+      if (gs) g = group_start(v2, RC * R + t, R, q, bw, d, live, r, g0 + ((RC * R + t) >> gshift), maxq);
+      // the quantizer of column c on the window (the same value in every
+      // lane of the row)
+      const float w = win[t & 1];
+      const float rr = fminf(fmaxf(rint_grid(__fmul_rn(w, g.isc)), g.lo), g.hi);
       const float deq = __fmul_rn(g.sc, rr);
-      const float ne = __fmul_rn(__fsub_rn(deq, w), iur[t]);   // -e, exactly
+      const float ne = ORD ? __fmul_rn(__fsub_rn(deq, w), iur[t])       // -e, exactly
+                           : __fmul_rn(fmaf(g.sc, rr, -w), iur[t]);
+      // column c + 1 in the window: U[c][c + 1]
+      const float uw = upw[t * UP_ROW + ((t + 1) & 7) * UP_LD + ((t + 1) >> 3)];
+      win[(t + 1) & 1] = ORD ? __fadd_rn(win[(t + 1) & 1], __fmul_rn(ne, uw)) : fmaf(ne, uw, win[(t + 1) & 1]);
+      // the owner lane keeps the result of its column
       if (q == o) {
         if (kt & 1) v2[kt >> 1].y = deq;
         else v2[kt >> 1].x = deq;
         e4[kt] = -ne;
-        code4 |= ((uint32_t)__fadd_rn(rr, g.zp) & 0xFFu) << (8 * kt);
+        code4 |= (__float_as_uint(__fadd_rn(rr, g.zp2)) & 0xFFu) << (8 * kt);
       }
-      const float nb = __shfl_sync(0xffffffffu, ne, src_base + o);
-      const float2 ne2 = make_float2(nb, nb);
-      // later columns: registers from kt on (U is zero on and below the
-      // diagonal, so earlier columns in the same pair are left unchanged)
+      // later columns in the strided registers: from register kt on (U is
+      // zero on and below the diagonal, so earlier columns in the same pair
+      // are left unchanged)
+      const float2 ne2 = make_float2(ne, ne);
       const float4* u4 = reinterpret_cast<const float4*>(up + t * UP_ROW);
 #pragma unroll
-      for (int i = kt >> 2; i < NREG / 4; ++i) {
+      for (int i = 0; i < NREG / 4; ++i) {
         const float4 u = u4[i];
         if (2 * i >= (kt >> 1)) upd2<ORD>(v2[2 * i], ne2, make_float2(u.x, u.y));
         upd2<ORD>(v2[2 * i + 1], ne2, make_float2(u.z, u.w));
       }
+      // column c + 2 (updated up to column c) from its owner into the slot
+      // column c leaves
+      const int k2 = (t + 2) >> 3, o2 = (t + 2) & 7;
+      const float x2 = (k2 & 1) ? v2[k2 >> 1].y : v2[k2 >> 1].x;
+      win[t & 1] = __shfl_sync(0xffffffffu, x2, src_base + o2);
     }
     // retire registers 0..3: columns 32 R + 8 k + q
     if (live) {
