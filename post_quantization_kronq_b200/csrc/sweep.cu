@@ -2,26 +2,30 @@
 //
 // KronQ README intro (extends GPTQ/GPTAQ) and "Reproduce from scratch"
 // (--w_bits --w_groupsize --w_asym).  Rows of W~ are independent once U is
-// known, so the in-block sweep runs eight lanes per row and four rows per
-// warp with no block-wide synchronisation.  The 128 columns of a block are
-// dealt out round-robin: lane q holds columns q, q + 8, ..., q + 120 in
-// registers.  For column c, every lane evaluates the quantizer on its
-// register of that column (only the owner lane, q = c mod 8, keeps the
-// result), the owner's scaled error e = (w - deq) / U_cc is broadcast with
-// one shuffle, and every lane applies it to all of its later columns.  Since
-// each lane holds columns spread over the whole block, all eight lanes have
-// update work at every step.  Outside the ordered test mode the updates run
-// two columns at a time as packed float32x2 fused multiply-adds (sm_100).
-// The block is processed in four rounds of 32 columns; after a round the lane's four retired registers are stored and
-// the register file shifts down by four, so the code of one round serves all
-// four with static register indices.
+// known, so the in-block sweep needs no block-wide synchronisation.  Sixteen
+// lanes share a pair of rows: lane q holds, for both rows, the columns q,
+// q + 16, ..., q + 112 of the 128-column block in registers, so every lane
+// has later columns to update at every step and each value of U read from
+// shared memory serves two rows.
+//
+// Every lane also holds a window of each row's next two columns c and
+// c + 1, so the sixteen lanes evaluate the quantizer of column c on the same
+// value and get the same scaled error e = (w - deq) / U_cc without a
+// cross-lane step in the column chain.  After column c the window's column
+// c + 1 takes its update, and the owner of column c + 2 (whose register now
+// has every update up to column c) hands its value over with one shuffle,
+// needed only after column c + 1's quantizer.  Window and owner register
+// receive the same updates in the same order, so they hold the same value.
+// The block runs in four rounds of 32 columns; after a round the two retired
+// registers of each row are stored and the registers shift down by two, so
+// one round's code serves all four with static register indices.
 //
 // Arithmetic: the quantizer and the error are single float32 operations
 // (divisions by the group scale and by U_cc are multiplications by their
 // correctly rounded reciprocals).  In the ordered test mode each update is a
-// scalar product then a difference (one rounding each), in ascending column
-// order per element: bit for bit the float32 mirror.  Otherwise each update
-// is one packed fused multiply-add.
+// product then a difference (one rounding each), in ascending column order
+// per element: bit for bit the float32 mirror.  Otherwise each update is one
+// fused multiply-add, two columns at a time as packed float32x2 (sm_100).
 //
 // After each block the later columns get W[:, later] -= E_blk U[blk, later]
 // (the lazy-batch update), either as a fast GEMM or, in the ordered test mode,
@@ -33,20 +37,23 @@ namespace kq {
 namespace {
 
 constexpr int BW = 128;        // block width (columns)
-constexpr int LPR = 8;         // lanes per row
-constexpr int NREG = BW / LPR; // registers per lane: register k holds column 8k + q
+constexpr int LPR = 16;        // lanes per pair of rows
+constexpr int NREG = BW / LPR; // registers per row and lane: register k holds column 16k + q
+constexpr int NP = NREG / 2;   // register pairs per row
 constexpr int RC = 32;         // columns per round
 constexpr int NROUND = BW / RC;
+constexpr int RET = RC / LPR;  // registers retired per round (one pair)
 constexpr int WARPS = 8;       // warps per CTA
-constexpr int ROWS_PER_CTA = WARPS * 32 / LPR;   // 32
-// U block in shared memory, permuted: Up[c][q][k] = U[c][8k + q] for
-// 8k + q > c (zero on and below the diagonal and past the block), k < 16,
-// and zero for 16 <= k < 28 (the rounds read up to k = 4 R + 15).  A stride
-// of 28 floats puts the eight lanes of a row on distinct banks for the
-// 16-byte reads of one column.
-constexpr int UP_LD = 28;
+constexpr int ROWS_PER_CTA = WARPS * 32 / LPR * 2;   // 32
+// U block in shared memory, permuted: Up[c][q][k] = U[c][16k + q] for
+// 16k + q > c (zero on and below the diagonal and past the block), k < 8,
+// and zero for 8 <= k < 14 (round R reads k = 2R .. 2R + 7).  A stride of 18
+// floats puts the sixteen lanes of a half warp on distinct bank pairs for
+// the 8-byte reads of one column.
+constexpr int UP_LD = 18;
 constexpr int UP_ROW = LPR * UP_LD;
 constexpr int SWEEP_SMEM = (BW * UP_ROW + BW) * (int)sizeof(float);
+constexpr int UB_PER_THREAD = (BW * BW / 4) / (WARPS * 32);   // float4 loads of the U block
 
 struct BlockArgs {
   SweepDesc d;
@@ -94,18 +101,22 @@ __device__ __forceinline__ Grid make_grid(float sc, float zp, float maxq) {
   return g;
 }
 
-// Grid of the group that starts at block column cs: the eight lanes of the
-// row reduce over their registers in [cs, min(cs + group, bw)).  Register k
-// holds column 32 R + 8 k + q in round R.
-__device__ __forceinline__ Grid group_start(const float2 (&v2)[NREG / 2], int cs, int R, int q, int bw,
+__device__ __forceinline__ float reg_of(const float2 (&v)[NP], int k) {
+  return (k & 1) ? v[k >> 1].y : v[k >> 1].x;
+}
+
+// Grid of the group that starts at block column cs, for one row: the
+// sixteen lanes reduce over their registers in [cs, min(cs + group, bw)).
+// Register k holds column 32 R + 16 k + q in round R.
+__device__ __forceinline__ Grid group_start(const float2 (&v)[NP], int cs, int R, int q, int bw,
                                             const SweepDesc& d, bool live, int64_t r, int64_t gi,
                                             float maxq) {
   const int ce = min(cs + d.group, bw);
   float lo = INFINITY, hi = -INFINITY;
 #pragma unroll
   for (int k = 0; k < NREG; ++k) {
-    const int col = RC * R + 8 * k + q;
-    const float x = (k & 1) ? v2[k >> 1].y : v2[k >> 1].x;
+    const int col = RC * R + LPR * k + q;
+    const float x = reg_of(v, k);
     if (col >= cs && col < ce) {
       lo = fminf(lo, x);
       hi = fmaxf(hi, x);
@@ -138,6 +149,11 @@ __device__ __forceinline__ void upd2(float2& v, float2 ne, float2 u) {
   }
 }
 
+template <bool ORD>
+__device__ __forceinline__ float upd1(float v, float ne, float u) {
+  return ORD ? __fadd_rn(v, __fmul_rn(ne, u)) : fmaf(ne, u, v);
+}
+
 // rint for the quantizer: adding and removing 1.5 * 2^23 rounds to the
 // nearest integer, ties to even, for |x| < 2^22 (two adds on the FMA pipe).
 // Larger |x| give values beyond any grid, which the clamp that follows maps
@@ -146,22 +162,30 @@ __device__ __forceinline__ float rint_grid(float x) {
   return __fsub_rn(__fadd_rn(x, 12582912.f), 12582912.f);
 }
 
+// bf16 hi/lo split of one float4 into 4 + 4 bf16.
+__device__ __forceinline__ void split4(float4 x, __nv_bfloat16* dh, __nv_bfloat16* dl) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(x.x), h1 = __float2bfloat16_rn(x.y);
+  const __nv_bfloat16 h2 = __float2bfloat16_rn(x.z), h3 = __float2bfloat16_rn(x.w);
+  __nv_bfloat162 hh[2] = {__halves2bfloat162(h0, h1), __halves2bfloat162(h2, h3)};
+  __nv_bfloat162 ll[2] = {
+      __halves2bfloat162(__float2bfloat16_rn(x.x - __bfloat162float(h0)),
+                         __float2bfloat16_rn(x.y - __bfloat162float(h1))),
+      __halves2bfloat162(__float2bfloat16_rn(x.z - __bfloat162float(h2)),
+                         __float2bfloat16_rn(x.w - __bfloat162float(h3)))};
+  *reinterpret_cast<uint2*>(dh) = *reinterpret_cast<uint2*>(hh);
+  *reinterpret_cast<uint2*>(dl) = *reinterpret_cast<uint2*>(ll);
+}
+
 // One block of up to 128 columns.  GM: group - 1 for in-block groups of 16
 // to 128 columns (group starts known at compile time), -2 for in-block
 // groups of 1 to 8 columns (tested per column), -1 when the block's grid was
 // computed beforehand (one group per row, or groups wider than a block).
-//
-// Besides its strided registers, every lane of a row holds a window of the
-// row's next two columns c and c + 1, so all eight lanes evaluate the
-// quantizer of column c on the same value and get the same error without a
-// cross-lane step in the column chain.  After column c the window's column
-// c + 1 takes its update, and the owner of column c + 2 (whose register now
-// has every update up to column c) hands its value to the row's lanes with
-// one shuffle, which is needed only after column c + 1's quantizer.  The
-// window and the owner's register receive the same updates in the same
-// order, so they hold the same value.
+// With groups of 32 columns or more the grid is fixed within a round: the
+// owner keeps the rounded quotient and the error and the outputs are formed
+// when the round retires; otherwise the owner keeps deq and the code.
 template <bool ORD, int GM>
 __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a) {
+  constexpr bool PERCOL = (GM == 15 || GM == -2);
   const SweepDesc& d = a.d;
   extern __shared__ __align__(16) float smem[];
   float* Up = smem;
@@ -170,17 +194,19 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
   const int q = lane & (LPR - 1);
   const int64_t n = d.n, j0 = a.j0;
   const int bw = a.bw;
-  const int64_t r = (int64_t)blockIdx.x * ROWS_PER_CTA + (tid >> 3);
-  const bool live = r < d.m;
+  const int64_t r0 = (int64_t)blockIdx.x * ROWS_PER_CTA + (tid >> 4) * 2;   // rows r0, r0 + 1
+  const bool live[2] = {r0 < d.m, r0 + 1 < d.m};
   const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(d.U) & 15) == 0);
+  const int64_t j1 = j0 + bw;
 
   // Issue every load of the block's inputs first: the U block (16-byte
   // loads when rows are aligned; bw is then a multiple of 4, so a load never
-  // passes the block's last column), U's diagonal and the row's columns q,
-  // q + 8, ... (zero past bw, for dead columns and for rows past m).
-  float4 ub[(BW * BW / 4) / (WARPS * 32)];
+  // passes the block's last column), U's diagonal, the rows' columns q,
+  // q + 16, ... (zero past bw and for rows past m), and the row of U whose
+  // bf16 split this CTA writes.
+  float4 ub[UB_PER_THREAD];
 #pragma unroll
-  for (int it = 0; it < (BW * BW / 4) / (WARPS * 32); ++it) {
+  for (int it = 0; it < UB_PER_THREAD; ++it) {
     const int idx = it * (WARPS * 32) + tid;
     const int k = idx >> 5, c = (idx & 31) * 4;
     ub[it] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -197,81 +223,97 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
     }
   }
   const float udiag = (tid < bw) ? d.U[(j0 + tid) * n + j0 + tid] : 1.f;
-  float2 v2[NREG / 2];
-  const float* wrow = d.W + r * n + j0;
+  float2 v[2][NP];
 #pragma unroll
-  for (int i = 0; i < NREG / 2; ++i) {
-    const int c0 = 16 * i + q, c1 = c0 + 8;
-    v2[i] = make_float2((live && c0 < bw) ? wrow[c0] : 0.f, (live && c1 < bw) ? wrow[c1] : 0.f);
+  for (int h = 0; h < 2; ++h) {
+    const float* wrow = d.W + (r0 + h) * n + j0;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const int c0 = 32 * p + q, c1 = c0 + 16;
+      v[h][p] = make_float2((live[h] && c0 < bw) ? wrow[c0] : 0.f, (live[h] && c1 < bw) ? wrow[c1] : 0.f);
+    }
+  }
+  // The tensor-core trailing update reads bf16 hi/lo copies of this block's
+  // rows of U, columns j1..; each CTA writes rows blockIdx.x, + gridDim.x, ...
+  // The first row's loads are issued here (up to 4096 - 128 columns).
+  const bool split = !ORD && j1 < n;
+  const bool split_fast = split && vec && (int)gridDim.x >= bw && (int)blockIdx.x < bw &&
+                          (n - j1) <= 4 * 4 * WARPS * 32;
+  float4 sv[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t c = j1 + 4 * tid + (int64_t)i * 4 * WARPS * 32;
+    sv[i] = (split_fast && c < n) ? *reinterpret_cast<const float4*>(d.U + (j0 + blockIdx.x) * n + c)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   if (d.info && *d.info != 0) return;
   if (d.dead) {
 #pragma unroll
-    for (int i = 0; i < NREG / 2; ++i) {
-      const int c0 = 16 * i + q, c1 = c0 + 8;
-      if (c0 < bw && d.dead[j0 + c0]) v2[i].x = 0.f;
-      if (c1 < bw && d.dead[j0 + c1]) v2[i].y = 0.f;
+    for (int p = 0; p < NP; ++p) {
+      const int c0 = 32 * p + q, c1 = c0 + 16;
+      const bool z0 = c0 < bw && d.dead[j0 + c0], z1 = c1 < bw && d.dead[j0 + c1];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (z0) v[h][p].x = 0.f;
+        if (z1) v[h][p].y = 0.f;
+      }
     }
   }
 
   // U block into the permuted layout (strictly upper part), zero pads, and
   // the correctly rounded reciprocals of the diagonal (0 past bw).
 #pragma unroll
-  for (int it = 0; it < (BW * BW / 4) / (WARPS * 32); ++it) {
+  for (int it = 0; it < UB_PER_THREAD; ++it) {
     const int idx = it * (WARPS * 32) + tid;
     const int k = idx >> 5, c = (idx & 31) * 4;
     const float x[4] = {ub[it].x, ub[it].y, ub[it].z, ub[it].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int cc = c + i;
-      Up[(k * LPR + (cc & 7)) * UP_LD + (cc >> 3)] = (cc > k && cc < bw) ? x[i] : 0.f;
+      Up[(k * LPR + (cc & (LPR - 1))) * UP_LD + (cc >> 4)] = (cc > k && cc < bw) ? x[i] : 0.f;
     }
   }
   for (int t = tid; t < BW * LPR * 3; t += WARPS * 32) {
     const int row = t / 3, p = t - 3 * (t / 3);
-    *reinterpret_cast<float4*>(Up + row * UP_LD + NREG + 4 * p) = make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float2*>(Up + row * UP_LD + NREG + 2 * p) = make_float2(0.f, 0.f);
   }
   if (tid < BW) iu[tid] = (tid < bw) ? __frcp_rn(udiag) : 0.f;
 
-  // bf16 hi/lo copy of this block's rows of U, columns j1.. (operand B of
-  // the tensor-core trailing update); rows are spread over the CTAs.
-  const int64_t j1 = j0 + bw;
-  if (!ORD && j1 < n) {
+  if (split_fast) {
+    const int64_t k = blockIdx.x;
+    __nv_bfloat16* dh = d.Uh + ((int64_t)a.slot * BW + k) * d.ldu;
+    __nv_bfloat16* dl = d.Ul + ((int64_t)a.slot * BW + k) * d.ldu;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t c = j1 + 4 * tid + (int64_t)i * 4 * WARPS * 32;
+      if (c < n) split4(sv[i], dh + c, dl + c);
+    }
+  } else if (split) {
     for (int64_t k = blockIdx.x; k < bw; k += gridDim.x) {
       const float* src = d.U + (j0 + k) * n;
       __nv_bfloat16* dh = d.Uh + ((int64_t)a.slot * BW + k) * d.ldu;
       __nv_bfloat16* dl = d.Ul + ((int64_t)a.slot * BW + k) * d.ldu;
       if (vec) {
-#pragma unroll 4
-        for (int64_t c = j1 + 4 * tid; c < n; c += 4 * blockDim.x) {
-          const float4 x = *reinterpret_cast<const float4*>(src + c);
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(x.x), h1 = __float2bfloat16_rn(x.y);
-          const __nv_bfloat16 h2 = __float2bfloat16_rn(x.z), h3 = __float2bfloat16_rn(x.w);
-          __nv_bfloat162 hh[2] = {__halves2bfloat162(h0, h1), __halves2bfloat162(h2, h3)};
-          __nv_bfloat162 ll[2] = {
-              __halves2bfloat162(__float2bfloat16_rn(x.x - __bfloat162float(h0)),
-                                 __float2bfloat16_rn(x.y - __bfloat162float(h1))),
-              __halves2bfloat162(__float2bfloat16_rn(x.z - __bfloat162float(h2)),
-                                 __float2bfloat16_rn(x.w - __bfloat162float(h3)))};
-          *reinterpret_cast<uint2*>(dh + c) = *reinterpret_cast<uint2*>(hh);
-          *reinterpret_cast<uint2*>(dl + c) = *reinterpret_cast<uint2*>(ll);
-        }
+        for (int64_t c = j1 + 4 * tid; c < n; c += 4 * blockDim.x)
+          split4(*reinterpret_cast<const float4*>(src + c), dh + c, dl + c);
       } else {
         for (int64_t c = j1 + tid; c < n; c += blockDim.x) {
           const float x = src[c];
-          const __nv_bfloat16 h = __float2bfloat16_rn(x);
-          dh[c] = h;
-          dl[c] = __float2bfloat16_rn(x - __bfloat162float(h));
+          const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+          dh[c] = hb;
+          dl[c] = __float2bfloat16_rn(x - __bfloat162float(hb));
         }
       }
     }
   }
 
   const float maxq = (float)((1 << d.bits) - 1);
-  Grid g = make_grid(1.f, 0.f, maxq);
-  if (GM == -1 && live) {
+  Grid g[2] = {make_grid(1.f, 0.f, maxq), make_grid(1.f, 0.f, maxq)};
+  if (GM == -1) {
     const int64_t gi = (d.group == -1) ? 0 : j0 / d.group;
-    g = make_grid(d.scales[r * d.ngroups + gi], d.zeros[r * d.ngroups + gi], maxq);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (live[h]) g[h] = make_grid(d.scales[(r0 + h) * d.ngroups + gi], d.zeros[(r0 + h) * d.ngroups + gi], maxq);
   }
   int gshift = 0;
   while (GM != -1 && (1 << gshift) < d.group) ++gshift;
@@ -280,85 +322,111 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
   __syncthreads();
 
   const int src_base = lane & ~(LPR - 1);
-  const int64_t wbase = r * n + j0;
-  // the window: columns 0 and 1 (register 0 of lanes 0 and 1)
-  float win[2];
-  win[0] = __shfl_sync(0xffffffffu, v2[0].x, src_base + 0);
-  win[1] = __shfl_sync(0xffffffffu, v2[0].x, src_base + 1);
+  // the windows: columns 0 and 1 (register 0 of lanes 0 and 1)
+  float win[2][2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    win[h][0] = __shfl_sync(0xffffffffu, v[h][0].x, src_base + 0);
+    win[h][1] = __shfl_sync(0xffffffffu, v[h][0].x, src_base + 1);
+  }
 #pragma unroll 1
   for (int R = 0; R < NROUND; ++R) {
-    const float* up = Up + (RC * R) * UP_ROW + q * UP_LD + 4 * R;
-    const float* upw = Up + (RC * R) * UP_ROW + 4 * R;
+    const float* up = Up + (RC * R) * UP_ROW + q * UP_LD + 2 * R;
+    const float* upw = Up + (RC * R) * UP_ROW + 2 * R;
     const float* iur = iu + RC * R;
-    float e4[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t code4 = 0;
+    float ke[2][RET];      // the owner's -e of its retired columns
+    uint32_t code2[2] = {0u, 0u};
 #pragma unroll
     for (int t = 0; t < RC; ++t) {
-      const int kt = t >> 3, o = t & 7;
+      const int kt = t >> 4, o = t & (LPR - 1);
       bool gs = false;
       if (GM >= 0) {
         gs = (t & (GM & (RC - 1))) == 0 && ((RC * R) & GM) == 0 && RC * R + t < bw;
       } else if (GM == -2) {
         gs = ((RC * R + t) & gmask) == 0 && RC * R + t < bw;
       }
-      if (gs) g = group_start(v2, RC * R + t, R, q, bw, d, live, r, g0 + ((RC * R + t) >> gshift), maxq);
-      // the quantizer of column c on the window (the same value in every
-      // lane of the row)
-      const float w = win[t & 1];
-      const float rr = fminf(fmaxf(rint_grid(__fmul_rn(w, g.isc)), g.lo), g.hi);
-      const float deq = __fmul_rn(g.sc, rr);
-      const float ne = ORD ? __fmul_rn(__fsub_rn(deq, w), iur[t])       // -e, exactly
-                           : __fmul_rn(fmaf(g.sc, rr, -w), iur[t]);
-      // column c + 1 in the window: U[c][c + 1]
-      const float uw = upw[t * UP_ROW + ((t + 1) & 7) * UP_LD + ((t + 1) >> 3)];
-      win[(t + 1) & 1] = ORD ? __fadd_rn(win[(t + 1) & 1], __fmul_rn(ne, uw)) : fmaf(ne, uw, win[(t + 1) & 1]);
-      // the owner lane keeps the result of its column
-      if (q == o) {
-        if (kt & 1) v2[kt >> 1].y = deq;
-        else v2[kt >> 1].x = deq;
-        e4[kt] = -ne;
-        code4 |= (__float_as_uint(__fadd_rn(rr, g.zp2)) & 0xFFu) << (8 * kt);
-      }
-      // later columns in the strided registers: from register kt on (U is
-      // zero on and below the diagonal, so earlier columns in the same pair
-      // are left unchanged)
-      const float2 ne2 = make_float2(ne, ne);
-      const float4* u4 = reinterpret_cast<const float4*>(up + t * UP_ROW);
+      if (gs) {
 #pragma unroll
-      for (int i = 0; i < NREG / 4; ++i) {
-        const float4 u = u4[i];
-        if (2 * i >= (kt >> 1)) upd2<ORD>(v2[2 * i], ne2, make_float2(u.x, u.y));
-        upd2<ORD>(v2[2 * i + 1], ne2, make_float2(u.z, u.w));
+        for (int h = 0; h < 2; ++h)
+          g[h] = group_start(v[h], RC * R + t, R, q, bw, d, live[h], r0 + h, g0 + ((RC * R + t) >> gshift), maxq);
+      }
+      const float ivu = iur[t];
+      const float uw = upw[t * UP_ROW + ((t + 1) & (LPR - 1)) * UP_LD + ((t + 1) >> 4)];
+      float ne[2], rr[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // the quantizer of column c on the window (the same value in the
+        // sixteen lanes of the row)
+        const float w = win[h][t & 1];
+        rr[h] = fminf(fmaxf(rint_grid(__fmul_rn(w, g[h].isc)), g[h].lo), g[h].hi);
+        ne[h] = ORD ? __fmul_rn(__fsub_rn(__fmul_rn(g[h].sc, rr[h]), w), ivu)   // -e, exactly
+                    : __fmul_rn(fmaf(g[h].sc, rr[h], -w), ivu);
+        // column c + 1 in the window: U[c][c + 1]
+        win[h][(t + 1) & 1] = upd1<ORD>(win[h][(t + 1) & 1], ne[h], uw);
+      }
+      // the owner lane keeps its column's result
+      if (q == o) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          ke[h][kt] = ne[h];
+          if (PERCOL) {
+            const float deq = __fmul_rn(g[h].sc, rr[h]);
+            if (kt) v[h][0].y = deq;
+            else v[h][0].x = deq;
+            code2[h] |= (__float_as_uint(__fadd_rn(rr[h], g[h].zp2)) & 0xFFu) << (8 * kt);
+          } else {
+            if (kt) v[h][0].y = rr[h];
+            else v[h][0].x = rr[h];
+          }
+        }
+      }
+      // later columns in the registers: every pair (U is zero on and below
+      // the diagonal, so the retired and current columns stay unchanged)
+      const float2* u2 = reinterpret_cast<const float2*>(up + t * UP_ROW);
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const float2 u = u2[p];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) upd2<ORD>(v[h][p], make_float2(ne[h], ne[h]), u);
       }
       // column c + 2 (updated up to column c) from its owner into the slot
       // column c leaves
-      const int k2 = (t + 2) >> 3, o2 = (t + 2) & 7;
-      const float x2 = (k2 & 1) ? v2[k2 >> 1].y : v2[k2 >> 1].x;
-      win[t & 1] = __shfl_sync(0xffffffffu, x2, src_base + o2);
-    }
-    // retire registers 0..3: columns 32 R + 8 k + q
-    if (live) {
+      const int k2 = (t + 2) >> 4, o2 = (t + 2) & (LPR - 1);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int col = RC * R + 8 * k + q;
-        if (col < bw) {
-          const float x = (k & 1) ? v2[k >> 1].y : v2[k >> 1].x;
-          d.W[wbase + col] = x;
-          d.codes[wbase + col] = (uint8_t)((code4 >> (8 * k)) & 0xFFu);
-          if (a.Eb) a.Eb[r * a.lde + col] = e4[k];
-          if (!ORD) {
-            const __nv_bfloat16 h = __float2bfloat16_rn(e4[k]);
-            const int64_t eo = r * d.lde + (int64_t)a.slot * BW + col;
-            d.Eh[eo] = h;
-            d.El[eo] = __float2bfloat16_rn(e4[k] - __bfloat162float(h));
-          }
+      for (int h = 0; h < 2; ++h)
+        win[h][t & 1] = __shfl_sync(0xffffffffu, reg_of(v[h], k2), src_base + o2);
+    }
+    // retire registers 0 and 1: columns 32 R + q and 32 R + 16 + q
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (!live[h]) continue;
+      const int64_t r = r0 + h;
+#pragma unroll
+      for (int k = 0; k < RET; ++k) {
+        const int col = RC * R + LPR * k + q;
+        if (col >= bw) continue;
+        const float x = reg_of(v[h], k);
+        const float deq = PERCOL ? x : __fmul_rn(g[h].sc, x);
+        const uint32_t code = PERCOL ? ((code2[h] >> (8 * k)) & 0xFFu)
+                                     : (__float_as_uint(__fadd_rn(x, g[h].zp2)) & 0xFFu);
+        const float e = -ke[h][k];
+        d.W[r * n + j0 + col] = deq;
+        d.codes[r * n + j0 + col] = (uint8_t)code;
+        if (a.Eb) a.Eb[r * a.lde + col] = e;
+        if (!ORD) {
+          const __nv_bfloat16 hb = __float2bfloat16_rn(e);
+          const int64_t eo = r * d.lde + (int64_t)a.slot * BW + col;
+          d.Eh[eo] = hb;
+          d.El[eo] = __float2bfloat16_rn(e - __bfloat162float(hb));
         }
       }
     }
 #pragma unroll
-    for (int i = 0; i < NREG / 2 - 2; ++i) v2[i] = v2[i + 2];
-    v2[NREG / 2 - 2] = make_float2(0.f, 0.f);
-    v2[NREG / 2 - 1] = make_float2(0.f, 0.f);
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int p = 0; p < NP - 1; ++p) v[h][p] = v[h][p + 1];
+      v[h][NP - 1] = make_float2(0.f, 0.f);
+    }
   }
 }
 
