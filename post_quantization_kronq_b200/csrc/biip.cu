@@ -87,6 +87,34 @@ __device__ __forceinline__ void radix16_pass(float* cur, int RS, int logR) {
   __syncthreads();
 }
 
+// Loads of one group of R <= 8 rows for rows up to 8 x RP_THREADS long:
+// thread t takes columns t, t + RP_THREADS, ... of every row, all loads
+// issued before any is used.
+template <bool BF16>
+__device__ __forceinline__ void load_group(const RowPass& p, int L, int64_t r0, int rows_here,
+                                           float (&v)[8][8]) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const int64_t row = (r0 + rr) * p.ld_in + tid;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int j = tid + c * RP_THREADS;
+      v[c][rr] = 0.f;
+      if (j < L && rr < rows_here) {
+        if (BF16) v[c][rr] = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[row + c * RP_THREADS]);
+        else v[c][rr] = reinterpret_cast<const float*>(p.in)[row + c * RP_THREADS];
+      }
+    }
+  }
+}
+
+// Persistent: CTA b transforms the row groups b, b + gridDim.x, ... (R
+// rows each).  F4096 (rows of 4096 = 2^12, three radix-16 passes): the next
+// group's loads are issued into registers right after the current group
+// reaches shared memory, so they overlap its transform and its transposed
+// store.  Other lengths load each group when it starts.
+template <bool BF16, bool F4096>
 __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
   extern __shared__ __align__(16) float sm[];
   const RowPass& p = A.p;
@@ -95,9 +123,8 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
   float* buf0 = sm;
   float* buf1 = sm + R * RS;
   float* Cm = sm + R * RS * (A.two_buf ? 2 : 1);
-  const int64_t r0 = (int64_t)blockIdx.x * R;
-  const int rows_here = (int)((p.rows - r0) < R ? (p.rows - r0) : R);
   const int tid = threadIdx.x;
+  const int64_t ngroups = (p.rows + R - 1) / R;
 
   if (p.rotate && K > 1) {
     for (int t = tid; t < K * K; t += RP_THREADS) {
@@ -107,184 +134,197 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
     }
   }
 
-  // 1. load rows (forward: times sign and scale of the column); the column
-  //    factor is computed once per column and reused for the R rows.
-  //    Rows up to 8 x RP_THREADS long: all of a thread's loads (8 columns x
-  //    R rows) are issued before any is used, one memory latency per CTA.
-  if (L <= 8 * RP_THREADS) {
-    float v[8][8];
+  const bool reg_load = L <= 8 * RP_THREADS;
+  float v[8][8];
+  int64_t grp = blockIdx.x;
+  if (F4096 && grp < ngroups) {
+    const int64_t r0 = grp * R;
+    load_group<BF16>(p, L, r0, (int)((p.rows - r0) < R ? (p.rows - r0) : R), v);
+  }
+  for (; grp < ngroups; grp += gridDim.x) {
+    const int64_t r0 = grp * R;
+    const int rows_here = (int)((p.rows - r0) < R ? (p.rows - r0) : R);
+
+    // 1. rows into shared memory (forward: times sign and scale of the
+    //    column); the column factor is computed once per column and reused
+    //    for the R rows.
+    if (reg_load) {
+      if (!F4096) load_group<BF16>(p, L, r0, rows_here, v);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int j = tid + c * RP_THREADS;
+      for (int c = 0; c < 8; ++c) {
+        const int j = tid + c * RP_THREADS;
+        if (j < L) {
+          const float f = p.inverse ? 1.f : col_factor(p, j);
+          const int pj = padx(j);
+#pragma unroll
+          for (int rr = 0; rr < 8; ++rr)
+            if (rr < R) buf0[rr * RS + pj] = v[c][rr] * f;
+        }
+      }
+    } else for (int j = tid; j < L; j += RP_THREADS) {
+      const float f = p.inverse ? 1.f : col_factor(p, j);
+      const int pj = padx(j);
+      float w[8];
 #pragma unroll
       for (int rr = 0; rr < 8; ++rr) {
-        v[c][rr] = 0.f;
-        if (j < L && rr < rows_here) {
+        w[rr] = 0.f;
+        if (rr < rows_here) {
           const int64_t idx = (r0 + rr) * p.ld_in + j;
-          v[c][rr] = p.in_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[idx])
-                               : reinterpret_cast<const float*>(p.in)[idx];
+          w[rr] = BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[idx])
+                       : reinterpret_cast<const float*>(p.in)[idx];
         }
       }
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr)
+        if (rr < R) buf0[rr * RS + pj] = w[rr] * f;
     }
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int j = tid + c * RP_THREADS;
-      if (j < L) {
-        const float f = p.inverse ? 1.f : col_factor(p, j);
-        const int pj = padx(j);
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr)
-          if (rr < R) buf0[rr * RS + pj] = v[c][rr] * f;
-      }
+    __syncthreads();
+    // the next group's loads, in flight during this group's transform
+    const int64_t nxt = grp + gridDim.x;
+    if (F4096 && nxt < ngroups) {
+      const int64_t n0 = nxt * R;
+      load_group<BF16>(p, L, n0, (int)((p.rows - n0) < R ? (p.rows - n0) : R), v);
     }
-  } else for (int j = tid; j < L; j += RP_THREADS) {
-    const float f = p.inverse ? 1.f : col_factor(p, j);
-    const int pj = padx(j);
-    float v[8];
-#pragma unroll
-    for (int rr = 0; rr < 8; ++rr) {
-      v[rr] = 0.f;
-      if (rr < rows_here) {
-        const int64_t idx = (r0 + rr) * p.ld_in + j;
-        v[rr] = p.in_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[idx])
-                          : reinterpret_cast<const float*>(p.in)[idx];
-      }
-    }
-#pragma unroll
-    for (int rr = 0; rr < 8; ++rr)
-      if (rr < R) buf0[rr * RS + pj] = v[rr] * f;
-  }
-  __syncthreads();
 
-  float* cur = buf0;
-  if (p.rotate) {
-    // 2. DCT along b (odd factor)
-    if (K > 1) {
-      const int items = R * P;
-      for (int t = tid; t < items; t += RP_THREADS) {
-        const int rr = t / P;
-        const int a = t - rr * P;
-        float* row = buf0 + rr * RS;
-        const int base = a * K;
-        if (!A.two_buf) {
-          float y[KREG];
+    float* cur = buf0;
+    if (F4096) {
+      // length 4096: three radix-16 passes with compile-time offsets
+      if (p.rotate) {
+        radix16_pass<0>(cur, RS, A.logR);
+        radix16_pass<4>(cur, RS, A.logR);
+        radix16_pass<8>(cur, RS, A.logR);
+      }
+    } else if (p.rotate) {
+      // 2. DCT along b (odd factor)
+      if (K > 1) {
+        const int items = R * P;
+        for (int t = tid; t < items; t += RP_THREADS) {
+          const int rr = t / P;
+          const int a = t - rr * P;
+          float* row = buf0 + rr * RS;
+          const int base = a * K;
+          if (!A.two_buf) {
+            float y[KREG];
 #pragma unroll
-          for (int b = 0; b < KREG; ++b) y[b] = (b < K) ? row[padx(base + b)] : 0.f;
+            for (int b = 0; b < KREG; ++b) y[b] = (b < K) ? row[padx(base + b)] : 0.f;
 #pragma unroll
-          for (int o = 0; o < KREG; ++o) {
-            if (o < K) {
+            for (int o = 0; o < KREG; ++o) {
+              if (o < K) {
+                float acc = 0.f;
+#pragma unroll
+                for (int b = 0; b < KREG; ++b)
+                  if (b < K) acc = fmaf(p.inverse ? Cm[b * K + o] : Cm[o * K + b], y[b], acc);
+                row[padx(base + o)] = acc;
+              }
+            }
+          } else {
+            float* orow = buf1 + rr * RS;
+            for (int o = 0; o < K; ++o) {
               float acc = 0.f;
-#pragma unroll
-              for (int b = 0; b < KREG; ++b)
-                if (b < K) acc = fmaf(p.inverse ? Cm[b * K + o] : Cm[o * K + b], y[b], acc);
-              row[padx(base + o)] = acc;
+              for (int b = 0; b < K; ++b)
+                acc = fmaf(p.inverse ? Cm[b * K + o] : Cm[o * K + b], row[padx(base + b)], acc);
+              orow[padx(base + o)] = acc;
             }
           }
-        } else {
-          float* orow = buf1 + rr * RS;
-          for (int o = 0; o < K; ++o) {
-            float acc = 0.f;
-            for (int b = 0; b < K; ++b)
-              acc = fmaf(p.inverse ? Cm[b * K + o] : Cm[o * K + b], row[padx(base + b)], acc);
-            orow[padx(base + o)] = acc;
-          }
         }
+        if (A.two_buf) cur = buf1;
+        __syncthreads();
       }
-      if (A.two_buf) cur = buf1;
-      __syncthreads();
-    }
-    // 3. FWHT along a: radix-16 register passes over 4-bit groups of a.
-    //    Item order (b fastest, then the low bits of a, then the high bits)
-    //    keeps neighbouring threads on neighbouring shared-memory words.
-    if (K == 1 && A.logP == 12) {
-      // length 4096: three radix-16 passes with compile-time offsets
-      radix16_pass<0>(cur, RS, A.logR);
-      radix16_pass<4>(cur, RS, A.logR);
-      radix16_pass<8>(cur, RS, A.logR);
-    } else for (int lo = 0; lo < A.logP; lo += 4) {
-      const int nb = (A.logP - lo) < 4 ? (A.logP - lo) : 4;
-      const int G = 1 << nb;
-      const int per_row = L >> nb;
-      const int items = per_row << A.logR;
-      const int lo_mask = (1 << lo) - 1;
-      if (K == 1 && G == 16) {
-        // power-of-two length, full radix-16 pass: shifts and masks only
-        int lpr = 0;
-        while ((1 << lpr) < per_row) ++lpr;
+      // 3. FWHT along a: radix-16 register passes over 4-bit groups of a.
+      //    Item order (b fastest, then the low bits of a, then the high bits)
+      //    keeps neighbouring threads on neighbouring shared-memory words.
+      if (K == 1 && A.logP == 12) {
+        // length 4096: three radix-16 passes with compile-time offsets
+        radix16_pass<0>(cur, RS, A.logR);
+        radix16_pass<4>(cur, RS, A.logR);
+        radix16_pass<8>(cur, RS, A.logR);
+      } else for (int lo = 0; lo < A.logP; lo += 4) {
+        const int nb = (A.logP - lo) < 4 ? (A.logP - lo) : 4;
+        const int G = 1 << nb;
+        const int per_row = L >> nb;
+        const int items = per_row << A.logR;
+        const int lo_mask = (1 << lo) - 1;
+        if (K == 1 && G == 16) {
+          // power-of-two length, full radix-16 pass: shifts and masks only
+          int lpr = 0;
+          while ((1 << lpr) < per_row) ++lpr;
+          for (int t = tid; t < items; t += RP_THREADS) {
+            const int rr = t >> lpr;
+            const int rem = t & (per_row - 1);
+            const int a0 = ((rem >> lo) << (lo + 4)) | (rem & lo_mask);
+            float* row = cur + rr * RS;
+            float x[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) x[u] = row[padx(a0 + (u << lo))];
+#pragma unroll
+            for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+              for (int u = 0; u < 16; ++u)
+                if ((u & h) == 0) {
+                  const float s0 = x[u], s1 = x[u | h];
+                  x[u] = s0 + s1;
+                  x[u | h] = s0 - s1;
+                }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) row[padx(a0 + (u << lo))] = x[u];
+          }
+          __syncthreads();
+          continue;
+        }
         for (int t = tid; t < items; t += RP_THREADS) {
-          const int rr = t >> lpr;
-          const int rem = t & (per_row - 1);
-          const int a0 = ((rem >> lo) << (lo + 4)) | (rem & lo_mask);
+          const int rr = t / per_row;
+          int rem = t - rr * per_row;
+          int b = 0;
+          if (K > 1) {
+            const int q = rem / K;
+            b = rem - q * K;
+            rem = q;
+          }
+          const int a0 = ((rem >> lo) << (lo + nb)) | (rem & lo_mask);
           float* row = cur + rr * RS;
           float x[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) x[u] = row[padx(a0 + (u << lo))];
+          for (int u = 0; u < 16; ++u)
+            if (u < G) x[u] = row[padx((a0 + (u << lo)) * K + b)];
 #pragma unroll
-          for (int h = 1; h < 16; h <<= 1)
+          for (int h = 1; h < 16; h <<= 1) {
+            if (h < G) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-              if ((u & h) == 0) {
-                const float s0 = x[u], s1 = x[u | h];
-                x[u] = s0 + s1;
-                x[u | h] = s0 - s1;
-              }
-#pragma unroll
-          for (int u = 0; u < 16; ++u) row[padx(a0 + (u << lo))] = x[u];
-        }
-        __syncthreads();
-        continue;
-      }
-      for (int t = tid; t < items; t += RP_THREADS) {
-        const int rr = t / per_row;
-        int rem = t - rr * per_row;
-        int b = 0;
-        if (K > 1) {
-          const int q = rem / K;
-          b = rem - q * K;
-          rem = q;
-        }
-        const int a0 = ((rem >> lo) << (lo + nb)) | (rem & lo_mask);
-        float* row = cur + rr * RS;
-        float x[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (u < G) x[u] = row[padx((a0 + (u << lo)) * K + b)];
-#pragma unroll
-        for (int h = 1; h < 16; h <<= 1) {
-          if (h < G) {
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              if (u < G && (u & h) == 0) {
-                const float s0 = x[u], s1 = x[u | h];
-                x[u] = s0 + s1;
-                x[u | h] = s0 - s1;
+              for (int u = 0; u < 16; ++u) {
+                if (u < G && (u & h) == 0) {
+                  const float s0 = x[u], s1 = x[u | h];
+                  x[u] = s0 + s1;
+                  x[u | h] = s0 - s1;
+                }
               }
             }
           }
-        }
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (u < G) row[padx((a0 + (u << lo)) * K + b)] = x[u];
+          for (int u = 0; u < 16; ++u)
+            if (u < G) row[padx((a0 + (u << lo)) * K + b)] = x[u];
+        }
+        __syncthreads();
       }
-      __syncthreads();
     }
-  }
 
-  // 4. transposed store: consecutive threads take consecutive rows of one
-  //    column, so every warp writes R-float runs of the output rows.
-  const float nrm = p.rotate ? A.norm : 1.f;
-  const int tot = L << A.logR;
-  const int rr = tid & (R - 1);
-  const int jstep = RP_THREADS >> A.logR;
-  if (rr < rows_here) {
-    float* o = p.out + (int64_t)(tid >> A.logR) * p.ld_out + r0 + rr;
-    const int64_t ostep = (int64_t)jstep * p.ld_out;
-    const float* src = cur + rr * RS;
-    for (int t = tid, j = tid >> A.logR; t < tot; t += RP_THREADS, j += jstep, o += ostep) {
-      float v = src[padx(j)] * nrm;
-      if (p.inverse) v = v * col_factor(p, j);
-      *o = v;
+    // 4. transposed store: consecutive threads take consecutive rows of one
+    //    column, so every warp writes R-float runs of the output rows.
+    const float nrm = p.rotate ? A.norm : 1.f;
+    const int tot = L << A.logR;
+    const int rr = tid & (R - 1);
+    const int jstep = RP_THREADS >> A.logR;
+    if (rr < rows_here) {
+      float* o = p.out + (int64_t)(tid >> A.logR) * p.ld_out + r0 + rr;
+      const int64_t ostep = (int64_t)jstep * p.ld_out;
+      const float* src = cur + rr * RS;
+      for (int t = tid, j = tid >> A.logR; t < tot; t += RP_THREADS, j += jstep, o += ostep) {
+        float x = src[padx(j)] * nrm;
+        if (p.inverse) x = x * col_factor(p, j);
+        *o = x;
+      }
     }
+    // shared memory is refilled by the next group
+    __syncthreads();
   }
 }
 
@@ -392,10 +432,24 @@ kronq_status rowpass(const RowPass& p, cudaStream_t s) {
   A.logR = 0;
   while ((1 << A.logR) < R) ++A.logR;
   const int64_t smem = R * bytes_per_row + cbytes;
-  cudaError_t e = allow_smem(reinterpret_cast<const void*>(&rowpass_kernel), (int)smem);
+  const bool f4096 = (p.L == 4096 && K == 1);
+  const void* fn = f4096 ? (p.in_bf16 ? reinterpret_cast<const void*>(&rowpass_kernel<true, true>)
+                                      : reinterpret_cast<const void*>(&rowpass_kernel<false, true>))
+                         : (p.in_bf16 ? reinterpret_cast<const void*>(&rowpass_kernel<true, false>)
+                                      : reinterpret_cast<const void*>(&rowpass_kernel<false, false>));
+  cudaError_t e = allow_smem(fn, (int)smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rowpass)");
-  const int64_t grid = ceil_div(p.rows, R);
-  rowpass_kernel<<<(unsigned)grid, RP_THREADS, (size_t)smem, s>>>(A);
+  // one CTA per SM (the row buffers take most of shared memory), each
+  // looping over row groups
+  const int64_t groups = ceil_div(p.rows, R);
+  const int64_t grid = groups < (int64_t)sm_count() ? groups : (int64_t)sm_count();
+  if (f4096) {
+    if (p.in_bf16) rowpass_kernel<true, true><<<(unsigned)grid, RP_THREADS, (size_t)smem, s>>>(A);
+    else rowpass_kernel<false, true><<<(unsigned)grid, RP_THREADS, (size_t)smem, s>>>(A);
+  } else {
+    if (p.in_bf16) rowpass_kernel<true, false><<<(unsigned)grid, RP_THREADS, (size_t)smem, s>>>(A);
+    else rowpass_kernel<false, false><<<(unsigned)grid, RP_THREADS, (size_t)smem, s>>>(A);
+  }
   KQ_LAUNCH_CHECK("rowpass_kernel");
   return KRONQ_OK;
 }
