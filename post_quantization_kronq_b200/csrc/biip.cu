@@ -61,7 +61,13 @@ __device__ __forceinline__ void radix16_pass(float* cur, int RS, int logR) {
   for (int t = threadIdx.x; t < items; t += RP_THREADS) {
     const int rr = t >> 8;
     const int rem = t & (PER_ROW - 1);
-    const int a0 = ((rem >> LO) << (LO + 4)) | (rem & ((1 << LO) - 1));
+    int hi = rem >> LO;
+    if (LO == 4) {
+      // the two 16-item halves of a warp take groups two apart (bank offset
+      // 16 instead of 8), so the warp's loads and stores hit 32 distinct banks
+      hi = (hi & ~3) | ((hi & 1) << 1) | ((hi >> 1) & 1);
+    }
+    const int a0 = (hi << (LO + 4)) | (rem & ((1 << LO) - 1));
     float* base = cur + rr * RS + padx(a0);
     float x[16];
 #pragma unroll
@@ -123,8 +129,14 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
   float* buf0 = sm;
   float* buf1 = sm + R * RS;
   float* Cm = sm + R * RS * (A.two_buf ? 2 : 1);
+  float* cfs = Cm + ((p.rotate && K > 1) ? K * K : 0);   // F4096: column factors
   const int tid = threadIdx.x;
   const int64_t ngroups = (p.rows + R - 1) / R;
+  if (F4096) {
+    // every group uses the same column factors: computed once per CTA
+    for (int j = tid; j < L; j += RP_THREADS) cfs[j] = col_factor(p, j);
+    __syncthreads();
+  }
 
   if (p.rotate && K > 1) {
     for (int t = tid; t < K * K; t += RP_THREADS) {
@@ -154,7 +166,7 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
       for (int c = 0; c < 8; ++c) {
         const int j = tid + c * RP_THREADS;
         if (j < L) {
-          const float f = p.inverse ? 1.f : col_factor(p, j);
+          const float f = p.inverse ? 1.f : (F4096 ? cfs[j] : col_factor(p, j));
           const int pj = padx(j);
 #pragma unroll
           for (int rr = 0; rr < 8; ++rr)
@@ -319,7 +331,7 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
       const float* src = cur + rr * RS;
       for (int t = tid, j = tid >> A.logR; t < tot; t += RP_THREADS, j += jstep, o += ostep) {
         float x = src[padx(j)] * nrm;
-        if (p.inverse) x = x * col_factor(p, j);
+        if (p.inverse) x = x * (F4096 ? cfs[j] : col_factor(p, j));
         *o = x;
       }
     }
@@ -431,8 +443,8 @@ kronq_status rowpass(const RowPass& p, cudaStream_t s) {
   A.R = R;
   A.logR = 0;
   while ((1 << A.logR) < R) ++A.logR;
-  const int64_t smem = R * bytes_per_row + cbytes;
   const bool f4096 = (p.L == 4096 && K == 1);
+  const int64_t smem = R * bytes_per_row + cbytes + (f4096 ? p.L * 4 : 0);
   const void* fn = f4096 ? (p.in_bf16 ? reinterpret_cast<const void*>(&rowpass_kernel<true, true>)
                                       : reinterpret_cast<const void*>(&rowpass_kernel<false, true>))
                          : (p.in_bf16 ? reinterpret_cast<const void*>(&rowpass_kernel<true, false>)
