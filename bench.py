@@ -45,6 +45,7 @@ TOKENS = 131072
 # dram__bytes_read.sum / dram__bytes_write.sum of one syrk_bf16_tc_kernel launch
 # at T = 16384, d = 4096 (ncu, B200), used for roofline.traffic
 SYRK_READ_BYTES_T16384 = 225.659136e6
+E2E_CHUNK = 16384   # tokens per host->device copy chunk in the end-to-end pass
 SYRK_WRITE_BYTES_D4096 = 41.663232e6
 WORKLOAD = "llama2-7b q_proj 4096x4096, T=131072 tokens, W{bits} g{group} asym, BiIP full"
 
@@ -313,10 +314,9 @@ def run_kronq(args):
         d2h = sum(t.numel() * t.element_size() for t in houts)
 
         def e2e_step():
-            X.copy_(hX, non_blocking=True)
-            G.copy_(hG, non_blocking=True)
-            W.copy_(hW, non_blocking=True)
-            step()
+            # token chunks of X and G copied on a second stream while the
+            # factor accumulation of the earlier chunks runs
+            lp.run_from_host(hX, hG, hW, X, G, W, chunk=E2E_CHUNK, stream=stream)
             for h, o in zip(houts, outs):
                 h.copy_(o, non_blocking=True)
 
@@ -337,7 +337,9 @@ def run_kronq(args):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
         e2e = {"value": world * M * N_IN * e_steps / (e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+               "pipeline": f"X, G copied in {E2E_CHUNK}-token chunks on a second stream, "
+                           "overlapping the factor accumulation and the previous step's sweep"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -70,3 +70,55 @@ class LayerPass:
             self.sensitivity(stream=stream)
         self.transform(W, stream=stream)
         self.quantize(stream=stream)
+
+    def run_from_host(self, hX, hG, hW, X, G, W, chunk: int = 16384, with_sensitivity: bool = True,
+                      stream=None, copy_stream=None):
+        """One layer pass from pinned host inputs, copies overlapped with compute.
+
+        Token chunks of X and G (hX, hG: pinned host tensors) are copied into the
+        device buffers X and G on ``copy_stream`` while the factor accumulation
+        of the chunks already on the device runs on ``stream``; W's copy goes
+        last on the copy stream.  Across calls, the next call's copies of X and
+        G wait only for this call's last accumulation (and W's copy for this
+        call's BiIP forward), so they overlap this call's BiIP and sweep.  The
+        arithmetic is that of ``run(X, G, W, chunk)``: same launches, same order.
+        """
+        compute = torch.cuda.current_stream() if stream is None else stream
+        if copy_stream is None:
+            if getattr(self, "_copy_stream", None) is None:
+                self._copy_stream = torch.cuda.Stream(device=X.device)
+            copy_stream = self._copy_stream
+        T = X.shape[0]
+        prev_acc = getattr(self, "_ev_acc_done", None)
+        prev_w = getattr(self, "_ev_w_done", None)
+        if prev_acc is None:
+            copy_stream.wait_stream(compute)
+        else:
+            copy_stream.wait_event(prev_acc)
+        ready = []
+        with torch.cuda.stream(copy_stream):
+            for t0 in range(0, max(T, 1), chunk):
+                t1 = min(T, t0 + chunk)
+                X[t0:t1].copy_(hX[t0:t1], non_blocking=True)
+                G[t0:t1].copy_(hG[t0:t1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy_stream)
+                ready.append((t0, t1, ev))
+            if prev_w is not None:
+                copy_stream.wait_event(prev_w)
+            W.copy_(hW, non_blocking=True)
+            w_ready = torch.cuda.Event()
+            w_ready.record(copy_stream)
+        for t0, t1, ev in ready:
+            compute.wait_event(ev)
+            kronq_accumulate_factors(X[t0:t1], self.HX, zero_first=(t0 == 0), stream=compute)
+            kronq_accumulate_factors(G[t0:t1], self.HG, zero_first=(t0 == 0), stream=compute)
+        self._ev_acc_done = torch.cuda.Event()
+        self._ev_acc_done.record(compute)
+        if with_sensitivity:
+            self.sensitivity(stream=compute)
+        compute.wait_event(w_ready)
+        self.transform(W, stream=compute)
+        self._ev_w_done = torch.cuda.Event()
+        self._ev_w_done.record(compute)
+        self.quantize(stream=compute)
