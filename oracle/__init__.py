@@ -18,9 +18,11 @@ Modules
   alloc    -- O7: inter-layer bit allocation from tr(H_G) * tr(H_X).
   pack     -- int2/int4 code packing.
   pipeline -- the whole layer pass chained from the above.
+  estimators -- Kronecker factor estimators (input, marginal, Frobenius,
+              FlipFlop) of the "WaterKron and FlipFlop Hessian" page, Table 1.
 
 Every function is pinned by tests under ``tests/test_oracle_*.py`` against
 closed forms, invariants, library special cases, brute force or the values
 printed on the pages.  Parity is pinned for every function here.
 """
-from . import factors, biip, sweep, loss, alloc, pack, pipeline  # noqa: F401
+from . import factors, biip, sweep, loss, alloc, pack, pipeline, estimators  # noqa: F401
