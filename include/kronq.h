@@ -254,6 +254,45 @@ size_t kronq_kfac_loss_workspace_bytes(int64_t m, int64_t n);
 kronq_status kronq_kfac_loss(const float* E, const float* HG, int64_t m, int64_t n, double* out,
                              void* workspace, size_t ws_bytes, kronq_stream_t s);
 
+/* ---------------------------------------------------------------------------
+ * Kronecker factor estimators A (x) B ~ H = E[x x^T (x) g g^T]
+ * ("WaterKron and FlipFlop Hessian" page, Table 1 and its caption).
+ *
+ *   KRONQ_EST_INPUT      A = E[x x^T],               B = I
+ *   KRONQ_EST_MARGINAL   A = E[x x^T],               B = E[g g^T]
+ *   KRONQ_EST_FROBENIUS  A = E[(g^T B g) x x^T] / ||B||_F^2,
+ *                        B = E[(x^T A x) g g^T] / ||A||_F^2
+ *   KRONQ_EST_FLIPFLOP   A = E[(g^T B^-1 g) x x^T] / m,
+ *                        B = E[(x^T A^-1 x) g g^T] / n
+ * E is the mean over the T tokens.  Frobenius and FlipFlop start from
+ * B = I and run `iters` sweeps (A from B, then B from A); each update is the
+ * exact minimiser of the row's target over one factor (||H - A (x) B||_F;
+ * for FlipFlop the Gaussian fit tr((A (x) B)^-1 H) + log det(A (x) B)).
+ *
+ * X: T x n bf16, G: T x m bf16, device, row-major with row strides n and m;
+ * n and m multiples of 8 (16-byte rows for the tensor-core loads).  A (n x n)
+ * and B (m x m): fp32 device outputs, both triangles written.  info: device
+ * int, 0 on success, else the failing pivot + 1 of the Cholesky factor of a
+ * FlipFlop factor that is not positive definite (the remaining steps are
+ * skipped).  Per-token weights come from a tensor-core product of the tokens
+ * with a bf16 hi/lo split of the other factor (or of the Cholesky factor of
+ * its inverse), the weighted second moment from the tensor-core SYRK of the
+ * sqrt(weight)-scaled tokens rounded to bf16.  Workspace of
+ * kronq_kron_factors_workspace_bytes(T, n, m) bytes, 256-byte aligned.
+ * Asynchronous on s.
+ * ------------------------------------------------------------------------- */
+typedef enum {
+  KRONQ_EST_INPUT = 0,
+  KRONQ_EST_MARGINAL = 1,
+  KRONQ_EST_FROBENIUS = 2,
+  KRONQ_EST_FLIPFLOP = 3
+} kronq_estimator;
+
+size_t kronq_kron_factors_workspace_bytes(int64_t T, int64_t n, int64_t m);
+kronq_status kronq_kron_factors(const void* X, const void* G, int64_t T, int64_t n, int64_t m,
+                                kronq_estimator est, int iters, float* A, float* B, int* info,
+                                void* workspace, size_t ws_bytes, kronq_stream_t s);
+
 /* Number of kernels this library has launched in the process so far (all
  * devices and streams); a host counter, no synchronisation. */
 uint64_t kronq_launch_count(void);

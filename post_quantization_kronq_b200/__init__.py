@@ -21,7 +21,12 @@ __all__ = [
     "kronq_quantize_layer_static",
     "kronq_pack", "kronq_unpack", "kronq_device_status", "kronq_kfac_loss_workspace_bytes",
     "kronq_kfac_loss", "kronq_launch_count", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
+    "EST_INPUT", "EST_MARGINAL", "EST_FROBENIUS", "EST_FLIPFLOP",
+    "kronq_kron_factors_workspace_bytes", "kronq_kron_factors",
 ]
+
+# kronq_estimator (Table 1 rows of the "WaterKron and FlipFlop Hessian" page)
+EST_INPUT, EST_MARGINAL, EST_FROBENIUS, EST_FLIPFLOP = 0, 1, 2, 3
 
 
 def _ptr(t):
@@ -180,6 +185,25 @@ def kronq_device_status(stream=None) -> int:
     v = ctypes.c_int(0)
     check(lib.kronq_device_status(ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+def kronq_kron_factors_workspace_bytes(T: int, n: int, m: int) -> int:
+    return int(lib.kronq_kron_factors_workspace_bytes(T, n, m))
+
+
+def kronq_kron_factors(X, G, est: int, iters: int, A, B, info, ws=None, stream=None):
+    """Kronecker factors (A n x n, B m x m, fp32 out) of E[x x^T (x) g g^T]
+    from bf16 tokens X (T x n) and G (T x m); info (device int) 0 on success."""
+    import torch
+    T, n = X.shape
+    m = G.shape[1]
+    if X.dtype != torch.bfloat16 or G.dtype != torch.bfloat16:
+        raise ValueError("X and G must be bfloat16")
+    for t, name in ((X, "X"), (G, "G"), (A, "A"), (B, "B"), (info, "info")):
+        _rowmajor(t, name)
+    ws = workspace(kronq_kron_factors_workspace_bytes(T, n, m), X.device) if ws is None else ws
+    check(lib.kronq_kron_factors(_ptr(X), _ptr(G), T, n, m, int(est), int(iters), _ptr(A), _ptr(B),
+                                 _ptr(info), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def kronq_kfac_loss_workspace_bytes(m: int, n: int) -> int:

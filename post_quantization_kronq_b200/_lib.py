@@ -60,6 +60,9 @@ SIGNATURES = {
     "kronq_device_status": (_int, [_ip, _vp]),
     "kronq_kfac_loss_workspace_bytes": (_sz, [_i64, _i64]),
     "kronq_kfac_loss": (_int, [_vp, _vp, _i64, _i64, _dp, _vp, _sz, _vp]),
+    "kronq_kron_factors_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "kronq_kron_factors": (_int, [_vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _sz,
+                                  _vp]),
     "kronq_launch_count": (ctypes.c_uint64, []),
     "kronq_last_error": (ctypes.c_char_p, []),
     "kronq_version": (ctypes.c_char_p, []),

@@ -4,6 +4,7 @@
     python -m post_quantization_kronq_b200.opbench biip --m 4096 --n 4096
     python -m post_quantization_kronq_b200.opbench quantize --m 4096 --n 4096 --bits 2
     python -m post_quantization_kronq_b200.opbench pack --m 8192 --n 28672 --bits 2
+    python -m post_quantization_kronq_b200.opbench kronfactors --est flipflop --tokens 131072 --m 4096 --n 4096
 
 Meant for profiling a single kernel family (e.g. under ncu) at a size that
 is smaller than the full benchmark; prints one JSON line with the mean
@@ -29,7 +30,9 @@ def main(argv=None):
     from synth import llama_layer
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["accumulate", "biip", "quantize", "pack"])
+    ap.add_argument("op", choices=["accumulate", "biip", "quantize", "pack", "kronfactors"])
+    ap.add_argument("--est", choices=["input", "marginal", "frobenius", "flipflop"], default="flipflop")
+    ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--tokens", type=int, default=16384)
     ap.add_argument("--d", type=int, default=4096)
     ap.add_argument("--m", type=int, default=4096)
@@ -45,6 +48,19 @@ def main(argv=None):
         H = torch.empty(a.d, a.d, device=dev)
         run = lambda: kq.kronq_accumulate_factors(X, H, zero_first=True)  # noqa: E731
         units = {"flops": a.tokens * a.d * (a.d + 1)}
+    elif a.op == "kronfactors":
+        _, X, G = llama_layer(a.m, a.n, a.tokens, seed=1, device=dev)
+        A = torch.empty(a.n, a.n, device=dev)
+        B = torch.empty(a.m, a.m, device=dev)
+        info = torch.zeros(1, dtype=torch.int32, device=dev)
+        est = {"input": kq.EST_INPUT, "marginal": kq.EST_MARGINAL, "frobenius": kq.EST_FROBENIUS,
+               "flipflop": kq.EST_FLIPFLOP}[a.est]
+        ws = kq.workspace(kq.kronq_kron_factors_workspace_bytes(a.tokens, a.n, a.m), dev)
+        run = lambda: kq.kronq_kron_factors(X, G, est, a.iters, A, B, info, ws=ws)  # noqa: E731
+        # per sweep: two weight products (2 T m^2 and 2 T n^2 flop) and two
+        # SYRKs (T n (n+1) and T m (m+1))
+        units = {"flops_per_sweep": 2 * a.tokens * (a.m * a.m + a.n * a.n)
+                 + a.tokens * (a.n * (a.n + 1) + a.m * (a.m + 1))}
     else:
         W, X, G = llama_layer(a.m, a.n, 2 * max(a.m, a.n), seed=1, device=dev)
         lp = LayerPass(a.m, a.n, bits=a.bits, group=a.group, device=dev)
@@ -80,6 +96,9 @@ def main(argv=None):
     e1.record(s)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.reps
+    if a.op == "kronfactors":
+        units["info"] = int(info.item())
+        units["tflops"] = units["flops_per_sweep"] * a.iters / (ms / 1e3) / 1e12
     print(json.dumps({"op": a.op, "ms_per_call": ms, "args": vars(a), **units}))
     return 0
 

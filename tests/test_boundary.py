@@ -170,3 +170,24 @@ def test_shard_units_partition():
         for w in (1, 2, 3, 8):
             got = sum((shard_units(n, r, w) for r in range(w)), [])
             assert got == list(range(n))
+
+
+def test_kron_factors_validation():
+    L = _lib.lib
+    ws = L.kronq_kron_factors_workspace_bytes(1000, 128, 64)
+    assert ws > 0 and L.kronq_kron_factors_workspace_bytes(1000, 0, 64) == 0
+    ok = dict(T=1000, n=128, m=64, est=3, iters=2)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return _st(L.kronq_kron_factors(FAKE, FAKE, a["T"], a["n"], a["m"], a["est"], a["iters"], FAKE,
+                                        FAKE, FAKE, ctypes.c_void_p(4096 * 256),
+                                        kw.get("ws", ws), None))
+    assert call(est=4) == _lib.ERR_INVALID_ARG
+    assert call(n=60) == _lib.ERR_INVALID_ARG        # below 64
+    assert call(m=100) == _lib.ERR_INVALID_ARG       # not a multiple of 8
+    assert call(T=0) == _lib.ERR_INVALID_ARG
+    assert call(iters=-1) == _lib.ERR_INVALID_ARG
+    assert call(ws=ws - 1) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_kron_factors(None, FAKE, 1000, 128, 64, 3, 2, FAKE, FAKE, FAKE,
+                                    ctypes.c_void_p(4096 * 256), ws, None)) == _lib.ERR_INVALID_ARG
