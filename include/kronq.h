@@ -293,6 +293,24 @@ kronq_status kronq_kron_factors(const void* X, const void* G, int64_t T, int64_t
                                 kronq_estimator est, int iters, float* A, float* B, int* info,
                                 void* workspace, size_t ws_bytes, kronq_stream_t s);
 
+/* ---------------------------------------------------------------------------
+ * Deploy-path matvec from packed codes (KronQ README intro: packed int4/int2
+ * weights, a fused dequant + BiIP matvec for single-token decode):
+ *   y = D_o^-1 U^T Q V D_i^-1 x,  Q[i, j] = scales[i, g] (q[i, j] - zeros[i, g]),
+ * g = j / group (0 when group == -1), q from `packed` (m x ceil(n bits / 32)
+ * uint32 words, least significant bits first along n: kronq_pack's layout).
+ * U, V, d_in, d_out, seed and mode are those of kronq_biip_forward.
+ *   x: n activations, bf16 or float32 (xdt); y: m float32 out.  All device
+ *   memory.  bits 2 or 4.  Workspace of kronq_decode_matvec_workspace_bytes
+ *   bytes, 256-byte aligned.  Asynchronous on s.
+ * ------------------------------------------------------------------------- */
+size_t kronq_decode_matvec_workspace_bytes(int64_t m, int64_t n);
+kronq_status kronq_decode_matvec(const uint32_t* packed, const float* scales, const float* zeros,
+                                 int64_t m, int64_t n, int bits, int group, uint64_t seed,
+                                 kronq_biip_mode mode, const float* d_in, const float* d_out,
+                                 const void* x, kronq_dtype xdt, float* y, void* workspace,
+                                 size_t ws_bytes, kronq_stream_t s);
+
 /* Number of kernels this library has launched in the process so far (all
  * devices and streams); a host counter, no synchronisation. */
 uint64_t kronq_launch_count(void);

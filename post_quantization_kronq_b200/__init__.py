@@ -23,6 +23,7 @@ __all__ = [
     "kronq_kfac_loss", "kronq_launch_count", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
     "EST_INPUT", "EST_MARGINAL", "EST_FROBENIUS", "EST_FLIPFLOP",
     "kronq_kron_factors_workspace_bytes", "kronq_kron_factors",
+    "kronq_decode_matvec_workspace_bytes", "kronq_decode_matvec",
 ]
 
 # kronq_estimator (Table 1 rows of the "WaterKron and FlipFlop Hessian" page)
@@ -204,6 +205,23 @@ def kronq_kron_factors(X, G, est: int, iters: int, A, B, info, ws=None, stream=N
     ws = workspace(kronq_kron_factors_workspace_bytes(T, n, m), X.device) if ws is None else ws
     check(lib.kronq_kron_factors(_ptr(X), _ptr(G), T, n, m, int(est), int(iters), _ptr(A), _ptr(B),
                                  _ptr(info), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def kronq_decode_matvec_workspace_bytes(m: int, n: int) -> int:
+    return int(lib.kronq_decode_matvec_workspace_bytes(m, n))
+
+
+def kronq_decode_matvec(packed, scales, zeros, n: int, bits: int, group: int, seed: int, mode: str,
+                        d_in, d_out, x, y, ws=None, stream=None):
+    """y (m, float32) = D_o^-1 U^T Q V D_i^-1 x from packed codes (int32 words)."""
+    m = packed.shape[0]
+    for t, name in ((packed, "packed"), (scales, "scales"), (zeros, "zeros"), (d_in, "d_in"),
+                    (d_out, "d_out"), (x, "x"), (y, "y")):
+        _rowmajor(t, name)
+    ws = workspace(kronq_decode_matvec_workspace_bytes(m, n), x.device) if ws is None else ws
+    check(lib.kronq_decode_matvec(_ptr(packed), _ptr(scales), _ptr(zeros), m, n, bits, group, seed,
+                                  BIIP_MODES[mode], _ptr(d_in), _ptr(d_out), _ptr(x), _dtype_code(x),
+                                  _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def kronq_kfac_loss_workspace_bytes(m: int, n: int) -> int:

@@ -63,6 +63,9 @@ SIGNATURES = {
     "kronq_kron_factors_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "kronq_kron_factors": (_int, [_vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _sz,
                                   _vp]),
+    "kronq_decode_matvec_workspace_bytes": (_sz, [_i64, _i64]),
+    "kronq_decode_matvec": (_int, [_vp, _vp, _vp, _i64, _i64, _int, _int, _u64, _int, _vp, _vp, _vp,
+                                   _int, _vp, _vp, _sz, _vp]),
     "kronq_launch_count": (ctypes.c_uint64, []),
     "kronq_last_error": (ctypes.c_char_p, []),
     "kronq_version": (ctypes.c_char_p, []),

@@ -5,6 +5,7 @@
     python -m post_quantization_kronq_b200.opbench quantize --m 4096 --n 4096 --bits 2
     python -m post_quantization_kronq_b200.opbench pack --m 8192 --n 28672 --bits 2
     python -m post_quantization_kronq_b200.opbench kronfactors --est flipflop --tokens 131072 --m 4096 --n 4096
+    python -m post_quantization_kronq_b200.opbench decode --m 4096 --n 4096 --bits 2 --reps 100
 
 Meant for profiling a single kernel family (e.g. under ncu) at a size that
 is smaller than the full benchmark; prints one JSON line with the mean
@@ -30,7 +31,7 @@ def main(argv=None):
     from synth import llama_layer
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["accumulate", "biip", "quantize", "pack", "kronfactors"])
+    ap.add_argument("op", choices=["accumulate", "biip", "quantize", "pack", "kronfactors", "decode"])
     ap.add_argument("--est", choices=["input", "marginal", "frobenius", "flipflop"], default="flipflop")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--tokens", type=int, default=16384)
@@ -48,6 +49,21 @@ def main(argv=None):
         H = torch.empty(a.d, a.d, device=dev)
         run = lambda: kq.kronq_accumulate_factors(X, H, zero_first=True)  # noqa: E731
         units = {"flops": a.tokens * a.d * (a.d + 1)}
+    elif a.op == "decode":
+        ng = -(-a.n // a.group)
+        codes = torch.randint(0, 2 ** a.bits, (a.m, a.n), dtype=torch.uint8, device=dev)
+        packed = torch.empty(a.m, kq.words_per_row(a.n, a.bits), dtype=torch.int32, device=dev)
+        kq.kronq_pack(codes, a.bits, packed)
+        sc = torch.rand(a.m, ng, device=dev) * 0.05 + 0.005
+        zp = torch.randint(0, 2 ** a.bits, (a.m, ng), device=dev).float()
+        d_in = torch.ones(a.n, device=dev)
+        d_out = torch.ones(a.m, device=dev)
+        x = torch.randn(a.n, device=dev).to(torch.bfloat16)
+        y = torch.empty(a.m, device=dev)
+        ws = kq.workspace(kq.kronq_decode_matvec_workspace_bytes(a.m, a.n), dev)
+        run = lambda: kq.kronq_decode_matvec(packed, sc, zp, a.n, a.bits, a.group, 0, "full",  # noqa: E731
+                                             d_in, d_out, x, y, ws=ws)
+        units = {"bytes": packed.numel() * 4 + 2 * sc.numel() * 4 + a.n * 2 + a.m * 4}
     elif a.op == "kronfactors":
         _, X, G = llama_layer(a.m, a.n, a.tokens, seed=1, device=dev)
         A = torch.empty(a.n, a.n, device=dev)
@@ -96,6 +112,8 @@ def main(argv=None):
     e1.record(s)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.reps
+    if a.op == "decode":
+        units["gbs"] = units["bytes"] / (ms / 1e3) / 1e9
     if a.op == "kronfactors":
         units["info"] = int(info.item())
         units["tflops"] = units["flops_per_sweep"] * a.iters / (ms / 1e3) / 1e12

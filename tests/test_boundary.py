@@ -191,3 +191,21 @@ def test_kron_factors_validation():
     assert call(ws=ws - 1) == _lib.ERR_INVALID_ARG
     assert _st(L.kronq_kron_factors(None, FAKE, 1000, 128, 64, 3, 2, FAKE, FAKE, FAKE,
                                     ctypes.c_void_p(4096 * 256), ws, None)) == _lib.ERR_INVALID_ARG
+
+
+def test_decode_matvec_validation():
+    L = _lib.lib
+    ws = L.kronq_decode_matvec_workspace_bytes(64, 96)
+    assert ws > 0 and L.kronq_decode_matvec_workspace_bytes(0, 96) == 0
+    W = ctypes.c_void_p(4096 * 256)
+
+    def call(m=64, n=96, bits=4, group=32, mode=0, xdt=1, nbytes=ws, x=FAKE):
+        return _st(L.kronq_decode_matvec(FAKE, FAKE, FAKE, m, n, bits, group, 7, mode, FAKE, FAKE, x,
+                                         xdt, FAKE, W, nbytes, None))
+    assert call(bits=3) == _lib.ERR_INVALID_ARG
+    assert call(group=0) == _lib.ERR_INVALID_ARG
+    assert call(mode=4) == _lib.ERR_INVALID_ARG
+    assert call(xdt=9) == _lib.ERR_INVALID_ARG
+    assert call(nbytes=ws - 1) == _lib.ERR_INVALID_ARG
+    assert call(x=None) == _lib.ERR_INVALID_ARG
+    assert call(n=257 * 2) == _lib.ERR_UNSUPPORTED      # odd factor 257 of a rotated dimension
