@@ -57,6 +57,42 @@ def _peaks():
         return None
 
 
+def phase_rooflines(phases_ms, m: int, n: int, T: int, peaks):
+    """Each timed phase's algorithmic work over the measured peak of its bound.
+
+    accumulate_HX_HG  tensor: T n (n+1) + T m (m+1) flop (the distinct entries
+                      of the two SYRKs)
+    sensitivity       HBM: the two diagonals, 4 (n + m) bytes
+    biip_forward      HBM: 16 m n + 16 n^2 + 16 m^2 bytes (W's norms read
+                      2 m n; its two passes read 2 + 4 and write 4 + 4 bytes
+                      per element; each factor takes two fp32 passes in and out)
+    quantize_and_pack bound by its sequential chains (64 diagonal steps of
+                      the factorisation, n column steps of the sweep); shown
+                      against the tensor peak with 2 n^3 / 3 + m n^2 flop (the
+                      reverse Cholesky factor and its triangular inverse, and
+                      the error feedback of the sweep)
+    """
+    if peaks:
+        tpk, hpk, src = peaks["bf16_tflops_sustained"], peaks["hbm_gbs"], "measured"
+    else:
+        tpk, hpk, src = 1400.0, 6650.0, "fallback"
+    work = {
+        "accumulate_HX_HG": ("tensor", T * n * (n + 1) + T * m * (m + 1), "TFLOP/s", tpk, 1e12),
+        "sensitivity": ("hbm", 4 * (n + m), "GB/s", hpk, 1e9),
+        "biip_forward": ("hbm", 16 * m * n + 16 * n * n + 16 * m * m, "GB/s", hpk, 1e9),
+        "quantize_and_pack": ("latency (sequential chains)", 2 * n ** 3 / 3 + m * n * n, "TFLOP/s", tpk, 1e12),
+    }
+    out = {}
+    for name, ms in phases_ms.items():
+        if name not in work or ms <= 0:
+            continue
+        bound, units, unit, peak, scale = work[name]
+        achieved = units / (ms / 1e3) / scale
+        out[name] = {"bound": bound, "achieved": achieved, "unit": unit, "peak": peak,
+                     "frac": achieved / peak, "peak_source": src}
+    return out
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi sampling during the timed region (200 ms period)."""
@@ -363,6 +399,7 @@ def run_kronq(args):
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": launches,
         "phases_ms": {k: round(v, 4) for k, v in phases.items()},
+        "phase_roofline": phase_rooflines(phases, M, N_IN, TOKENS, peaks),
         "sensitivity": list(lp.sens) if lp.sens else None,
     }
     print(json.dumps(line), flush=True)
