@@ -21,9 +21,10 @@ Modules
   estimators -- Kronecker factor estimators (input, marginal, Frobenius,
               FlipFlop) of the "WaterKron and FlipFlop Hessian" page, Table 1.
   decode   -- the deploy path's dequant + BiIP matvec from packed codes.
+  options  -- recipe options named without a definition (act-order).
 
 Every function is pinned by tests under ``tests/test_oracle_*.py`` against
 closed forms, invariants, library special cases, brute force or the values
 printed on the pages.  Parity is pinned for every function here.
 """
-from . import factors, biip, sweep, loss, alloc, pack, pipeline, estimators, decode  # noqa: F401
+from . import factors, biip, sweep, loss, alloc, pack, pipeline, estimators, decode, options  # noqa: F401
