@@ -22,9 +22,10 @@ Modules
               FlipFlop) of the "WaterKron and FlipFlop Hessian" page, Table 1.
   decode   -- the deploy path's dequant + BiIP matvec from packed codes.
   options  -- recipe options named without a definition (act-order).
+  twosided -- two-sided adaptive rounding under H_X (x) H_G (BaKron abstract).
 
 Every function is pinned by tests under ``tests/test_oracle_*.py`` against
 closed forms, invariants, library special cases, brute force or the values
 printed on the pages.  Parity is pinned for every function here.
 """
-from . import factors, biip, sweep, loss, alloc, pack, pipeline, estimators, decode, options  # noqa: F401
+from . import factors, biip, sweep, loss, alloc, pack, pipeline, estimators, decode, options, twosided  # noqa: F401
