@@ -16,6 +16,13 @@
  *      and per-group scales at 2/3/4 bits           -> kronq_quantize_layer
  *   5. packed int4/int2 storage (KronQ README "Model zoo") -> kronq_pack
  *
+ * Around the pass:
+ *   - the Kronecker factor estimators of the "WaterKron and FlipFlop
+ *     Hessian" page, Table 1 (input, marginal, Frobenius, FlipFlop)
+ *                                                    -> kronq_kron_factors
+ *   - the deploy path's matvec from packed codes (KronQ README intro: fused
+ *     dequant + BiIP matvec for single-token decode) -> kronq_decode_matvec
+ *
  * Conventions (all calls):
  *   - Matrices are row-major.  W is m x n (out x in), X is T x n, G is T x m.
  *   - Every array argument is DEVICE memory owned by the caller, except where
