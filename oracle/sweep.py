@@ -113,6 +113,24 @@ def chol_upper_of_inverse(A):
     return L.T
 
 
+def chol_upper_of_inverse_f32(A):
+    """The same U computed in float32 by LAPACK: the Cholesky factor of the
+    index-reversed float32 matrix (A = R R^T with R upper, eliminating from
+    the last index), then the float32 triangular inverse U = R^-1.
+
+    Not a step of the method: it measures what a float32 factorisation of a
+    given factor can achieve (its error grows with the factor's condition
+    number), the floor against which the float32 GPU factorisation is held.
+    """
+    import scipy.linalg as sl
+
+    A32 = np.asarray(A, dtype=np.float32)
+    n = A32.shape[0]
+    L = sl.cholesky(np.ascontiguousarray(A32[::-1, ::-1]), lower=True, check_finite=False)
+    R = np.ascontiguousarray(L[::-1, ::-1])
+    return sl.solve_triangular(R, np.eye(n, dtype=np.float32), lower=False, check_finite=False)
+
+
 def reverse_chol_failure(A) -> int:
     """LAPACK-style info for a factorisation that eliminates from the last
     index down: 0 when A is positive definite, else 1 + the largest j whose

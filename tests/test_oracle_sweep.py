@@ -220,3 +220,27 @@ def test_symmetric_grid():
     s, z = sweep.grid_params(wg, 2, asym=True)
     assert np.allclose(s, [5.0 / 3, 0.5 / 3, 2.0 / 3])
     assert np.array_equal(z, [np.rint(3.0 / (5.0 / 3)), 0.0, np.rint(1.0 / (2.0 / 3))])
+
+
+def test_float32_factorisation_floor():
+    # the float32 LAPACK route gives the same upper factor as the float64
+    # definition to float32 accuracy on a well-conditioned matrix, and its
+    # error grows with the condition number
+    rng = np.random.default_rng(4)
+    n = 96
+    X = rng.standard_normal((4 * n, n))
+    A, _ = sweep.damp(X.T @ X, 0.01)
+    U = sweep.chol_upper_of_inverse(A)
+    U32 = sweep.chol_upper_of_inverse_f32(A)
+    assert U32.dtype == np.float32
+    assert np.array_equal(U32, np.triu(U32))
+    assert np.linalg.norm(U32 - U) / np.linalg.norm(U) < 1e-5
+    assert np.abs(U32.astype(np.float64).T @ U32.astype(np.float64) @ A - np.eye(n)).max() < 1e-4
+    # an ill-conditioned factor (a large common mean, as rectified inputs give)
+    Xr = np.abs(X) + 3.0
+    Ar, _ = sweep.damp(Xr.T @ Xr, 0.01)
+    Ur = sweep.chol_upper_of_inverse(Ar)
+    Ur32 = sweep.chol_upper_of_inverse_f32(Ar)
+    e_good = np.linalg.norm(U32 - U) / np.linalg.norm(U)
+    e_bad = np.linalg.norm(Ur32 - Ur) / np.linalg.norm(Ur)
+    assert e_bad > 3 * e_good
