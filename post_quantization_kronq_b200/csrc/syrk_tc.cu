@@ -7,18 +7,24 @@
 // memory (d contiguous), which tcgen05 supports for bf16.
 //
 // Design (sm_100a):
-//  * one CTA per 128 x 256 output tile of the upper triangle (tiles entirely
-//    below the diagonal are never launched: ~half of the dense work);
+//  * persistent: one CTA per SM walks 128 x 256 output tiles of the upper
+//    triangle (tiles entirely below the diagonal are never computed: ~half
+//    of the dense work), tile t = blockIdx.x + i * gridDim.x;
 //  * warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner), warps 2-5 =
-//    epilogue; 4-stage smem ring of 64-token slices (48 KB per stage);
+//    epilogue; 4-stage smem ring of 64-token slices (48 KB per stage) that
+//    runs across tile boundaries;
 //  * tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M = 128, N = 256, K = 16,
-//    accumulator in 256 TMEM columns;
+//    two accumulators of 256 TMEM columns: the epilogue of tile i reads one
+//    while the MMAs of tile i + 1 fill the other;
 //  * epilogue: tcgen05.ld 32x32b, each element written once: (i, j) for
 //    i <= j and its mirror (j, i) for i < j, so H stays fully symmetric.
-//    Each output element belongs to exactly one CTA: no atomics.
-//  * the whole token range is one K loop, so concurrently running CTAs walk
-//    the same token slices and each slice of A is read from HBM about once
-//    per wave (the rest hits L2).
+//    Each output element belongs to exactly one tile: no atomics.
+//  * tile order: strips of 16 tile rows, column-major inside a strip, so
+//    the ~148 tiles in flight at any time span ~2k rows and ~2.4k columns
+//    of H and share their token slices in L2 (all tiles have the same K
+//    loop, so the CTAs walk the tokens nearly in step).  A row-major order
+//    over a wide H makes every concurrent tile read different columns and
+//    the kernel DRAM-bound.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -33,32 +39,47 @@ constexpr int BOX_BYTES = 64 * BK * 2;                 // one 64-column x 64-tok
 constexpr int A_BYTES = BM * BK * 2;                   // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                   // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;         // 48 KB
+constexpr int NBARS = 2 * STAGES + 4;                  // full, empty, acc_full[2], acc_empty[2]
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = BN;
+constexpr int EPI_WARPS = 4;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int STRIP = 16;                              // tile rows per raster strip
 
 struct SyrkArgs {
   float* H;
   int64_t d;
   int nk;       // number of 64-token slices
   int nr, nc;   // row / column tile counts
+  int ntiles;   // tiles of the upper triangle
   int accumulate;
 };
 
+// Tile t of the raster order -> (tile row, tile column).  Tile (tr, tc) is
+// kept when it reaches the upper triangle: tc >= tr * BM / BN = tr / 2, i.e.
+// tr < 2 tc + 2.  Strips of STRIP tile rows, column-major inside a strip.
 __device__ __forceinline__ void tile_of(int t, int nr, int nc, int& tr, int& tc) {
-  for (tr = 0; tr < nr; ++tr) {
-    const int first = (tr * BM) / BN;
-    const int cnt = nc - first;
+  for (int s0 = 0; s0 < nr; s0 += STRIP) {
+    const int s1 = min(s0 + STRIP, nr);
+    int cnt = 0;
+    for (int r = s0; r < s1; ++r) cnt += nc - r / 2;
     if (t < cnt) {
-      tc = first + t;
-      return;
+      for (int c = s0 / 2; c < nc; ++c) {
+        const int rend = min(s1, 2 * c + 2);
+        const int k = rend - s0;
+        if (t < k) {
+          tr = s0 + t;
+          tc = c;
+          return;
+        }
+        t -= k;
+      }
     }
     t -= cnt;
   }
-  tc = nc;  // unreachable for a valid grid
+  tr = nr;  // unreachable for t < ntiles
+  tc = nc;
 }
-
-__device__ __forceinline__ void put(float* p, float x, int acc) { *p = acc ? (*p + x) : x; }
 
 __global__ void __launch_bounds__(THREADS, 1)
     syrk_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmap, SyrkArgs args) {
@@ -66,22 +87,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t full0 = smem_u32(&bars[0]);
   const uint32_t empty0 = smem_u32(&bars[STAGES]);
-  const uint32_t accbar = smem_u32(&bars[2 * STAGES]);
+  const uint32_t accfull0 = smem_u32(&bars[2 * STAGES]);
+  const uint32_t accempty0 = smem_u32(&bars[2 * STAGES + 2]);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int tr, tc;
-  tile_of(blockIdx.x, args.nr, args.nc, tr, tc);
-  const int r0 = tr * BM, c0 = tc * BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(accbar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accfull0 + 8 * b, 1);
+      mbar_init(accempty0 + 8 * b, EPI_WARPS);
+    }
+    *abort_s = 0;
     fence_mbar_init();
     prefetch_tmap(&tmap);
   }
@@ -94,102 +118,166 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t stage0 = smem_u32(smem);
+  const int nk = args.nk;
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < args.nk; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait(empty0 + 8 * s, ph ^ 1)) break;
-        const uint32_t full = full0 + 8 * s;
-        mbar_arrive_expect_tx(full, STAGE_BYTES);
-        const uint32_t a = stage0 + s * STAGE_BYTES;
-        const uint32_t b = a + A_BYTES;
-        const int y = kb * BK;
-        tma_load_2d(a, &tmap, full, r0, y);
-        tma_load_2d(a + BOX_BYTES, &tmap, full, r0 + 64, y);
+      uint32_t it = 0;   // k slices issued, over all tiles
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < args.ntiles; t += gridDim.x) {
+        int tr, tc;
+        tile_of(t, args.nr, args.nc, tr, tc);
+        const int r0 = tr * BM, c0 = tc * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (*abort_s || !mbar_wait(empty0 + 8 * s, ph ^ 1)) {
+            *abort_s = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t full = full0 + 8 * s;
+          mbar_arrive_expect_tx(full, STAGE_BYTES);
+          const uint32_t a = stage0 + s * STAGE_BYTES;
+          const uint32_t b = a + A_BYTES;
+          const int y = kb * BK;
+          tma_load_2d(a, &tmap, full, r0, y);
+          tma_load_2d(a + BOX_BYTES, &tmap, full, r0 + 64, y);
 #pragma unroll
-        for (int h = 0; h < 4; ++h) tma_load_2d(b + h * BOX_BYTES, &tmap, full, c0 + 64 * h, y);
-        issued = kb + 1;
+          for (int h = 0; h < 4; ++h) tma_load_2d(b + h * BOX_BYTES, &tmap, full, c0 + 64 * h, y);
+        }
       }
       // Make sure no copy is still landing when the CTA leaves (normally
       // these phases completed long ago and each test returns at once).
-      for (int kb = issued - STAGES > 0 ? issued - STAGES : 0; kb < issued; ++kb)
-        mbar_wait(full0 + 8 * (kb % STAGES), (kb / STAGES) & 1);
+      for (uint32_t k = it > STAGES ? it - STAGES : 0; k < it; ++k)
+        mbar_wait(full0 + 8 * (k % STAGES), (k / STAGES) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, true, true);
-      for (int kb = 0; kb < args.nk; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait(full0 + 8 * s, ph)) break;
-        tc_fence_after();
-        const uint32_t a = stage0 + s * STAGE_BYTES;
-        const uint32_t b = a + A_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          // 16 tokens = 16 rows of 128 B inside every box: +2048 B per step.
-          const uint64_t ad = smem_desc_sw128(a + kk * 2048, BOX_BYTES, 1024);
-          const uint64_t bd = smem_desc_sw128(b + kk * 2048, BOX_BYTES, 1024);
-          mma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+      uint32_t it = 0;
+      int tl = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < args.ntiles; t += gridDim.x, ++tl) {
+        const int b = tl & 1;
+        const uint32_t u = (uint32_t)(tl >> 1);
+        // the epilogue of tile tl - 2 has read accumulator b
+        if (u > 0 && (*abort_s || !mbar_wait(accempty0 + 8 * b, (u - 1) & 1))) {
+          *abort_s = 1;
+          break;
         }
-        mma_commit(empty0 + 8 * s);
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(b * BN);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (*abort_s || !mbar_wait(full0 + 8 * s, ph)) {
+            *abort_s = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = stage0 + s * STAGE_BYTES;
+          const uint32_t bb = a + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // 16 tokens = 16 rows of 128 B inside every box: +2048 B per step.
+            const uint64_t ad = smem_desc_sw128(a + kk * 2048, BOX_BYTES, 1024);
+            const uint64_t bd = smem_desc_sw128(bb + kk * 2048, BOX_BYTES, 1024);
+            mma_bf16(acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(empty0 + 8 * s);
+        }
+        if (ok) mma_commit(accfull0 + 8 * b);
       }
-      mma_commit(accbar);
     }
     __syncwarp();
   } else {
     // Epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (its sub-partition).
     const int q = warp & 3;
-    bool ok = true;
-    if (lane == 0) ok = mbar_wait(accbar, 0);
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    __syncwarp();
-    if (ok) {
+    const int64_t d = args.d;
+    float* H = args.H;
+    const int accm = args.accumulate;
+    int tl = 0;
+    for (int t = blockIdx.x; t < args.ntiles; t += gridDim.x, ++tl) {
+      const int b = tl & 1;
+      const uint32_t u = (uint32_t)(tl >> 1);
+      int ok = 1;
+      if (lane == 0) ok = (!*abort_s && mbar_wait(accfull0 + 8 * b, u & 1)) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      if (!ok) {
+        if (lane == 0) *abort_s = 1;
+        break;
+      }
       tc_fence_after();
-      const int64_t d = args.d;
+      int tr, tc;
+      tile_of(t, args.nr, args.nc, tr, tc);
+      const int r0 = tr * BM, c0 = tc * BN;
       const int64_t i = r0 + q * 32 + lane;
-      float* H = args.H;
-      const int acc = args.accumulate;
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; ++cc) {
-        uint32_t v[32];
-        __syncwarp();  // the TMEM load is warp-collective
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + cc * 32, v);
-        tmem_wait_ld();
         const int64_t jb = c0 + cc * 32;
-        if (i < d) {
-          const bool dense = (jb >= i) && (jb + 32 <= d) &&
-                             ((reinterpret_cast<uintptr_t>(H + i * d + jb) & 15) == 0);
+        // Every load of the element pair (i, jb..jb+31) / (jb..jb+31, i) is
+        // issued before the accumulator is read and before any store, so the
+        // read-modify-write costs one memory round trip per 32 columns
+        // instead of one per element.
+        const bool dense = (i < d) && (jb >= i) && (jb + 32 <= d) &&
+                           ((reinterpret_cast<uintptr_t>(H + i * d + jb) & 15) == 0);
+        float old[32], mir[32];
+        if (accm) {
           if (dense) {
-            float4* dst = reinterpret_cast<float4*>(H + i * d + jb);
+            const float4* src = reinterpret_cast<const float4*>(H + i * d + jb);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              float4 x = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
-                                     __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3]));
-              if (acc) {
-                const float4 o = dst[t];
-                x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
-              }
-              dst[t] = x;
+            for (int e = 0; e < 8; ++e) {
+              const float4 o = src[e];
+              old[4 * e] = o.x; old[4 * e + 1] = o.y; old[4 * e + 2] = o.z; old[4 * e + 3] = o.w;
             }
           } else {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-              const int64_t j = jb + t;
-              if (j < d && i <= j) put(H + i * d + j, __uint_as_float(v[t]), acc);
+            for (int e = 0; e < 32; ++e) {
+              const int64_t j = jb + e;
+              old[e] = (i < d && j < d && i <= j) ? H[i * d + j] : 0.f;
             }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int64_t j = jb + e;
+            mir[e] = (i < d && j < d && i < j) ? H[j * d + i] : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) old[e] = mir[e] = 0.f;
+        }
+        uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(b * BN + cc * 32), v);
+        tmem_wait_ld();
+        if (dense) {
+          float4* dst = reinterpret_cast<float4*>(H + i * d + jb);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]) + old[4 * e], __uint_as_float(v[4 * e + 1]) + old[4 * e + 1],
+                                 __uint_as_float(v[4 * e + 2]) + old[4 * e + 2],
+                                 __uint_as_float(v[4 * e + 3]) + old[4 * e + 3]);
+        } else if (i < d) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int64_t j = jb + e;
+            if (j < d && i <= j) H[i * d + j] = __uint_as_float(v[e]) + old[e];
           }
         }
         // Mirror (j, i) for i < j: 32 lanes write 32 consecutive floats.
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const int64_t j = jb + t;
-          if (i < d && j < d && i < j) put(H + j * d + i, __uint_as_float(v[t]), acc);
+        for (int e = 0; e < 32; ++e) {
+          const int64_t j = jb + e;
+          if (i < d && j < d && i < j) H[j * d + i] = __uint_as_float(v[e]) + mir[e];
         }
       }
+      // accumulator b may be refilled once all four warps have read it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty0 + 8 * b);
     }
   }
   tc_fence_before();
@@ -256,10 +344,12 @@ kronq_status syrk_bf16_tc(const void* A, int64_t T, int64_t d, int64_t lda, floa
   args.accumulate = zero_first ? 0 : 1;
   int64_t ntiles = 0;
   for (int tr = 0; tr < args.nr; ++tr) ntiles += args.nc - (tr * BM) / BN;
+  args.ntiles = (int)ntiles;
 
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(&syrk_bf16_tc_kernel), SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(syrk)");
-  syrk_bf16_tc_kernel<<<(unsigned)ntiles, THREADS, SMEM_BYTES, s>>>(map, args);
+  const int64_t grid = ntiles < (int64_t)sm_count() ? ntiles : (int64_t)sm_count();
+  syrk_bf16_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, s>>>(map, args);
   KQ_LAUNCH_CHECK("syrk_bf16_tc_kernel");
   return KRONQ_OK;
 }
