@@ -257,6 +257,19 @@ kronq_status kronq_unpack(const uint32_t* in, int64_t m, int64_t n, int bits, ui
  *   Synchronises the stream.
  * ------------------------------------------------------------------------- */
 kronq_status kronq_device_status(int* out, kronq_stream_t s);
+/* kronq_wait_selftest: launches one CTA whose bounded wait is never
+ *   satisfied, so that it gives up after limit_ns (0 < limit_ns <= 1e9)
+ *   exactly as a stuck wait inside the pass would: which 0 waits on an
+ *   mbarrier phase that nothing completes (the wait of every tensor-core
+ *   kernel), which 1 on a step counter that no CTA advances (the cross-CTA
+ *   wait of the persistent factorisation, which then raises its abort
+ *   flag).  The wait records KRONQ_ERR_TIMEOUT in the device status word
+ *   (read and cleared by kronq_device_status) and the kernel returns; the
+ *   CUDA context stays usable.  workspace: >= 3 ints of device memory;
+ *   on return w[0] = counter (0), w[1] = abort flag (1 for which 1),
+ *   w[2] = 1 when the wait gave up.  Asynchronous on s. */
+kronq_status kronq_wait_selftest(int which, uint64_t limit_ns, void* workspace, size_t ws_bytes,
+                                 kronq_stream_t s);
 size_t kronq_kfac_loss_workspace_bytes(int64_t m, int64_t n);
 kronq_status kronq_kfac_loss(const float* E, const float* HG, int64_t m, int64_t n, double* out,
                              void* workspace, size_t ws_bytes, kronq_stream_t s);

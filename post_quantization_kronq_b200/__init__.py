@@ -19,7 +19,8 @@ __all__ = [
     "kronq_allocate_topn_types", "kronq_biip_workspace_bytes", "kronq_biip_forward",
     "kronq_biip_inverse", "kronq_quantize_workspace_bytes", "kronq_quantize_layer",
     "kronq_quantize_layer_static",
-    "kronq_pack", "kronq_unpack", "kronq_device_status", "kronq_kfac_loss_workspace_bytes",
+    "kronq_pack", "kronq_unpack", "kronq_device_status", "kronq_wait_selftest",
+    "kronq_kfac_loss_workspace_bytes",
     "kronq_kfac_loss", "kronq_launch_count", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
     "EST_INPUT", "EST_MARGINAL", "EST_FROBENIUS", "EST_FLIPFLOP",
     "kronq_kron_factors_workspace_bytes", "kronq_kron_factors",
@@ -186,6 +187,13 @@ def kronq_device_status(stream=None) -> int:
     v = ctypes.c_int(0)
     check(lib.kronq_device_status(ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+def kronq_wait_selftest(which: int, limit_ns: int, ws, stream=None):
+    """One CTA whose bounded wait (0: mbarrier, 1: cross-CTA counter) is never
+    satisfied gives up after limit_ns; read the result with kronq_device_status."""
+    check(lib.kronq_wait_selftest(int(which), int(limit_ns), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream)))
 
 
 def kronq_kron_factors_workspace_bytes(T: int, n: int, m: int) -> int:

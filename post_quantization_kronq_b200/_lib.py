@@ -58,6 +58,7 @@ SIGNATURES = {
     "kronq_pack": (_int, [_vp, _i64, _i64, _int, _vp, _vp]),
     "kronq_unpack": (_int, [_vp, _i64, _i64, _int, _vp, _vp]),
     "kronq_device_status": (_int, [_ip, _vp]),
+    "kronq_wait_selftest": (_int, [_int, _u64, _vp, _sz, _vp]),
     "kronq_kfac_loss_workspace_bytes": (_sz, [_i64, _i64]),
     "kronq_kfac_loss": (_int, [_vp, _vp, _i64, _i64, _dp, _vp, _sz, _vp]),
     "kronq_kron_factors_workspace_bytes": (_sz, [_i64, _i64, _i64]),

@@ -441,6 +441,16 @@ kronq_status kronq_device_status(int* out, kronq_stream_t s) {
   return KRONQ_OK;
 }
 
+kronq_status kronq_wait_selftest(int which, uint64_t limit_ns, void* workspace, size_t ws_bytes,
+                                 kronq_stream_t s) {
+  if (which != 0 && which != 1) return fail(KRONQ_ERR_INVALID_ARG, "wait_selftest: which must be 0 or 1");
+  if (limit_ns == 0 || limit_ns > 1000000000ull)
+    return fail(KRONQ_ERR_INVALID_ARG, "wait_selftest: limit_ns must be in (0, 1e9]");
+  if (!workspace || ws_bytes < 3 * sizeof(int) || !aligned(workspace, 4))
+    return fail(KRONQ_ERR_INVALID_ARG, "wait_selftest: workspace must hold 3 ints, 4-byte aligned");
+  return wait_selftest(which, (unsigned long long)limit_ns, static_cast<int*>(workspace), as_stream(s));
+}
+
 size_t kronq_kfac_loss_workspace_bytes(int64_t m, int64_t n) {
   if (m <= 0 || n <= 0) return 0;
   Carver c(nullptr);

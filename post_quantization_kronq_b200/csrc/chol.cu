@@ -799,7 +799,8 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // Thread 0 waits until *p >= target (bounded, and ended by the abort flag);
 // the result is shared with the whole CTA.  Orders the CTA's later reads
 // (generic and TMA) after the other CTAs' published writes.
-__device__ __forceinline__ bool cta_wait(const int* p, int target, int* abortf) {
+__device__ __forceinline__ bool cta_wait(const int* p, int target, int* abortf,
+                                         unsigned long long limit_ns = kWaitLimitNs) {
   int ok = 1;
   if (threadIdx.x == 0 && ld_acquire_gpu(p) < target) {
     const unsigned long long t0 = global_ns();
@@ -809,7 +810,7 @@ __device__ __forceinline__ bool cta_wait(const int* p, int target, int* abortf) 
         ok = 0;
         break;
       }
-      if ((it & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+      if ((it & 63u) == 0 && global_ns() - t0 > limit_ns) {
         record_timeout();
         atomicExch(abortf, 1);
         ok = 0;
@@ -1018,7 +1019,41 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
   }
 }
 
+// Self-test of the two bounded waits above: one CTA waits on a condition
+// that nothing satisfies, with a short bound.  which 0: an mbarrier phase
+// that no thread or copy completes (mbar_wait, as every tensor-core kernel
+// uses it); which 1: a step counter that no CTA increments (cta_wait, as the
+// persistent factorisation uses it), which also raises the abort flag.
+// w[0] = counter, w[1] = abort flag, w[2] = 1 when the wait gave up.
+__global__ void __launch_bounds__(32) wait_selftest_kernel(int which, unsigned long long limit_ns, int* w) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    w[0] = 0;
+    w[1] = 0;
+    w[2] = 0;
+    __threadfence();
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  bool gave_up;
+  if (which == 0) {
+    int ok = 1;
+    if (threadIdx.x == 0) ok = mbar_wait(smem_u32(&bar), 0u, limit_ns) ? 1 : 0;
+    gave_up = __syncthreads_and(ok) == 0;
+  } else {
+    gave_up = !cta_wait(&w[0], 1, &w[1], limit_ns);
+  }
+  if (threadIdx.x == 0) w[2] = gave_up ? 1 : 0;
+}
+
 }  // namespace
+
+kronq_status wait_selftest(int which, unsigned long long limit_ns, int* w, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(which, limit_ns, w);
+  KQ_LAUNCH_CHECK("wait_selftest_kernel");
+  return KRONQ_OK;
+}
 
 cudaError_t status_fetch_chol(int* out, cudaStream_t s) {
   int v = 0;

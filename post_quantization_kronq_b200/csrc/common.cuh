@@ -96,14 +96,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity; gives up after kWaitLimitNs,
-// records KRONQ_ERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Waits for the phase with the given parity; gives up after limit_ns
+// (kWaitLimitNs unless a self-test passes a shorter bound), records
+// KRONQ_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+    if ((it & 255u) == 0 && global_ns() - t0 > limit_ns) {
       record_timeout();
       return false;
     }

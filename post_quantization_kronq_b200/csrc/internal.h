@@ -127,6 +127,9 @@ cudaError_t status_fetch_schur(int* out, cudaStream_t s);
 // In: H (n x n) full symmetric.  Out: U (upper) with U^T U = (H + lambda I)^-1,
 // dead-column flags, info.  ws: see chol_workspace_bytes.
 size_t chol_workspace_bytes(int64_t n);
+// One CTA whose bounded wait (which 0: mbarrier, 1: cross-CTA counter) is
+// never satisfied; gives up after limit_ns.  w: 3 device ints.
+kronq_status wait_selftest(int which, unsigned long long limit_ns, int* w, cudaStream_t s);
 cudaError_t status_fetch_chol(int* out, cudaStream_t s);
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
                                 uint8_t* dead, int* info, void* ws, cudaStream_t s);

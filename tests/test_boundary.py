@@ -209,3 +209,12 @@ def test_decode_matvec_validation():
     assert call(nbytes=ws - 1) == _lib.ERR_INVALID_ARG
     assert call(x=None) == _lib.ERR_INVALID_ARG
     assert call(n=257 * 2) == _lib.ERR_UNSUPPORTED      # odd factor 257 of a rotated dimension
+
+
+def test_wait_selftest_validation():
+    L = _lib.lib
+    assert _st(L.kronq_wait_selftest(2, 1000000, FAKE, 16, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_wait_selftest(0, 0, FAKE, 16, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_wait_selftest(0, 2000000000, FAKE, 16, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_wait_selftest(1, 1000000, None, 16, None)) == _lib.ERR_INVALID_ARG
+    assert _st(L.kronq_wait_selftest(1, 1000000, FAKE, 8, None)) == _lib.ERR_INVALID_ARG
