@@ -2,6 +2,7 @@
 
     python -m post_quantization_kronq_b200.opbench accumulate --tokens 16384 --d 4096 [--reps 3]
     python -m post_quantization_kronq_b200.opbench biip --m 4096 --n 4096
+    python -m post_quantization_kronq_b200.opbench biip_inverse --m 2048 --n 28672
     python -m post_quantization_kronq_b200.opbench quantize --m 4096 --n 4096 --bits 2
     python -m post_quantization_kronq_b200.opbench pack --m 8192 --n 28672 --bits 2
     python -m post_quantization_kronq_b200.opbench kronfactors --est flipflop --tokens 131072 --m 4096 --n 4096
@@ -31,7 +32,8 @@ def main(argv=None):
     from synth import llama_layer
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["accumulate", "biip", "quantize", "pack", "kronfactors", "decode"])
+    ap.add_argument("op", choices=["accumulate", "biip", "biip_inverse", "quantize", "pack", "kronfactors",
+                                   "decode"])
     ap.add_argument("--est", choices=["input", "marginal", "frobenius", "flipflop"], default="flipflop")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--tokens", type=int, default=16384)
@@ -49,6 +51,14 @@ def main(argv=None):
         H = torch.empty(a.d, a.d, device=dev)
         run = lambda: kq.kronq_accumulate_factors(X, H, zero_first=True)  # noqa: E731
         units = {"flops": a.tokens * a.d * (a.d + 1)}
+    elif a.op == "biip_inverse":
+        # two row passes over W alone (rows of n, then rows of m), no factors
+        Wt = torch.randn(a.m, a.n, device=dev)
+        d_in = torch.ones(a.n, device=dev)
+        d_out = torch.ones(a.m, device=dev)
+        ws = kq.workspace(kq.kronq_biip_workspace_bytes(a.m, a.n), dev)
+        run = lambda: kq.kronq_biip_inverse(Wt, 0, "full", d_in, d_out, ws=ws)  # noqa: E731
+        units = {"bytes": 16 * a.m * a.n}
     elif a.op == "decode":
         ng = -(-a.n // a.group)
         codes = torch.randint(0, 2 ** a.bits, (a.m, a.n), dtype=torch.uint8, device=dev)
@@ -112,7 +122,7 @@ def main(argv=None):
     e1.record(s)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.reps
-    if a.op == "decode":
+    if a.op in ("decode", "biip_inverse"):
         units["gbs"] = units["bytes"] / (ms / 1e3) / 1e9
     if a.op == "kronfactors":
         units["info"] = int(info.item())

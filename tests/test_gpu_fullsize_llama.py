@@ -1,0 +1,217 @@
+"""Parity at the Llama MLP sizes, in the launch configuration the benchmark
+uses: one LayerPass over bf16 X, G, W resident on the device, the factors
+accumulated in token chunks.
+
+  Llama-2-7B MLP     up 11008 x 4096 (W2 g64), down 4096 x 11008 (W3 g128),
+                     T = 131072 tokens
+  Llama-3-70B MLP    gate 28672 x 8192, down 8192 x 28672 (W2 g128),
+                     T = 262144 tokens in 16 chunks of 16384
+
+(KronQ README "Model zoo": Llama-2-7B and Llama-3-70B; abstract: 2-bit
+Llama-3-70B.)  The odd factors of these lengths (43 for 11008, 7 for 14336
+and 28672) take the DCT paths of the row transform; the factorisation runs
+128 to 448 diagonal steps.  The float64 oracle checks each stage on what it
+can compute piece by piece, fed the GPU's output of the previous stage:
+
+* factors: a 64 x 64 block of H_X and of H_G at sampled indices, from the
+  same bf16 tokens' sampled channels; the traces against the float64 sum of
+  the GPU factor's diagonal;
+* BiIP: the rescale vectors, and sampled rows of W~, H~_X and H~_G (rows of
+  the oracle's rotations times the rescaled inputs, then the rotation);
+* the factor U: against the oracle's U of the GPU's damped H~_X (for
+  n = 28672 its trailing 4096 x 4096 block, which the reverse factorisation
+  computes from that block of H alone, and U^T U A e_j = e_j on sampled
+  columns j), within twice the error of a float32 LAPACK factorisation of
+  the same matrix -- float32 is the precision of the kernels, and its error
+  grows with the condition number (1e5 and more for the rectified down_proj
+  inputs);
+* the sweep: 64 sampled rows of the GPU's W~ through the float64 sweep
+  given the GPU's U (codes within 0.5 %), and end to end against the
+  oracle's U: codes within 0.5 %, or within 1.5 x the disagreement that the
+  float32 LAPACK factor alone causes when that is larger; the rows'
+  quadratic error within 1 %.
+"""
+import numpy as np
+import pytest
+import torch
+from scipy.linalg import solve_triangular
+
+from oracle import biip, factors, sweep
+from post_quantization_kronq_b200.layer import LayerPass
+from synth import llama_layer
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+CASES = [
+    # name, m, n, T, chunk, bits, group, w_std, rectified X (down_proj input)
+    ("llama2_7b_up", 11008, 4096, 131072, 131072, 2, 64, 0.02, False),
+    ("llama2_7b_down", 4096, 11008, 131072, 131072, 3, 128, 0.02, True),
+    ("llama3_70b_gate", 28672, 8192, 262144, 16384, 2, 128, 0.015, False),
+    ("llama3_70b_down", 8192, 28672, 262144, 16384, 2, 128, 0.015, True),
+]
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _columns(A, idx, chunk=32768):
+    """A[:, idx] of a device bf16 token matrix, as float64 on the host."""
+    it = torch.as_tensor(idx, device=A.device)
+    return np.concatenate([A[t0:t0 + chunk].index_select(1, it).float().cpu().numpy()
+                           for t0 in range(0, A.shape[0], chunk)]).astype(np.float64)
+
+
+def _rows_times(R, H, d, chunk=2048):
+    """R @ (H / d[:, None] / d[None, :]) for a device fp32 H, row chunks."""
+    out = np.zeros((R.shape[0], H.shape[1]))
+    for r0 in range(0, H.shape[0], chunk):
+        Hc = to_np(H[r0:r0 + chunk]) / d[r0:r0 + chunk, None] / d[None, :]
+        out += R[:, r0:r0 + Hc.shape[0]] @ Hc
+    return out
+
+
+def _rotation_rows(rows, L, seed, side):
+    """Rows ``rows`` of the oracle's rotation of length L (e_i^T V = row i)."""
+    E = np.zeros((len(rows), L))
+    E[np.arange(len(rows)), rows] = 1.0
+    return biip.rotate_rows(E, seed, side, inverse=True)
+
+
+def _u_times(U, V, chunk=2048, transpose=False):
+    """U @ V (or U^T @ V) for a device fp32 U (upper triangle used), V host."""
+    n = U.shape[0]
+    out = np.zeros((n, V.shape[1]))
+    for r0 in range(0, n, chunk):
+        Uc = np.triu(to_np(U[r0:r0 + chunk]), k=r0)
+        if transpose:
+            out += Uc.T @ V[r0:r0 + Uc.shape[0]]
+        else:
+            out[r0:r0 + Uc.shape[0]] = Uc @ V
+    return out
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_llama_mlp_full_size_sampled(case):
+    name, m, n, T, chunk, bits, group, w_std, rect = case
+    seed = 0
+    rng = np.random.default_rng(11)
+    W, X, G = llama_layer(m, n, T, seed=seed, device=DEV, w_std=w_std, rectified=rect)
+    lp = LayerPass(m, n, bits=bits, group=group, seed=seed)
+    lp.accumulate(X, G, chunk=chunk)
+    trx, trg, s = lp.sensitivity()
+    HX = lp.HX.clone()
+    HG = lp.HG.clone()
+    lp.transform(W)
+    Wt = lp.Wt.clone()
+    HXt = lp.HX.clone()
+    lp.quantize()
+    torch.cuda.synchronize()
+    assert int(lp.info.item()) == 0
+
+    # ---- factors: a sampled block of each, and the traces
+    for A, H, d, tr in ((X, HX, n, trx), (G, HG, m, trg)):
+        idx = np.sort(rng.choice(d, 64, replace=False))
+        ref = factors.factor(_columns(A, idx))
+        it = torch.as_tensor(idx, device=DEV)
+        got = to_np(H.index_select(0, it).index_select(1, it))
+        assert rel(got, ref) < 1e-3
+        diag = to_np(torch.diagonal(H))
+        assert abs(tr - factors.trace_of_factor(np.diag(diag))) <= 1e-6 * tr
+    assert abs(s - trx * trg) <= 1e-12 * s
+    del X, G
+    torch.cuda.empty_cache()
+
+    # ---- BiIP: rescale vectors and sampled rows of the three transforms
+    Wn = to_np(W)
+    din = biip.rescale_vector(to_np(torch.diagonal(HX)), np.sum(Wn * Wn, axis=0), 0.25)
+    dout = biip.rescale_vector(to_np(torch.diagonal(HG)), np.sum(Wn * Wn, axis=1), 0.25)
+    assert rel(to_np(lp.d_in), din) < 1e-5 and rel(to_np(lp.d_out), dout) < 1e-5
+    rw = np.sort(rng.choice(m, 8, replace=False))
+    Wp = (dout[:, None] * Wn) * din[None, :]
+    ref_w = biip.rotate_rows(_rotation_rows(rw, m, seed, 1) @ Wp, seed, 0)
+    assert rel(to_np(Wt[torch.as_tensor(rw, device=DEV)]), ref_w) < 1e-5
+    del Wn, Wp
+    rx = np.sort(rng.choice(n, 8, replace=False))
+    ref_hx = biip.rotate_rows(_rows_times(_rotation_rows(rx, n, seed, 0), HX, din), seed, 0)
+    assert rel(to_np(HXt[torch.as_tensor(rx, device=DEV)]), ref_hx) < 1e-5
+    rg = np.sort(rng.choice(m, 4, replace=False))
+    ref_hg = biip.rotate_rows(_rows_times(_rotation_rows(rg, m, seed, 1), HG, dout), seed, 1)
+    assert rel(to_np(lp.HG[torch.as_tensor(rg, device=DEV)]), ref_hg) < 1e-5
+    del HX, HG
+    torch.cuda.empty_cache()
+
+    # ---- the factor U of the damped H~_X, held to the float32 floor: the
+    # error of a float32 LAPACK factorisation of the same matrix (it grows
+    # with the condition number; rectified down_proj inputs give a large
+    # common mean and condition numbers of 1e5 and more)
+    hxt_diag = to_np(torch.diagonal(HXt))
+    dead = hxt_diag == 0
+    lam = 0.01 * float(np.mean(np.where(dead, 1.0, hxt_diag)))
+    Ug = np.triu(to_np(lp.HX))
+    U = U32 = None
+    if n <= 11008:
+        H1, _, _ = sweep.dead_columns(to_np(HXt), np.zeros((1, n)))
+        A, _ = sweep.damp(H1, 0.01)
+        U = sweep.chol_upper_of_inverse(A)
+        U32 = sweep.chol_upper_of_inverse_f32(A)
+        e_gpu, e_32 = rel(Ug, U), rel(U32, U)
+        assert e_gpu <= max(2 * e_32, 2e-5), (e_gpu, e_32)
+        del A, H1
+    else:
+        # the reverse factorisation's trailing block depends on that block
+        # of the damped factor alone
+        j = n - 4096
+        H1, _, _ = sweep.dead_columns(to_np(HXt[j:, j:]), np.zeros((1, 4096)))
+        Hs = H1.copy()
+        Hs[np.diag_indices_from(Hs)] += lam     # the damping of the whole matrix
+        Ut = sweep.chol_upper_of_inverse(Hs)
+        Ut32 = sweep.chol_upper_of_inverse_f32(Hs)
+        e_gpu, e_32 = rel(Ug[j:, j:], Ut), rel(Ut32, Ut)
+        assert e_gpu <= max(2 * e_32, 2e-5), (e_gpu, e_32)
+        del H1, Hs, Ut, Ut32
+        # U^T U A e_j = e_j on sampled columns of the whole matrix (a loose
+        # bound: the float32 residual scales with the condition number)
+        cols = np.array([0, 37, 63, 64, 5000, n // 2, n - 4097, n - 1])
+        Acols = to_np(HXt.index_select(1, torch.as_tensor(cols, device=DEV)))
+        Acols[cols, np.arange(len(cols))] += lam
+        Z = _u_times(lp.HX, _u_times(lp.HX, Acols), transpose=True)
+        Eye = np.zeros_like(Z)
+        Eye[cols, np.arange(len(cols))] = 1.0
+        assert rel(Z, Eye) < 0.1, rel(Z, Eye)
+
+    # ---- the sweep on sampled rows
+    rows = np.sort(rng.choice(m, 64, replace=False))
+    W1 = to_np(Wt[torch.as_tensor(rows, device=DEV)])
+    W1[:, dead] = 0.0
+    got = lp.codes[torch.as_tensor(rows, device=DEV)].cpu().numpy().astype(np.int64)
+    Q = to_np(lp.Wt[torch.as_tensor(rows, device=DEV)])
+    # given the GPU's factor, the float64 sweep takes the same decisions
+    ref_g = sweep.gptq_sweep(W1, Ug, bits, group, True, block=128)
+    dis_g = float(np.mean(got != ref_g["codes"]))
+    assert dis_g <= 0.005, dis_g
+    if U is not None:
+        # end to end against the float64 oracle: within 0.5 %, or within what
+        # the float32 factorisation alone causes when that is more
+        ref = sweep.gptq_sweep(W1, U, bits, group, True, block=128)
+        ref32 = sweep.gptq_sweep(W1, U32.astype(np.float64), bits, group, True, block=128)
+        dis = float(np.mean(got != ref["codes"]))
+        dis_32 = float(np.mean(ref32["codes"] != ref["codes"]))
+        assert dis <= max(0.005, 1.5 * dis_32), (dis, dis_32)
+        Uq = U
+    else:
+        ref = ref_g
+        Uq = Ug
+    # quadratic error of the rows under the damped factor: with dW = E U it
+    # is |E|^2 = |dW U^-1|^2, compared with the oracle sweep's
+    e_ref = float(np.sum(ref["E"] ** 2))
+    Ginv = solve_triangular(Uq, (W1 - Q).T, trans="T", lower=False).T   # dW U^-1
+    e_gpu = float(np.sum(Ginv ** 2))
+    assert abs(e_gpu - e_ref) / e_ref < 0.01, (e_gpu, e_ref)

@@ -201,6 +201,10 @@ def _sweep_inputs(m, n, seed):
 @pytest.mark.parametrize("m,n,bits,group,asym", [
     (69, 424, 4, 128, True), (69, 424, 2, 64, True), (69, 424, 3, -1, True),
     (40, 512, 2, 256, True), (33, 300, 4, 32, False), (16, 128, 3, 128, True), (5, 7, 2, -1, True),
+    # groups of 16 columns and fewer: the grid changes inside a 32-column
+    # round, so the sweep keeps per-column outputs (GPTQ's --w_groupsize)
+    (69, 424, 2, 16, True), (37, 300, 4, 8, True), (40, 264, 3, 4, False), (21, 160, 2, 2, True),
+    (19, 136, 4, 1, True),
 ])
 def test_sweep_bit_exact_against_f32_oracle(m, n, bits, group, asym):
     Wt, U = _sweep_inputs(m, n, seed=m * n)
@@ -236,6 +240,49 @@ def test_sweep_fast_path_close_to_ordered():
     torch.cuda.synchronize()
     dis = np.mean(lp.codes.cpu().numpy().astype(np.int64) != ref["codes"])
     assert dis <= 0.005
+
+
+# ------------------------------------------------------------------ dead columns
+# GPTQ's dead-column rule (a zero diagonal of H~_X): H_jj := 1 and the column
+# of W~ is quantized from zero.
+def test_dead_columns_given_factor():
+    m, n = 48, 384
+    W, X, _ = tiny_layer(m=m, n=n, T=4 * n, seed=21)
+    X[:, [3, 130, 257, 383]] = 0.0          # four input channels never active
+    H = (X.astype(np.float64).T @ X.astype(np.float64)).astype(np.float32)
+    assert np.all(np.diag(H)[[3, 130, 257, 383]] == 0.0)
+    lp = LayerPass(m, n, bits=3, group=128)
+    lp.HX.copy_(torch.from_numpy(H))
+    lp.Wt.copy_(torch.from_numpy(W))
+    lp.quantize()
+    torch.cuda.synchronize()
+    assert int(lp.info.item()) == 0
+    ref = sweep.quantize_factored(W, H, 3, 128, True, 0.01, block=128)
+    assert np.array_equal(np.nonzero(ref["dead"])[0], [3, 130, 257, 383])
+    assert rel(np.triu(to_np(lp.HX)), ref["U"]) < 2e-4
+    codes = lp.codes.cpu().numpy().astype(np.int64)
+    assert np.mean(codes != ref["codes"]) <= 0.005
+    Q = to_np(lp.Wt)
+    # a dead column is quantized from zero: its dequantised value is the
+    # grid point nearest 0, the same as the oracle's
+    assert np.allclose(Q[:, [3, 130, 257, 383]], ref["Q"][:, [3, 130, 257, 383]], rtol=0, atol=1e-6)
+
+
+def test_dead_columns_end_to_end_su_only():
+    # su_only rotates the output side only, so a zero input channel keeps an
+    # exact zero row and column in H~_X
+    m, n = 192, 256
+    W, X, G = tiny_layer(m=m, n=n, T=2048, seed=22)
+    X[:, [0, 77, 255]] = 0.0
+    lp, What = _gpu_pass(torch.from_numpy(X).to(DEV), torch.from_numpy(G).to(DEV),
+                         torch.from_numpy(W).to(DEV), 4, 64, mode="su_only", seed=3)
+    ref = pipeline.quantize_layer(X, G, W, bits=4, group=64, seed=3, mode="su_only", block=128)
+    assert int(lp.info.item()) == 0
+    assert np.array_equal(np.nonzero(ref["dead"])[0], [0, 77, 255])
+    dis = np.mean(lp.codes.cpu().numpy().astype(np.int64) != ref["codes"])
+    assert dis <= 0.005, dis
+    gl = loss.kfac_loss(W.astype(np.float64) - to_np(What), ref["HX"], ref["HG"])
+    assert abs(gl - ref["loss"]) / ref["loss"] < 0.01, (gl, ref["loss"])
 
 
 # ------------------------------------------------------------------ end to end
