@@ -1,22 +1,29 @@
 """Benchmark of KronQ's per-layer quantization pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kronq|reference]
-                    [--bits 2|3|4] [--group 128] [--no-e2e] [--no-cpu-baseline]
+                    [--workload llama3_70b_mlp|llama2_7b_q_proj] [--bits 2|3|4]
+                    [--no-e2e] [--no-cpu-baseline] [--no-also]
 
-Workload: a Llama-2-7B q_proj-shaped layer, W 4096 x 4096 bf16 ~ N(0, 0.02^2),
-X and G 131072 x 4096 bf16 (X Student-t(4) with lognormal per-channel scale,
-G N(0, 1e-4) with lognormal per-channel scale), 2-bit group-128 asymmetric
-(the pages' headline bit width), BiIP "full", alpha 0.25, damping 0.01.
+Default workload: the two layer shapes of a Llama-3-70B MLP block,
+gate_proj W 28672 x 8192 and down_proj W 8192 x 28672, bf16 ~ N(0, 0.015^2),
+each with its own X and G of 262144 tokens (128 sequences x 2048) bf16 (X
+Student-t(4) with lognormal per-channel scale, |t| for the down_proj input;
+G N(0, 1e-4) with lognormal per-channel scale), the factors accumulated in
+16 chunks of 16384 tokens; 2-bit group-128 asymmetric (the pages' headline
+2-bit Llama-3-70B), BiIP "full", alpha 0.25, damping 0.01.  Beside it (key
+"also"): a Llama-2-7B q_proj-shaped layer (4096 x 4096, T = 131072) at W2
+and W4.
 
-One step = the whole pass on inputs resident in HBM: H_X and H_G
-accumulation, trace sensitivity, BiIP forward, damping + Cholesky factor of
-the damped inverse + GPTQ sweep, int2 packing.  Metric: weights quantized
-per second (m n / seconds per layer, factor accumulation included).  Each
-step is timed with CUDA events on the launching stream; L2 is flushed by a
-256 MB write between steps (outside the timed interval).
+One step = the whole pass over every layer of the workload on inputs
+resident in HBM: H_X and H_G accumulation, trace sensitivity, BiIP forward,
+damping + Cholesky factor of the damped inverse + GPTQ sweep, int2/int4
+packing.  Metric: weights quantized per second (sum of m n over the step's
+layers / seconds per step, factor accumulation included).  Each phase is
+timed with CUDA events on the launching stream; L2 is flushed by a 256 MB
+write between steps (outside the timed interval).
 
-Under torchrun (N > 1) every rank quantizes its own layer (weak scaling, no
-data-path collective); the time is the max over ranks.
+Under torchrun (N > 1) every rank quantizes its own copy of the workload
+(weak scaling, no data-path collective); the time is the max over ranks.
 
 ``--impl reference`` times the CPU float64 oracle on this machine's host cores on
 a bounded sample of the same workload and reports the same metric
@@ -26,7 +33,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -40,14 +46,25 @@ if ROOT not in sys.path:
 
 METRIC = "weights quantized/sec per layer (incl. H_X/H_G accumulation); % of roofline"
 UNIT = "weights/s"
-M = N_IN = 4096
-TOKENS = 131072
-# dram__bytes_read.sum / dram__bytes_write.sum of one syrk_bf16_tc_kernel launch
-# at T = 16384, d = 4096 (ncu, B200), used for roofline.traffic
-SYRK_READ_BYTES_T16384 = 225.659136e6
-E2E_CHUNK = 16384   # tokens per host->device copy chunk in the end-to-end pass
-SYRK_WRITE_BYTES_D4096 = 41.663232e6
-WORKLOAD = "llama2-7b q_proj 4096x4096, T=131072 tokens, W{bits} g{group} asym, BiIP full"
+
+# name -> description, tokens, chunk (None: one call), bits, group, w_std,
+# layers [(sublayer, m, n, rectified X)]
+WORKLOADS = {
+    "llama3_70b_mlp": dict(
+        desc="llama3-70b MLP gate_proj 28672x8192 + down_proj 8192x28672, T=262144 tokens "
+             "(16 chunks of 16384), W{bits} g{group} asym, BiIP full",
+        tokens=262144, chunk=16384, bits=2, group=128, w_std=0.015,
+        layers=[("gate_proj", 28672, 8192, False), ("down_proj", 8192, 28672, True)]),
+    "llama2_7b_q_proj": dict(
+        desc="llama2-7b q_proj 4096x4096, T=131072 tokens, W{bits} g{group} asym, BiIP full",
+        tokens=131072, chunk=None, bits=2, group=128, w_std=0.02,
+        layers=[("q_proj", 4096, 4096, False)]),
+}
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one syrk_bf16_tc_kernel
+# launch (ncu, B200), keyed by (d, tokens per launch); None until the
+# current kernel has been captured at that shape.
+SYRK_TRAFFIC = {}
 
 
 def _peaks():
@@ -57,37 +74,64 @@ def _peaks():
         return None
 
 
-def phase_rooflines(phases_ms, m: int, n: int, T: int, peaks):
-    """Each timed phase's algorithmic work over the measured peak of its bound.
+def choose_peak(peaks, clocks):
+    """The bf16 tensor peak that applies to kernels timed inside this run:
+    the burst figure, unless the clocks sampled during the timed region show
+    the power cap (sw_power_cap, or a median SM clock below 93 % of the
+    maximum), when the sustained figure applies."""
+    if not peaks:
+        return 1590.0, 6650.0, "fallback (burst)"
+    capped = False
+    if clocks:
+        if "sw_power_cap" in (clocks.get("reasons") or []):
+            capped = True
+        sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+        if sm and mx and sm < 0.93 * mx:
+            capped = True
+    if capped:
+        return peaks["bf16_tflops_sustained"], peaks["hbm_gbs"], "measured sustained (power-capped clocks)"
+    return peaks["bf16_tflops"], peaks["hbm_gbs"], "measured burst (clocks not capped)"
 
-    accumulate_HX_HG  tensor: T n (n+1) + T m (m+1) flop (the distinct entries
-                      of the two SYRKs)
+
+def phase_work(layers, T: int):
+    """Algorithmic work of each timed phase summed over the layers (m, n):
+
+    accumulate_HX_HG  tensor: T n (n+1) + T m (m+1) flop (the distinct
+                      entries of the two SYRKs)
     sensitivity       HBM: the two diagonals, 4 (n + m) bytes
     biip_forward      HBM: 16 m n + 16 n^2 + 16 m^2 bytes (W's norms read
                       2 m n; its two passes read 2 + 4 and write 4 + 4 bytes
                       per element; each factor takes two fp32 passes in and out)
-    quantize_and_pack bound by its sequential chains (64 diagonal steps of
+    quantize_and_pack bound by its sequential chains (the diagonal steps of
                       the factorisation, n column steps of the sweep); shown
                       against the tensor peak with 2 n^3 / 3 + m n^2 flop (the
                       reverse Cholesky factor and its triangular inverse, and
                       the error feedback of the sweep)
     """
-    if peaks:
-        tpk, hpk, src = peaks["bf16_tflops_sustained"], peaks["hbm_gbs"], "measured"
-    else:
-        tpk, hpk, src = 1400.0, 6650.0, "fallback"
-    work = {
-        "accumulate_HX_HG": ("tensor", T * n * (n + 1) + T * m * (m + 1), "TFLOP/s", tpk, 1e12),
-        "sensitivity": ("hbm", 4 * (n + m), "GB/s", hpk, 1e9),
-        "biip_forward": ("hbm", 16 * m * n + 16 * n * n + 16 * m * m, "GB/s", hpk, 1e9),
-        "quantize_and_pack": ("latency (sequential chains)", 2 * n ** 3 / 3 + m * n * n, "TFLOP/s", tpk, 1e12),
+    w = {"accumulate_HX_HG": 0, "sensitivity": 0, "biip_forward": 0, "quantize_and_pack": 0}
+    for m, n in layers:
+        w["accumulate_HX_HG"] += T * n * (n + 1) + T * m * (m + 1)
+        w["sensitivity"] += 4 * (n + m)
+        w["biip_forward"] += 16 * m * n + 16 * n * n + 16 * m * m
+        w["quantize_and_pack"] += 2 * n ** 3 / 3 + m * n * n
+    return w
+
+
+def phase_rooflines(phases_ms, layers, T: int, tpk: float, hpk: float, src: str):
+    """Each timed phase's algorithmic work over the peak of its bound."""
+    kinds = {
+        "accumulate_HX_HG": ("tensor", "TFLOP/s", tpk, 1e12),
+        "sensitivity": ("hbm", "GB/s", hpk, 1e9),
+        "biip_forward": ("hbm", "GB/s", hpk, 1e9),
+        "quantize_and_pack": ("latency (sequential chains)", "TFLOP/s", tpk, 1e12),
     }
+    work = phase_work(layers, T)
     out = {}
     for name, ms in phases_ms.items():
-        if name not in work or ms <= 0:
+        if name not in kinds or ms <= 0:
             continue
-        bound, units, unit, peak, scale = work[name]
-        achieved = units / (ms / 1e3) / scale
+        bound, unit, peak, scale = kinds[name]
+        achieved = work[name] / (ms / 1e3) / scale
         out[name] = {"bound": bound, "achieved": achieved, "unit": unit, "peak": peak,
                      "frac": achieved / peak, "peak_source": src}
     return out
@@ -152,53 +196,91 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- CPU oracle sample
-def cpu_oracle_sample(bits: int, group: int, seed: int = 0, t_sample: int = 4096, rows: int = 64):
-    """Time the float64 oracle on a bounded sample of the workload and
-    extrapolate to one full layer by exact operation counts.
+def cpu_oracle_sample(wl: dict, bits: int, group: int, seed: int = 0, t_s: int = 1024,
+                      d_s: int = 2048, rows_s: int = 64, sweep_rows: int = 16):
+    """Time the float64 oracle on a bounded sample of every layer of the
+    workload and extrapolate to the full layers by exact operation counts.
 
-    Sample: factor accumulation over t_sample tokens of X (scaled by
-    2 * TOKENS / t_sample for H_X and H_G), the full BiIP of W and H_X
-    (scaled by 3/2 for H_G), the full inverse + Cholesky of the damped
-    H~_X, the non-lazy sweep of ``rows`` rows (scaled by M / rows), and the
-    packing of those rows (scaled likewise)."""
+    Per layer (m, n; T tokens):
+      factors   H = A^T A of t_s tokens x min(d, d_s) channels of X and of
+                G, scaled by (T / t_s) (d / d_s)^2 (cost T d^2)
+      BiIP      the oracle's row rotation of rows_s rows of each length, scaled
+                by the rows of the two-sided transforms of W (m rows of n,
+                n of m), H_X (2 n of n) and H_G (2 m of m)
+      factor U  dead columns, damping, inverse and Cholesky at min(n, d_s),
+                scaled by (n / n_s)^3
+      sweep     the non-lazy float64 sweep of sweep_rows rows with that U and
+                the packing of their codes, scaled by (m / sweep_rows)(n / n_s)^2
+    """
     import numpy as np
 
     from oracle import biip, factors, pack, sweep
     from synth import llama_layer
 
-    W, X, G = llama_layer(M, N_IN, t_sample, seed=seed, device="cpu")
-    Xn = X.float().numpy()
-    Wn = W.float().numpy().astype(np.float64)
-    t = {}
-    t0 = time.perf_counter()
-    HX = factors.factor(Xn)
-    t["factors"] = (time.perf_counter() - t0) * (2 * TOKENS / t_sample)
-    HG = HX.copy()  # same size; its values do not change the cost of what follows
-    t0 = time.perf_counter()
-    Wt, HXt, _, din, dout = biip.biip_forward(Wn, HX, None, seed, 0.25, "sv_only")
-    Wt = biip.rotate_rows(Wt.T, seed, 1).T
-    t["biip"] = (time.perf_counter() - t0) * 1.5
-    t0 = time.perf_counter()
-    H1, W1, _ = sweep.dead_columns(HXt, Wt)
-    A, _ = sweep.damp(H1, 0.01)
-    U = sweep.chol_upper_of_inverse(A)
-    t["factorisation"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    res = sweep.gptq_sweep(W1[:rows], U, bits, group, True, block=1)
-    if bits in (2, 4):
-        pack.pack(res["codes"], bits)
-    t["sweep"] = (time.perf_counter() - t0) * (M / rows)
+    T = wl["tokens"]
+    t = {"factors": 0.0, "biip": 0.0, "factorisation": 0.0, "sweep": 0.0}
+    weights = 0
+    for li, (_, m, n, rect) in enumerate(wl["layers"]):
+        weights += m * n
+        ns, ms_ = min(n, d_s), min(m, d_s)
+        W, X, G = llama_layer(ms_, ns, t_s, seed=seed + li, device="cpu", w_std=wl["w_std"],
+                              rectified=rect)
+        Xn = X.float().numpy()
+        Gn = G.float().numpy()
+        t0 = time.perf_counter()
+        HX = factors.factor(Xn)
+        t["factors"] += (time.perf_counter() - t0) * (T / t_s) * (n / ns) ** 2
+        t0 = time.perf_counter()
+        factors.factor(Gn)
+        t["factors"] += (time.perf_counter() - t0) * (T / t_s) * (m / ms_) ** 2
+        rng = np.random.default_rng(seed)
+        for L, nrows in ((n, m + 2 * n), (m, n + 2 * m)):
+            R = rng.standard_normal((rows_s, L))
+            t0 = time.perf_counter()
+            biip.rotate_rows(R, seed, 0)
+            t["biip"] += (time.perf_counter() - t0) * (nrows / rows_s)
+        Wn = W.float().numpy().astype(np.float64)
+        Wt = biip.rotate_rows(Wn, seed, 0)
+        HXt = biip.rotate_rows(biip.rotate_rows(HX, seed, 0).T, seed, 0).T
+        t0 = time.perf_counter()
+        H1, W1, _ = sweep.dead_columns(HXt, Wt)
+        A, _ = sweep.damp(H1, 0.01)
+        U = sweep.chol_upper_of_inverse(A)
+        t["factorisation"] += (time.perf_counter() - t0) * (n / ns) ** 3
+        t0 = time.perf_counter()
+        res = sweep.gptq_sweep(W1[:sweep_rows], U, bits, group, True, block=1)
+        if bits in (2, 4):
+            pack.pack(res["codes"], bits)
+        t["sweep"] += (time.perf_counter() - t0) * (m / sweep_rows) * (n / ns) ** 2
     total = sum(t.values())
     try:
         cores = len(os.sched_getaffinity(0))
     except AttributeError:
         cores = os.cpu_count()
-    sample = (f"oracle (numpy float64) on {t_sample} tokens for the factors, full BiIP and "
-              f"factorisation, {rows} rows for the sweep; extrapolated to the full layer by "
-              f"operation counts")
-    return {"value": M * N_IN / total, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": sample, "seconds_per_layer": total,
+    sample = (f"oracle (numpy float64) per layer: factors of {t_s} tokens x {d_s} channels, row "
+              f"rotations of {rows_s} rows, U at n = {d_s}, sweep of {sweep_rows} rows at n = {d_s}; "
+              f"extrapolated to the full layers by operation counts")
+    return {"value": weights / total, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": sample, "seconds_per_step": total,
             "phases_s": {k: round(v, 3) for k, v in t.items()}}
+
+
+def _workload(args):
+    wl = dict(WORKLOADS[args.workload])
+    if args.bits is not None:
+        wl["bits"] = args.bits
+    if args.group is not None:
+        wl["group"] = args.group
+    return wl
+
+
+def _config(wl, name, world):
+    return {"workload": wl["desc"].format(bits=wl["bits"], group=wl["group"]), "name": name,
+            "layers": [{"sublayer": s, "m": m, "n": n} for s, m, n, _ in wl["layers"]],
+            "tokens": wl["tokens"], "chunk": wl["chunk"], "bits": wl["bits"], "group": wl["group"],
+            "accumulate": "f32",
+            "l2": "flushed between steps (256 MB write, outside the timed interval); inputs larger than L2",
+            "parallelism": f"dp{world} (each rank its own copy of the workload)"}
 
 
 # ----------------------------------------------------------------- reference arm
@@ -207,21 +289,23 @@ def run_reference(args):
     if rank != 0:
         return 0
     os.environ.setdefault("OMP_NUM_THREADS", str(len(os.sched_getaffinity(0))))
+    wl = _workload(args)
     vals = []
     last = None
     for i in range(args.warmup + args.steps):
-        r = cpu_oracle_sample(args.bits, args.group, seed=i, t_sample=2048, rows=32)
+        r = cpu_oracle_sample(wl, wl["bits"], wl["group"], seed=i, t_s=512, d_s=1024, rows_s=32,
+                              sweep_rows=8)
         if i >= args.warmup:
-            vals.append(r["seconds_per_layer"])
+            vals.append(r["seconds_per_step"])
         last = r
-    spl = statistics.mean(vals)
-    value = M * N_IN / spl
+    sps = statistics.mean(vals)
+    weights = sum(m * n for _, m, n, _ in wl["layers"])
+    value = weights / sps
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": spl * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": sps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD.format(bits=args.bits, group=args.group),
-                       "m": M, "n": N_IN, "tokens": TOKENS, "bits": args.bits, "group": args.group},
+            "config": _config(wl, args.workload, 1),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
                              "sample": last["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -230,12 +314,82 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------- GPU arm
+def _make_layers(wl, dev, rank):
+    from post_quantization_kronq_b200.layer import LayerPass
+    from synth import llama_layer
+
+    out = []
+    for li, (name, m, n, rect) in enumerate(wl["layers"]):
+        W, X, G = llama_layer(m, n, wl["tokens"], seed=1000 + 10 * rank + li, device=dev,
+                              w_std=wl["w_std"], rectified=rect)
+        lp = LayerPass(m, n, bits=wl["bits"], group=wl["group"], seed=rank + li, device=dev)
+        out.append((name, W, X, G, lp))
+    return out
+
+
+def _time_steps(layers, chunk, steps, warmup, stream, flush, sampler=None, barrier=None):
+    """Runs warmup + steps passes over all layers; returns per-step phase
+    times (ms) summed over the layers, and the launches in the timed steps."""
+    import torch
+
+    import post_quantization_kronq_b200 as kq
+
+    names = ["accumulate_HX_HG", "sensitivity", "biip_forward", "quantize_and_pack"]
+
+    def step(recs=None):
+        for li, (_, W, X, G, lp) in enumerate(layers):
+            r = recs[li] if recs else None
+            if r:
+                r[0].record(stream)
+            lp.accumulate(X, G, chunk=chunk)
+            if r:
+                r[1].record(stream)
+            lp.sensitivity()
+            if r:
+                r[2].record(stream)
+            lp.transform(W)
+            if r:
+                r[3].record(stream)
+            lp.quantize()
+            if r:
+                r[4].record(stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    for _, _, _, _, lp in layers:
+        assert int(lp.info.item()) == 0, "factorisation reported a non-positive pivot"
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    recs = [[[ev() for _ in range(5)] for _ in layers] for _ in range(steps)]
+    if sampler:
+        sampler.start()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    l0 = kq.kronq_launch_count()
+    for k in range(steps):
+        flush.zero_()
+        step(recs[k])
+    torch.cuda.synchronize()
+    launches = kq.kronq_launch_count() - l0
+    if barrier:
+        barrier()
+    clocks = sampler.stop() if sampler else None
+    per_step = []
+    for k in range(steps):
+        ph = {nm: 0.0 for nm in names}
+        for r in recs[k]:
+            for i, nm in enumerate(names):
+                ph[nm] += r[i].elapsed_time(r[i + 1])
+        per_step.append(ph)
+    return per_step, launches, clocks
+
+
 def run_kronq(args):
     import torch
 
     import post_quantization_kronq_b200 as kq
-    from post_quantization_kronq_b200.layer import LayerPass
-    from synth import llama_layer
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -255,113 +409,84 @@ def run_kronq(args):
             dist.barrier()
 
     stream = torch.cuda.current_stream()
-    bits, group = args.bits, args.group
-    W, X, G = llama_layer(M, N_IN, TOKENS, seed=1000 + rank, device=dev)
-    lp = LayerPass(M, N_IN, bits=bits, group=group, seed=rank, device=dev)
+    wl = _workload(args)
+    T, chunk = wl["tokens"], wl["chunk"]
+    layers = _make_layers(wl, dev, rank)
+    shapes = [(m, n) for _, m, n, _ in wl["layers"]]
+    weights = sum(m * n for m, n in shapes)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-
-    def step(rec=None):
-        if rec is not None:
-            rec[0].record(stream)
-        lp.accumulate(X, G)
-        if rec is not None:
-            rec[1].record(stream)
-        lp.sensitivity()
-        if rec is not None:
-            rec[2].record(stream)
-        lp.transform(W)
-        if rec is not None:
-            rec[3].record(stream)
-        lp.quantize()
-        if rec is not None:
-            rec[4].record(stream)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    assert int(lp.info.item()) == 0, "factorisation reported a non-positive pivot"
-
-    recs = [[ev() for _ in range(5)] for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    sampler.start()
-    barrier()
-    torch.cuda.synchronize()
-    launches0 = kq.kronq_launch_count()
-    for k in range(args.steps):
-        flush.zero_()
-        torch.cuda.nvtx.range_push("kronq_timed_step")
-        step(recs[k])
-        torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
-    launches = kq.kronq_launch_count() - launches0
-    barrier()
-    clocks = sampler.stop()
-    step_ms = [r[0].elapsed_time(r[4]) for r in recs]
-    acc_ms = [r[0].elapsed_time(r[1]) for r in recs]
-    phases = {
-        "accumulate_HX_HG": statistics.mean(acc_ms),
-        "sensitivity": statistics.mean(r[1].elapsed_time(r[2]) for r in recs),
-        "biip_forward": statistics.mean(r[2].elapsed_time(r[3]) for r in recs),
-        "quantize_and_pack": statistics.mean(r[3].elapsed_time(r[4]) for r in recs),
-    }
+    per_step, launches, clocks = _time_steps(layers, chunk, args.steps, args.warmup, stream, flush,
+                                             ClockSampler(local), barrier)
+    step_ms = [sum(p.values()) for p in per_step]
     total_ms = sum(step_ms)
     if dist is not None:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-    value = world * M * N_IN * args.steps / (total_ms / 1e3)
+    value = world * weights * args.steps / (total_ms / 1e3)
+    phases = {nm: statistics.mean(p[nm] for p in per_step) for nm in per_step[0]}
 
-    # Roofline of the dominant kernel: the tcgen05 SYRK (two launches per step,
-    # one per factor, both d = 4096).  Algorithmic flops per launch: T d (d + 1).
-    syrk_launch_ms = statistics.mean(acc_ms) / 2.0
-    flops = TOKENS * N_IN * (N_IN + 1)
-    achieved = flops / (syrk_launch_ms / 1e3) / 1e12
     peaks = _peaks()
+    tpk, hpk, src = choose_peak(peaks, clocks)
+    # Roofline of the dominant kernel: the tcgen05 SYRK.  The accumulation
+    # phase is SYRK launches only (two factors per layer, one launch per
+    # token chunk); algorithmic flops T d (d + 1) per factor.
+    acc_ms = phases["accumulate_HX_HG"]
+    flops = sum(T * n * (n + 1) + T * m * (m + 1) for m, n in shapes)
+    per_layer_launches = 2 * (1 if chunk is None else -(-T // chunk))
+    nl = per_layer_launches * len(shapes)
+    achieved = flops / (acc_ms / 1e3) / 1e12
+    traffic = None
+    tkeys = []
+    for m, n in shapes:
+        for d in (n, m):
+            tkeys.append((d, T if chunk is None else chunk))
+    if all(k in SYRK_TRAFFIC for k in tkeys):
+        traffic = sum(SYRK_TRAFFIC[k] for k in tkeys) / len(tkeys)
+    roofline = {"bound": "tensor", "kernel": "syrk_bf16_tc_kernel", "achieved": achieved, "peak": tpk,
+                "unit": "TFLOP/s", "frac": achieved / tpk, "traffic": traffic,
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean per launch "
+                                  "over the step's launch shapes" if traffic else None,
+                "peak_source": src, "launches_per_step": nl,
+                "flops_per_launch_mean": flops / nl, "launch_ms_mean": acc_ms / nl}
     if peaks:
-        peak, peak_src = peaks["bf16_tflops_sustained"], "measured (sustained bf16, MEASURED_PEAKS.json)"
-    else:
-        peak, peak_src = 1400.0, "fallback (sustained)"
-    # DRAM traffic per launch, from one ncu capture of the same kernel at
-    # T = 16384, d = 4096 (dram__bytes_read.sum 225.66 MB, dram__bytes_write.sum
-    # 41.66 MB): the token reads grow in proportion to T, the H write does not.
-    traffic = SYRK_READ_BYTES_T16384 * (TOKENS / 16384) + SYRK_WRITE_BYTES_D4096
-    roofline = {"bound": "tensor", "kernel": "syrk_bf16_tc_kernel", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "traffic_source": "ncu capture at T=16384 (d=4096), reads scaled by T/16384",
-                "peak_source": peak_src,
-                "flops_per_launch": flops, "launch_ms": syrk_launch_ms}
+        roofline["frac_of_burst"] = achieved / peaks["bf16_tflops"]
+        roofline["frac_of_sustained"] = achieved / peaks["bf16_tflops_sustained"]
 
     # End to end through the public API: inputs copied from pinned host memory
     # every step, packed codes, scales and zeros copied back.
     e2e = None
     if not args.no_e2e:
-        hX = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
-        hG = torch.empty(G.shape, dtype=G.dtype, pin_memory=True)
-        hW = torch.empty(W.shape, dtype=W.dtype, pin_memory=True)
-        hX.copy_(X)
-        hG.copy_(G)
-        hW.copy_(W)
-        outs = [lp.packed if lp.packed is not None else lp.codes, lp.scales, lp.zeros]
-        houts = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-        h2d = sum(t.numel() * t.element_size() for t in (hX, hG, hW))
-        d2h = sum(t.numel() * t.element_size() for t in houts)
+        host = []
+        h2d = d2h = 0
+        for _, W, X, G, lp in layers:
+            hX = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
+            hG = torch.empty(G.shape, dtype=G.dtype, pin_memory=True)
+            hW = torch.empty(W.shape, dtype=W.dtype, pin_memory=True)
+            hX.copy_(X)
+            hG.copy_(G)
+            hW.copy_(W)
+            outs = [lp.packed if lp.packed is not None else lp.codes, lp.scales, lp.zeros]
+            houts = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+            h2d += sum(t.numel() * t.element_size() for t in (hX, hG, hW))
+            d2h += sum(t.numel() * t.element_size() for t in houts)
+            host.append((hX, hG, hW, outs, houts))
 
         def e2e_step():
-            # token chunks of X and G copied on a second stream while the
-            # factor accumulation of the earlier chunks runs
-            lp.run_from_host(hX, hG, hW, X, G, W, chunk=E2E_CHUNK, stream=stream)
-            for h, o in zip(houts, outs):
-                h.copy_(o, non_blocking=True)
+            # token chunks of X and G copied on each layer's copy stream while
+            # the factor accumulation of the earlier chunks runs
+            for (_, W, X, G, lp), (hX, hG, hW, outs, houts) in zip(layers, host):
+                lp.run_from_host(hX, hG, hW, X, G, W, chunk=chunk or 16384, stream=stream)
+                for h, o in zip(houts, outs):
+                    h.copy_(o, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
         e_steps = max(2, min(args.steps, 5))
         barrier()
         torch.cuda.synchronize()
-        e0, e1 = ev(), ev()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(e_steps):
             e2e_step()
@@ -372,14 +497,44 @@ def run_kronq(args):
             t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
-        e2e = {"value": world * M * N_IN * e_steps / (e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": world * weights * e_steps / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
-               "pipeline": f"X, G copied in {E2E_CHUNK}-token chunks on a second stream, "
-                           "overlapping the factor accumulation and the previous step's sweep"}
+               "pipeline": "X, G copied in 16384-token chunks on a second stream per layer, "
+                           "overlapping the factor accumulation and the other layers' passes"}
+        del host
+
+    sens = [lp.sens for _, _, _, _, lp in layers]
+    del layers
+    torch.cuda.empty_cache()
+
+    also = None
+    if not args.no_also and args.workload != "llama2_7b_q_proj":
+        also = {}
+        for b in (2, 4):
+            wq = dict(WORKLOADS["llama2_7b_q_proj"])
+            wq["bits"] = b
+            lq = _make_layers(wq, dev, rank)
+            ps, ln, _ = _time_steps(lq, wq["chunk"], args.steps, args.warmup, stream, flush)
+            tms = sum(sum(p.values()) for p in ps)
+            if dist is not None:
+                t = torch.tensor([tms], dtype=torch.float64, device=dev)
+                dist.all_reduce(t, op=dist.ReduceOp.MAX)
+                tms = float(t.item())
+            ph = {nm: statistics.mean(p[nm] for p in ps) for nm in ps[0]}
+            fl = wq["tokens"] * 4096 * 4097 * 2
+            also[f"llama2_7b_q_proj_w{b}"] = {
+                "workload": wq["desc"].format(bits=b, group=wq["group"]),
+                "value": world * 4096 * 4096 * args.steps / (tms / 1e3), "unit": UNIT,
+                "ms_per_step": tms / args.steps, "gpu_launches": ln,
+                "phases_ms": {k: round(v, 4) for k, v in ph.items()},
+                "syrk_tflops": fl / (ph["accumulate_HX_HG"] / 1e3) / 1e12,
+                "phase_roofline": phase_rooflines(ph, [(4096, 4096)], wq["tokens"], tpk, hpk, src)}
+            del lq
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        c = cpu_oracle_sample(bits, group)
+        c = cpu_oracle_sample(wl, wl["bits"], wl["group"])
         cpu = {k: c[k] for k in ("value", "unit", "cores", "kind", "sample")}
         cpu["phases_s"] = c["phases_s"]
 
@@ -392,15 +547,12 @@ def run_kronq(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD.format(bits=bits, group=group), "m": M, "n": N_IN,
-                   "tokens": TOKENS, "bits": bits, "group": group, "accumulate": "f32",
-                   "l2": "flushed between steps (256 MB write, outside the timed interval)",
-                   "parallelism": f"dp{world} (one layer per GPU)"},
+        "config": _config(wl, args.workload, world),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": launches,
         "phases_ms": {k: round(v, 4) for k, v in phases.items()},
-        "phase_roofline": phase_rooflines(phases, M, N_IN, TOKENS, peaks),
-        "sensitivity": list(lp.sens) if lp.sens else None,
+        "phase_roofline": phase_rooflines(phases, shapes, T, tpk, hpk, src),
+        "sensitivity": sens, "also": also,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -412,10 +564,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kronq", "reference"], default="kronq")
-    ap.add_argument("--bits", type=int, default=2, choices=[2, 3, 4])
-    ap.add_argument("--group", type=int, default=128)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama3_70b_mlp")
+    ap.add_argument("--bits", type=int, default=None, choices=[2, 3, 4])
+    ap.add_argument("--group", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-also", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
