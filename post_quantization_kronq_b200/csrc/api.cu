@@ -89,6 +89,7 @@ size_t biip_ws(int64_t m, int64_t n) {
   c.take<float>((size_t)n);
   c.take<float>((size_t)m);
   c.take<float>(wnorms_partial_floats(m, n));
+  c.take<float>((size_t)(m > n ? m : n));   // column factors of one row pass
   return c.size();
 }
 
@@ -175,6 +176,35 @@ kronq_status kronq_sensitivity(const float* HX, int64_t n, const float* HG, int6
   if (r != KRONQ_OK) return r;
   double h[2];
   KQ_CUDA(cudaMemcpyAsync(h, dev2, sizeof(h), cudaMemcpyDeviceToHost, st));
+  KQ_CUDA(cudaStreamSynchronize(st));
+  out3[0] = h[0];
+  out3[1] = h[1];
+  out3[2] = h[1] * h[0];
+  return KRONQ_OK;
+}
+
+size_t kronq_trace_tokens_workspace_bytes(void) {
+  return ((token_sqsum_partials() * sizeof(double)) + 255) & ~size_t(255);
+}
+
+kronq_status kronq_trace_tokens(const void* A, kronq_dtype dt, int64_t T, int64_t d, int64_t lda,
+                                double* trace, int zero_first, void* workspace, size_t ws_bytes,
+                                kronq_stream_t s) {
+  if (dt != KRONQ_BF16 && dt != KRONQ_F32) return fail(KRONQ_ERR_INVALID_ARG, "trace_tokens: bad dtype");
+  if (d <= 0 || T < 0 || lda < d) return fail(KRONQ_ERR_INVALID_ARG, "trace_tokens: need d > 0, T >= 0, lda >= d");
+  if (!trace || (T > 0 && !A)) return fail(KRONQ_ERR_INVALID_ARG, "trace_tokens: NULL pointer");
+  if (!aligned(trace, 8)) return fail(KRONQ_ERR_INVALID_ARG, "trace_tokens: trace must be 8-byte aligned");
+  if (!workspace || ws_bytes < kronq_trace_tokens_workspace_bytes() || !aligned(workspace, 256))
+    return fail(KRONQ_ERR_INVALID_ARG, "trace_tokens: workspace too small or not 256-byte aligned");
+  return token_sqsum(A, dt == KRONQ_BF16, T, d, lda, trace, zero_first, static_cast<double*>(workspace),
+                     as_stream(s));
+}
+
+kronq_status kronq_sensitivity_from_traces(const double* traces, double* out3, kronq_stream_t s) {
+  if (!traces || !out3) return fail(KRONQ_ERR_INVALID_ARG, "sensitivity_from_traces: NULL pointer");
+  cudaStream_t st = as_stream(s);
+  double h[2];
+  KQ_CUDA(cudaMemcpyAsync(h, traces, sizeof(h), cudaMemcpyDeviceToHost, st));
   KQ_CUDA(cudaStreamSynchronize(st));
   out3[0] = h[0];
   out3[1] = h[1];
@@ -269,6 +299,7 @@ kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64
   float* colsq = c.take<float>((size_t)n);
   float* rowsq = c.take<float>((size_t)m);
   float* part = c.take<float>(wnorms_partial_floats(m, n));
+  float* cfbuf = c.take<float>((size_t)(m > n ? m : n));
   const bool bf16 = wdt == KRONQ_BF16;
   kronq_status r;
   const bool need_in = rescale && use_in, need_out = rescale && use_out;
@@ -290,20 +321,20 @@ kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64
   p1.out = T; p1.ld_out = m;
   p1.rows = m; p1.L = n;
   p1.scale = d_in; p1.scale_mode = need_in ? 1 : 0;
-  p1.rotate = use_in; p1.inverse = false; p1.sign_state = s_in;
+  p1.rotate = use_in; p1.inverse = false; p1.sign_state = s_in; p1.cf = cfbuf;
   if ((r = rowpass(p1, st)) != KRONQ_OK) return r;
   RowPass p2;
   p2.in = T; p2.ld_in = m;
   p2.out = Wt; p2.ld_out = n;
   p2.rows = n; p2.L = m;
   p2.scale = d_out; p2.scale_mode = need_out ? 1 : 0;
-  p2.rotate = use_out; p2.inverse = false; p2.sign_state = s_out;
+  p2.rotate = use_out; p2.inverse = false; p2.sign_state = s_out; p2.cf = cfbuf;
   if ((r = rowpass(p2, st)) != KRONQ_OK) return r;
   // H~_X = V D_in^-1 H_X D_in^-1 V^T
   if (use_in) {
     RowPass h1;
     h1.in = HX; h1.ld_in = n; h1.out = T; h1.ld_out = n; h1.rows = n; h1.L = n;
-    h1.scale = d_in; h1.scale_mode = need_in ? 2 : 0; h1.rotate = true; h1.sign_state = s_in;
+    h1.scale = d_in; h1.scale_mode = need_in ? 2 : 0; h1.rotate = true; h1.sign_state = s_in; h1.cf = cfbuf;
     if ((r = rowpass(h1, st)) != KRONQ_OK) return r;
     RowPass h2 = h1;
     h2.in = T; h2.out = HX;
@@ -313,7 +344,7 @@ kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64
   if (use_out && HG) {
     RowPass g1;
     g1.in = HG; g1.ld_in = m; g1.out = T; g1.ld_out = m; g1.rows = m; g1.L = m;
-    g1.scale = d_out; g1.scale_mode = need_out ? 2 : 0; g1.rotate = true; g1.sign_state = s_out;
+    g1.scale = d_out; g1.scale_mode = need_out ? 2 : 0; g1.rotate = true; g1.sign_state = s_out; g1.cf = cfbuf;
     if ((r = rowpass(g1, st)) != KRONQ_OK) return r;
     RowPass g2 = g1;
     g2.in = T; g2.out = HG;
@@ -336,17 +367,24 @@ kronq_status kronq_biip_inverse(float* W, int64_t m, int64_t n, uint64_t seed, k
     return fail(KRONQ_ERR_INVALID_ARG, "biip_inverse: workspace too small or not 256-byte aligned");
   cudaStream_t st = as_stream(s);
   Carver c(workspace);
-  float* T = c.take<float>((size_t)(m * n));
+  int64_t big = m * n;
+  if (n * n > big) big = n * n;
+  if (m * m > big) big = m * m;
+  float* T = c.take<float>((size_t)big);
+  c.take<float>((size_t)n);
+  c.take<float>((size_t)m);
+  c.take<float>(wnorms_partial_floats(m, n));
+  float* cfbuf = c.take<float>((size_t)(m > n ? m : n));
   kronq_status r;
   RowPass p1;
   p1.in = W; p1.ld_in = n; p1.out = T; p1.ld_out = m; p1.rows = m; p1.L = n;
   p1.scale = d_in; p1.scale_mode = 2; p1.rotate = use_in; p1.inverse = true;
-  p1.sign_state = 2ull * seed;
+  p1.sign_state = 2ull * seed; p1.cf = cfbuf;
   if ((r = rowpass(p1, st)) != KRONQ_OK) return r;
   RowPass p2;
   p2.in = T; p2.ld_in = m; p2.out = W; p2.ld_out = n; p2.rows = n; p2.L = m;
   p2.scale = d_out; p2.scale_mode = 2; p2.rotate = use_out; p2.inverse = true;
-  p2.sign_state = 2ull * seed + 1ull;
+  p2.sign_state = 2ull * seed + 1ull; p2.cf = cfbuf;
   return rowpass(p2, st);
 }
 
@@ -360,24 +398,45 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
                                   const kronq_quant_params* p, uint8_t* codes, float* scales,
                                   float* zeros, float* E, int* info, void* workspace,
                                   size_t ws_bytes, kronq_stream_t s) {
-  if (!p) return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: params is NULL");
-  if (!Wt || !HX || !codes || !scales || !zeros || !info || m <= 0 || n <= 0)
-    return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: NULL pointer or non-positive size");
-  if (p->bits < 2 || p->bits > 4) return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: bits must be 2, 3 or 4");
-  if (p->asym != 0 && p->asym != 1) return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: asym must be 0 or 1");
-  if (p->block != 128) return fail(KRONQ_ERR_UNSUPPORTED, "quantize_layer: only block = 128 is implemented");
-  if (!(p->group == -1 || (p->group > 0 && (128 % p->group == 0 || p->group % 128 == 0))))
-    return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: group must be -1, a divisor of 128 or a multiple of 128");
-  if (!(p->damp_rel >= 0.f) || !isfinite(p->damp_rel))
-    return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: damp_rel must be finite and >= 0");
-  if (p->flags & ~(KRONQ_U_GIVEN | KRONQ_ORDERED_FP32 | KRONQ_WRITE_E))
-    return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: unknown flag");
-  if ((p->flags & KRONQ_WRITE_E) && !E) return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: KRONQ_WRITE_E needs E");
-  if (m > ((int64_t)1 << 31) / 16 || n > ((int64_t)1 << 20))
-    return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: size out of range");
+  kronq_status v = check_quant_args(Wt, HX, m, n, p, codes, scales, zeros, E, info, "quantize_layer");
+  if (v != KRONQ_OK) return v;
   if (!workspace || ws_bytes < quant_ws(m, n) || !aligned(workspace, 256))
     return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: workspace too small or not 256-byte aligned");
-  cudaStream_t st = as_stream(s);
+  const int mode = (p->flags & KRONQ_U_GIVEN) ? 1 : 0;
+  return quantize_core(Wt, HX, m, n, p, codes, scales, zeros, E, info, workspace, as_stream(s), mode);
+}
+
+}  // extern "C"
+
+namespace kq {
+
+kronq_status check_quant_args(float* Wt, float* HX, int64_t m, int64_t n, const kronq_quant_params* p,
+                              uint8_t* codes, float* scales, float* zeros, float* E, int* info,
+                              const char* who) {
+  const std::string w(who);
+  if (!p) return fail(KRONQ_ERR_INVALID_ARG, w + ": params is NULL");
+  if (!Wt || !HX || !codes || !scales || !zeros || !info || m <= 0 || n <= 0)
+    return fail(KRONQ_ERR_INVALID_ARG, w + ": NULL pointer or non-positive size");
+  if (p->bits < 2 || p->bits > 4) return fail(KRONQ_ERR_INVALID_ARG, w + ": bits must be 2, 3 or 4");
+  if (p->asym != 0 && p->asym != 1) return fail(KRONQ_ERR_INVALID_ARG, w + ": asym must be 0 or 1");
+  if (p->block != 128) return fail(KRONQ_ERR_UNSUPPORTED, w + ": only block = 128 is implemented");
+  if (!(p->group == -1 || (p->group > 0 && (128 % p->group == 0 || p->group % 128 == 0))))
+    return fail(KRONQ_ERR_INVALID_ARG, w + ": group must be -1, a divisor of 128 or a multiple of 128");
+  if (!(p->damp_rel >= 0.f) || !isfinite(p->damp_rel))
+    return fail(KRONQ_ERR_INVALID_ARG, w + ": damp_rel must be finite and >= 0");
+  if (p->flags & ~(KRONQ_U_GIVEN | KRONQ_ORDERED_FP32 | KRONQ_WRITE_E))
+    return fail(KRONQ_ERR_INVALID_ARG, w + ": unknown flag");
+  if ((p->flags & KRONQ_WRITE_E) && !E) return fail(KRONQ_ERR_INVALID_ARG, w + ": KRONQ_WRITE_E needs E");
+  if (m > ((int64_t)1 << 31) / 16 || n > ((int64_t)1 << 20))
+    return fail(KRONQ_ERR_INVALID_ARG, w + ": size out of range");
+  return KRONQ_OK;
+}
+
+size_t quantize_core_workspace_bytes(int64_t m, int64_t n) { return quant_ws(m, n); }
+
+kronq_status quantize_core(float* Wt, float* HX, int64_t m, int64_t n, const kronq_quant_params* p,
+                           uint8_t* codes, float* scales, float* zeros, float* E, int* info,
+                           void* workspace, cudaStream_t st, int mode) {
   Carver c(workspace);
   void* cws = c.take<uint8_t>(chol_workspace_bytes(n));
   uint8_t* dead = c.take<uint8_t>((size_t)n);
@@ -387,10 +446,12 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
   __nv_bfloat16* El = c.take<__nv_bfloat16>((size_t)(m * kg));
   __nv_bfloat16* Uh = c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
   __nv_bfloat16* Ul = c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
-  const bool u_given = (p->flags & KRONQ_U_GIVEN) != 0;
+  const bool u_given = mode == 1;
   kronq_status r;
   if (u_given) {
     r = chol_upper_inverse(HX, 0, 0.f, true, nullptr, info, cws, st);  // resets info only
+  } else if (mode == 2) {
+    r = chol_upper_inverse(HX, n, 0.f, true, nullptr, info, cws, st);  // already damped
   } else {
     r = chol_upper_inverse(HX, n, p->damp_rel, false, dead, info, cws, st);
   }
@@ -402,7 +463,7 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
   d.ngroups = (p->group == -1) ? 1 : ceil_div(n, p->group);
   d.E = (p->flags & KRONQ_WRITE_E) ? E : nullptr;
   d.Eblk = Eblk;
-  d.dead = u_given ? nullptr : dead;
+  d.dead = mode == 0 ? dead : nullptr;
   d.info = info;
   d.ordered = (p->flags & KRONQ_ORDERED_FP32) != 0;
   d.Eh = Eh; d.El = El; d.Uh = Uh; d.Ul = Ul; d.ldu = quant_ldu(n);
@@ -410,6 +471,10 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
   d.gblocks = (int)quant_gblocks(n);
   return gptq_sweep(d, st);
 }
+
+}  // namespace kq
+
+extern "C" {
 
 kronq_status kronq_pack(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* out,
                         kronq_stream_t s) {
@@ -429,15 +494,16 @@ kronq_status kronq_unpack(const uint32_t* in, int64_t m, int64_t n, int bits, ui
 
 kronq_status kronq_device_status(int* out, kronq_stream_t s) {
   if (!out) return fail(KRONQ_ERR_INVALID_ARG, "device_status: out is NULL");
-  int v[5] = {0, 0, 0, 0, 0};
+  int v[6] = {0, 0, 0, 0, 0, 0};
   cudaError_t e = status_fetch_syrk(&v[0], as_stream(s));
   if (e == cudaSuccess) e = status_fetch_trailing(&v[1], as_stream(s));
   if (e == cudaSuccess) e = status_fetch_schur(&v[2], as_stream(s));
   if (e == cudaSuccess) e = status_fetch_trigemm(&v[3], as_stream(s));
   if (e == cudaSuccess) e = status_fetch_chol(&v[4], as_stream(s));
+  if (e == cudaSuccess) e = status_fetch_schurk(&v[5], as_stream(s));
   if (e != cudaSuccess) return cuda_fail(e, "device_status");
   *out = 0;
-  for (int i = 0; i < 5 && *out == 0; ++i) *out = v[i];
+  for (int i = 0; i < 6 && *out == 0; ++i) *out = v[i];
   return KRONQ_OK;
 }
 

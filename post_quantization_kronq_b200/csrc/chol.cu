@@ -1081,11 +1081,23 @@ static size_t splits_bytes(int64_t n) {
   return (((size_t)3 * n * NB * sizeof(__nv_bfloat16)) + 255) & ~size_t(255);
 }
 
-size_t chol_workspace_bytes(int64_t n) {
+size_t chol_core_workspace_bytes(int64_t n) {
   // T / staging buffer, two buffers of bf16 hi/mid/lo panel splits
   // (3 x n x 64 each), the step counters of the persistent kernel
   const int64_t nblk = ceil_div(n, NB);
   return tbuf_bytes(n) + 2 * splits_bytes(n) + (size_t)(5 * nblk + 4) * sizeof(int);
+}
+
+size_t chol_workspace_bytes(int64_t n) {
+  return n > kOuterBlock ? chol_blocked_workspace_bytes(n) : chol_core_workspace_bytes(n);
+}
+
+size_t chol_tbuf_bytes(int64_t n) { return tbuf_bytes(n); }
+
+kronq_status damp_factor(float* H, int64_t n, float damp_rel, uint8_t* dead, int* info, cudaStream_t s) {
+  damp_kernel<<<1, 1024, 0, s>>>(H, n, damp_rel, dead, info);
+  KQ_LAUNCH_CHECK("damp_kernel");
+  return KRONQ_OK;
 }
 
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
@@ -1098,6 +1110,11 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
     KQ_LAUNCH_CHECK("zero_info_kernel");
   }
   if (n <= 0) return KRONQ_OK;
+  if (n > kOuterBlock) return chol_blocked(H, n, info, ws, s);
+  return chol_core(H, n, info, ws, s);
+}
+
+kronq_status chol_core(float* H, int64_t n, int* info, void* ws, cudaStream_t s) {
   float* Tbuf = reinterpret_cast<float*>(ws);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   __nv_bfloat16* splits = reinterpret_cast<__nv_bfloat16*>(wsb + tbuf_bytes(n));
@@ -1166,8 +1183,15 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
   }
   diag_store_kernel<<<(unsigned)nblk, 256, 0, s>>>(H, n, Tbuf, info);
   KQ_LAUNCH_CHECK("diag_store_kernel");
-  // Recursive inverse of the off-diagonal blocks.
-  for (int64_t S = NB; S < n; S *= 2) {
+  return chol_inverse_levels(H, n, NB, Tbuf, info, s);
+}
+
+kronq_status chol_inverse_levels(float* H, int64_t n, int64_t S0, float* Tbuf, const int* info,
+                                 cudaStream_t s) {
+  // Recursive inverse of the off-diagonal blocks: the diagonal blocks of
+  // size S0 (aligned from the top, the last one possibly short) hold U_JJ,
+  // the blocks above them R.
+  for (int64_t S = S0; S < n; S *= 2) {
     const int64_t npairs_full = n / (2 * S);  // pairs whose R22 has full size S
     struct Pair { int64_t p0, cnt, s2; };
     Pair groups[2] = {{0, npairs_full, S}, {npairs_full, 0, 0}};

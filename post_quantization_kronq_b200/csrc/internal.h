@@ -103,6 +103,7 @@ struct RowPass {
   bool rotate = true;
   bool inverse = false;
   uint64_t sign_state = 0;  // 2 * seed + side
+  float* cf = nullptr;      // optional scratch of L floats for the column factors
 };
 kronq_status rowpass(const RowPass& p, cudaStream_t s);
 // sum of squares along columns (colsq[n]) and rows (rowsq[m]) of W.
@@ -127,6 +128,21 @@ cudaError_t status_fetch_schur(int* out, cudaStream_t s);
 // In: H (n x n) full symmetric.  Out: U (upper) with U^T U = (H + lambda I)^-1,
 // dead-column flags, info.  ws: see chol_workspace_bytes.
 size_t chol_workspace_bytes(int64_t n);
+// Above this order the factorisation is blocked in two levels (chol_blocked).
+constexpr int64_t kOuterBlock = 4096;
+// The single-level factorisation of a contiguous n x n block (no damping,
+// info untouched unless a pivot fails) and its workspace.
+size_t chol_core_workspace_bytes(int64_t n);
+size_t chol_tbuf_bytes(int64_t n);
+kronq_status chol_core(float* H, int64_t n, int* info, void* ws, cudaStream_t s);
+// U = R^-1 from the diagonal blocks U_JJ of size S0 (aligned from the top)
+// and the off-diagonal blocks of R, level by level (tensor-core products).
+kronq_status chol_inverse_levels(float* H, int64_t n, int64_t S0, float* Tbuf, const int* info,
+                                 cudaStream_t s);
+// Two-level blocked factorisation for n > kOuterBlock (after damping).
+size_t chol_blocked_workspace_bytes(int64_t n);
+kronq_status chol_blocked(float* H, int64_t n, int* info, void* ws, cudaStream_t s);
+cudaError_t status_fetch_schurk(int* out, cudaStream_t s);
 // One CTA whose bounded wait (which 0: mbarrier, 1: cross-CTA counter) is
 // never satisfied; gives up after limit_ns.  w: 3 device ints.
 kronq_status wait_selftest(int which, unsigned long long limit_ns, int* w, cudaStream_t s);
@@ -181,6 +197,19 @@ struct SweepDesc {
 };
 kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s);
 
+// The body of kronq_quantize_layer after validation.  mode 0: dead columns,
+// damping and factorisation of HX; 1: HX holds U already; 2: HX is damped
+// already (no dead-column rule), factorisation only.
+size_t quantize_core_workspace_bytes(int64_t m, int64_t n);
+kronq_status check_quant_args(float* Wt, float* HX, int64_t m, int64_t n, const kronq_quant_params* p,
+                              uint8_t* codes, float* scales, float* zeros, float* E, int* info,
+                              const char* who);
+kronq_status quantize_core(float* Wt, float* HX, int64_t m, int64_t n, const kronq_quant_params* p,
+                           uint8_t* codes, float* scales, float* zeros, float* E, int* info,
+                           void* workspace, cudaStream_t st, int mode);
+// Dead-column rule and damping of H in place (dead flags out, info reset).
+kronq_status damp_factor(float* H, int64_t n, float damp_rel, uint8_t* dead, int* info, cudaStream_t s);
+
 // ------------------------------------------------------------ pack / misc
 kronq_status pack_codes(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* out,
                         cudaStream_t s);
@@ -188,6 +217,11 @@ kronq_status unpack_codes(const uint32_t* in, int64_t m, int64_t n, int bits, ui
                           cudaStream_t s);
 kronq_status diag_sums(const float* HX, int64_t n, const float* HG, int64_t m, double* dev2,
                        cudaStream_t s);
+// out (+)= sum of squares of the T x d token matrix A (float64); partial:
+// token_sqsum_partials() doubles of device scratch.
+size_t token_sqsum_partials();
+kronq_status token_sqsum(const void* A, bool bf16, int64_t T, int64_t d, int64_t lda, double* out,
+                         int zero_first, double* partial, cudaStream_t s);
 kronq_status dot_sum(const float* a, const float* b, int64_t count, double* dev1, double* partial,
                      cudaStream_t s);
 

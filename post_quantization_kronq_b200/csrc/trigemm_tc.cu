@@ -319,6 +319,8 @@ constexpr int TS_SPLIT = 2 * TS_BOX;              // 8 KB
 constexpr int TS_STAGE = 6 * TS_SPLIT;            // 48 KB: A hi/mid/lo, B hi/mid/lo
 constexpr int TNS = 2;
 constexpr int T_THREADS = CV_THREADS + 64;        // + producer warp + MMA warp
+constexpr int T_SEG = 4;                          // 32-deep chunks per accumulation segment
+constexpr uint32_t T_TMEM_COLS = 2 * BN;          // two segment accumulators
 constexpr int T_SMEM = TNF * TF_STAGE + TNS * TS_STAGE + 1024 + 256;
 static_assert(BM * C_LD * 4 <= TNF * TF_STAGE + TNS * TS_STAGE, "C staging fits");
 
@@ -343,14 +345,15 @@ __global__ void __launch_bounds__(T_THREADS, 1)
   uint8_t* fst = smem;                              // fp32 ring
   uint8_t* bst = smem + TNF * TF_STAGE;             // bf16 ring
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TNF * TF_STAGE + TNS * TS_STAGE);
-  // ffull[3] fempty[3] bfull[2] bempty[2] acc
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TNF + 2 * TNS + 1);
+  // ffull[3] fempty[3] bfull[2] bempty[2] accfull[2] accempty[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TNF + 2 * TNS + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto ffull = [&](int i) { return smem_u32(&bars[i]); };
   auto fempty = [&](int i) { return smem_u32(&bars[TNF + i]); };
   auto bfull = [&](int i) { return smem_u32(&bars[2 * TNF + i]); };
   auto bempty = [&](int i) { return smem_u32(&bars[2 * TNF + TNS + i]); };
-  const uint32_t accbar = smem_u32(&bars[2 * TNF + 2 * TNS]);
+  auto accfull = [&](int i) { return smem_u32(&bars[2 * TNF + 2 * TNS + i]); };
+  auto accempty = [&](int i) { return smem_u32(&bars[2 * TNF + 2 * TNS + 2 + i]); };
 
   const int bid = blockIdx.x;
   int tm, tn;
@@ -378,20 +381,55 @@ __global__ void __launch_bounds__(T_THREADS, 1)
       mbar_init(bfull(i), 8);
       mbar_init(bempty(i), 1);
     }
-    mbar_init(accbar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(accfull(i), 1);
+      mbar_init(accempty(i), 8);
+    }
     fence_mbar_init();
   }
   if (warp == 8) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_slot), T_TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int nseg = (nchunks + T_SEG - 1) / T_SEG;
 
   if (warp < 8) {
     bool ok = true;
+    // Accumulation in segments of T_SEG chunks (128 k): the MMAs of a
+    // segment go to one of two TMEM accumulators, and these warps add each
+    // finished segment into float32 registers with round-to-nearest (a
+    // single accumulator over a long K drifts by ~1e-5 relative per 2k of
+    // K).  Warp w owns TMEM lanes 32 (w % 4) and columns 64 (w / 4) .. +63.
+    const int q = warp & 3, hc = warp >> 2;
+    float acc[64];
+#pragma unroll
+    for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+    auto drain = [&](int sgi) -> bool {
+      const int b = sgi & 1;
+      int got = 1;
+      if (lane == 0) got = mbar_wait(accfull(b), (uint32_t)(sgi >> 1) & 1u) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      __syncwarp();
+      if (!got) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + (uint32_t)(b * BN + 64 * hc + 32 * h), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[32 * h + e] = __fadd_rn(acc[32 * h + e], __uint_as_float(v[e]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty(b));
+      return true;
+    };
     for (int s = 0; s < nchunks; ++s) {
       const int fs = s % TNF, fu = s / TNF, bs = s & 1, bu = s >> 1;
       const int kc = kbeg + s * TBK;
@@ -443,30 +481,22 @@ __global__ void __launch_bounds__(T_THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bfull(bs));
+      // the last chunk of segment sg is converted: the segment before it is
+      // (or soon will be) complete in its accumulator
+      const int sg = s / T_SEG;
+      if ((s % T_SEG == T_SEG - 1 || s == nchunks - 1) && sg >= 1 && !drain(sg - 1)) { ok = false; break; }
     }
-    // epilogue (as in the generic kernel)
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && nchunks > 0) {
-      int got = 1;
-      if (lane == 0) got = mbar_wait(accbar, 0) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, got, 0) != 0;
-    }
-    const int q = warp & 3, hc = warp >> 2;
+    if (ok && nseg > 0) ok = __all_sync(0xffffffffu, drain(nseg - 1));
+    // epilogue (as in the generic kernel), from the register sums
     const int r = 32 * q + lane;
     float* cst = reinterpret_cast<float*>(smem);
     if (ok) {
-      tc_fence_after();
-#pragma unroll 1
+#pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
-        __syncwarp();  // the TMEM load is warp-collective
-        if (nchunks > 0) {
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 64 * hc + 32 * cc, v);
-          tmem_wait_ld();
-        } else {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) v[t] = 0u;
-        }
+        for (int t = 0; t < 32; ++t) v[t] = __float_as_uint(acc[32 * cc + t]);
         float* dst = cst + r * C_LD + 64 * hc + 32 * cc;
 #pragma unroll
         for (int t = 0; t < 32; t += 4)
@@ -517,9 +547,15 @@ __global__ void __launch_bounds__(T_THREADS, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, true, true);
       for (int s = 0; s < nchunks; ++s) {
         const int bs = s & 1, bu = s >> 1;
+        const int sg = s / T_SEG, b = sg & 1;
+        const bool first = (s % T_SEG) == 0;
+        // a segment's accumulator is free once the converter warps have
+        // added the segment two back into their registers
+        if (first && sg >= 2 && !mbar_wait(accempty(b), (uint32_t)((sg >> 1) - 1) & 1u)) break;
         if (!mbar_wait(bfull(bs), bu & 1)) break;
         tc_fence_after();
         const uint32_t sa = smem_u32(bst + bs * TS_STAGE), sb = sa + 3 * TS_SPLIT;
+        const uint32_t acc = tmem + (uint32_t)(b * BN);
 #pragma unroll
         for (int kk = 0; kk < TBK / 16; ++kk) {
 #pragma unroll
@@ -529,12 +565,12 @@ __global__ void __launch_bounds__(T_THREADS, 1)
             const int pb = (t == 1 || t == 5) ? 1 : (t == 3 ? 2 : 0);
             const uint64_t da = smem_desc_sw128(sa + pa * TS_SPLIT + kk * 2048, TS_BOX, 1024);
             const uint64_t db = smem_desc_sw128(sb + pb * TS_SPLIT + kk * 2048, TS_BOX, 1024);
-            mma_bf16(tmem, da, db, idesc, (s > 0 || kk > 0 || t > 0) ? 1u : 0u);
+            mma_bf16(acc, da, db, idesc, (!first || kk > 0 || t > 0) ? 1u : 0u);
           }
         }
         mma_commit(bempty(bs));
+        if (s % T_SEG == T_SEG - 1 || s == nchunks - 1) mma_commit(accfull(b));
       }
-      if (nchunks > 0) mma_commit(accbar);
     }
     __syncwarp();
   }
@@ -542,7 +578,7 @@ __global__ void __launch_bounds__(T_THREADS, 1)
   __syncthreads();
   if (warp == 8) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, T_TMEM_COLS);
   }
 }
 
