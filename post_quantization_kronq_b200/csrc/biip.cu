@@ -340,6 +340,195 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
   }
 }
 
+// ------------------------------------------------------------ compile-time row transform
+// The same pass for the lengths of the Llama sublayers, L = K 2^LOGP with K
+// and LOGP known at compile time, so that every index of the DCT and the
+// radix-16 Walsh-Hadamard passes is a shift or a multiply by a constant:
+// R rows per CTA group (a power of two), 512 threads, the next group's
+// loads held in registers while the current group is transformed and
+// stored, the column factors (sign and rescale) read from a table computed
+// once per launch.  Arithmetic per element is that of rowpass_kernel.
+template <int K, int LOGP, int R>
+struct FastShape {
+  static constexpr int P = 1 << LOGP;
+  static constexpr int L = K * P;
+  static constexpr int CPT = (L + RP_THREADS - 1) / RP_THREADS;   // columns per thread and row
+  static constexpr int RS = (L + (L >> 5)) | 1;                   // padded row stride
+  static constexpr int LOGR = (R == 1) ? 0 : (R == 2) ? 1 : (R == 4) ? 2 : 3;
+};
+
+// One radix-2^NB pass over bits LO .. LO+NB-1 of a (index a K + b) of R rows.
+template <int K, int LOGP, int R, int LO, int NB>
+__device__ __forceinline__ void fwht_pass(float* buf) {
+  using S = FastShape<K, LOGP, R>;
+  constexpr int G = 1 << NB;
+  constexpr int IPR = (S::P / G) * K;          // items per row
+  constexpr int LOMASK = (1 << LO) - 1;
+  for (int t = threadIdx.x; t < IPR * R; t += RP_THREADS) {
+    const int rr = t / IPR;
+    const int rem = t - rr * IPR;
+    const int b = rem % K;
+    const int qv = rem / K;
+    const int a0 = ((qv >> LO) << (LO + NB)) | (qv & LOMASK);
+    float* row = buf + rr * S::RS;
+    float x[G];
+#pragma unroll
+    for (int u = 0; u < G; ++u) x[u] = row[padx((a0 + (u << LO)) * K + b)];
+#pragma unroll
+    for (int h = 1; h < G; h <<= 1)
+#pragma unroll
+      for (int u = 0; u < G; ++u)
+        if ((u & h) == 0) {
+          const float s0 = x[u], s1 = x[u | h];
+          x[u] = s0 + s1;
+          x[u | h] = s0 - s1;
+        }
+#pragma unroll
+    for (int u = 0; u < G; ++u) row[padx((a0 + (u << LO)) * K + b)] = x[u];
+  }
+  __syncthreads();
+}
+
+template <int K, int LOGP, int R, int LO>
+__device__ __forceinline__ void fwht_all(float* buf) {
+  if constexpr (LO < LOGP) {
+    constexpr int NB = (LOGP - LO) < 4 ? (LOGP - LO) : 4;
+    fwht_pass<K, LOGP, R, LO, NB>(buf);
+    fwht_all<K, LOGP, R, LO + NB>(buf);
+  }
+}
+
+template <bool BF16, int K, int LOGP, int R>
+__global__ void __launch_bounds__(RP_THREADS, 1) rowpass_fast_kernel(RowPass p, const float* cf) {
+  using S = FastShape<K, LOGP, R>;
+  extern __shared__ __align__(16) float sm[];
+  float* buf = sm;
+  float* Cm = sm + R * S::RS;   // K x K DCT matrix (K > 1)
+  const int tid = threadIdx.x;
+  const int64_t ngroups = (p.rows + R - 1) / R;
+  if (K > 1) {
+    for (int t = tid; t < K * K; t += RP_THREADS) {
+      const int i = t / K, j = t - (t / K) * K;
+      const double ci = (i == 0) ? sqrt(0.5) : 1.0;
+      Cm[t] = (float)(sqrt(2.0 / K) * ci * cospi((double)((2 * j + 1) * i) / (2.0 * K)));
+    }
+  }
+  float v[R][S::CPT];
+  auto load = [&](int64_t g) {
+    const int64_t r0 = g * R;
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr) {
+      const bool live = r0 + rr < p.rows;
+      const int64_t base = (r0 + rr) * p.ld_in;
+#pragma unroll
+      for (int c = 0; c < S::CPT; ++c) {
+        const int j = tid + c * RP_THREADS;
+        float x = 0.f;
+        if (live && j < S::L) {
+          if (BF16) x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[base + j]);
+          else x = reinterpret_cast<const float*>(p.in)[base + j];
+        }
+        v[rr][c] = x;
+      }
+    }
+  };
+  int64_t grp = blockIdx.x;
+  if (grp < ngroups) load(grp);
+  for (; grp < ngroups; grp += gridDim.x) {
+    const int64_t r0 = grp * R;
+    const int rows_here = (int)((p.rows - r0) < R ? (p.rows - r0) : R);
+    // 1. rows into shared memory, times the column factors (forward)
+#pragma unroll
+    for (int c = 0; c < S::CPT; ++c) {
+      const int j = tid + c * RP_THREADS;
+      if (j < S::L) {
+        const float f = p.inverse ? 1.f : (cf ? cf[j] : col_factor(p, j));
+#pragma unroll
+        for (int rr = 0; rr < R; ++rr) buf[rr * S::RS + padx(j)] = v[rr][c] * f;
+      }
+    }
+    __syncthreads();
+    if (grp + gridDim.x < ngroups) load(grp + gridDim.x);   // in flight during the transform
+    if (p.rotate) {
+      // 2. DCT along b: one thread per (row, a), all K inputs in registers,
+      //    each output written as soon as it is formed
+      if (K > 1) {
+        for (int t = tid; t < R * S::P; t += RP_THREADS) {
+          const int rr = t >> LOGP;
+          const int a = t & (S::P - 1);
+          float* row = buf + rr * S::RS;
+          float y[K];
+#pragma unroll
+          for (int bb = 0; bb < K; ++bb) y[bb] = row[padx(a * K + bb)];
+#pragma unroll
+          for (int o = 0; o < K; ++o) {
+            float acc = 0.f;
+#pragma unroll
+            for (int bb = 0; bb < K; ++bb) acc = fmaf(p.inverse ? Cm[bb * K + o] : Cm[o * K + bb], y[bb], acc);
+            row[padx(a * K + o)] = acc;
+          }
+        }
+        __syncthreads();
+      }
+      // 3. Walsh-Hadamard along a, radix-16 passes (a shorter last one)
+      fwht_all<K, LOGP, R, 0>(buf);
+    }
+    // 4. transposed store: consecutive threads take consecutive rows of one
+    //    column (R-float runs of the output rows)
+    const float nrm = p.rotate ? (float)(1.0 / sqrt((double)S::P)) : 1.f;
+    const int rr = tid & (R - 1);
+    constexpr int JSTEP = RP_THREADS >> S::LOGR;
+    if (rr < rows_here) {
+      const float* src = buf + rr * S::RS;
+      for (int j = tid >> S::LOGR; j < S::L; j += JSTEP) {
+        float x = src[padx(j)] * nrm;
+        if (p.inverse) x = x * (cf ? cf[j] : col_factor(p, j));
+        p.out[(int64_t)j * p.ld_out + r0 + rr] = x;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void colfactor_kernel(RowPass p, float* cf) {
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < (int)p.L; j += gridDim.x * blockDim.x)
+    cf[j] = col_factor(p, j);
+}
+
+template <bool BF16, int K, int LOGP, int R>
+kronq_status launch_fast(const RowPass& p, cudaStream_t s) {
+  using S = FastShape<K, LOGP, R>;
+  const float* cf = nullptr;
+  if (p.cf) {
+    colfactor_kernel<<<(unsigned)ceil_div(S::L, 256), 256, 0, s>>>(p, p.cf);
+    KQ_LAUNCH_CHECK("colfactor_kernel");
+    cf = p.cf;
+  }
+  const int smem = (R * S::RS + (K > 1 ? K * K : 0)) * (int)sizeof(float);
+  const void* fn = reinterpret_cast<const void*>(&rowpass_fast_kernel<BF16, K, LOGP, R>);
+  cudaError_t e = allow_smem(fn, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rowpass_fast)");
+  const int64_t groups = ceil_div(p.rows, R);
+  const int64_t grid = groups < (int64_t)sm_count() ? groups : (int64_t)sm_count();
+  rowpass_fast_kernel<BF16, K, LOGP, R><<<(unsigned)grid, RP_THREADS, (size_t)smem, s>>>(p, cf);
+  KQ_LAUNCH_CHECK("rowpass_fast_kernel");
+  return KRONQ_OK;
+}
+
+// The compile-time variants: (odd factor, log2 of the power of two, rows
+// per group).  Returns false when the length has none.
+template <bool BF16>
+bool try_fast(const RowPass& p, cudaStream_t s, kronq_status& r) {
+  switch (p.L) {
+    case 28672: r = launch_fast<BF16, 7, 12, 1>(p, s); return true;   // Llama-3-70B MLP
+    case 14336: r = launch_fast<BF16, 7, 11, 2>(p, s); return true;   // Llama-3-8B MLP
+    case 11008: r = launch_fast<BF16, 43, 8, 2>(p, s); return true;   // Llama-2-7B MLP
+    case 8192: r = launch_fast<BF16, 1, 13, 4>(p, s); return true;    // Llama-3-70B hidden
+    case 1024: r = launch_fast<BF16, 1, 10, 8>(p, s); return true;    // Llama-3-8B k/v
+    default: return false;
+  }
+}
+
 // ------------------------------------------------------------ norms
 template <typename T>
 __device__ __forceinline__ float ld_val(const void* W, int64_t idx) {
@@ -443,6 +632,10 @@ kronq_status rowpass(const RowPass& p, cudaStream_t s) {
   A.R = R;
   A.logR = 0;
   while ((1 << A.logR) < R) ++A.logR;
+  if (p.rotate) {
+    kronq_status r = KRONQ_OK;
+    if (p.in_bf16 ? try_fast<true>(p, s, r) : try_fast<false>(p, s, r)) return r;
+  }
   const bool f4096 = (p.L == 4096 && K == 1);
   const int64_t smem = R * bytes_per_row + cbytes + (f4096 ? p.L * 4 : 0);
   const void* fn = f4096 ? (p.in_bf16 ? reinterpret_cast<const void*>(&rowpass_kernel<true, true>)
