@@ -126,6 +126,23 @@ kronq_status kronq_accumulate_factors(const void* A, kronq_dtype dt, int64_t T, 
 kronq_status kronq_sensitivity(const float* HX, int64_t n, const float* HG, int64_t m,
                                double* out3, void* workspace, size_t ws_bytes, kronq_stream_t s);
 
+/* The same traces straight from the tokens, without forming the factors:
+ * tr(A^T A) = sum_t |a_t|^2 (a first pass over a whole model's sublayers,
+ * before any factor is accumulated, so that the bit allocation can run
+ * first).  A: T x d token rows, row stride lda (bf16 or float32), device.
+ * trace: ONE double of device memory, overwritten (zero_first != 0) or
+ * added to, so that token chunks can be streamed; the sum is formed in
+ * float64 in a fixed order.  workspace: kronq_trace_tokens_workspace_bytes()
+ * bytes of device memory, 256-byte aligned.  Asynchronous on s.
+ * kronq_sensitivity_from_traces: traces = two device doubles { tr(H_X),
+ * tr(H_G) } (e.g. two kronq_trace_tokens results); out3 (HOST) receives
+ * { tr(H_X), tr(H_G), tr(H_G) * tr(H_X) }.  Synchronises the stream. */
+size_t kronq_trace_tokens_workspace_bytes(void);
+kronq_status kronq_trace_tokens(const void* A, kronq_dtype dt, int64_t T, int64_t d, int64_t lda,
+                                double* trace, int zero_first, void* workspace, size_t ws_bytes,
+                                kronq_stream_t s);
+kronq_status kronq_sensitivity_from_traces(const double* traces, double* out3, kronq_stream_t s);
+
 /* Bit allocation over L sublayers (host only; KronQ README "Mapping paper
  * results to flags", --inter_layer_mp).  Budget mode: start at bmin bits,
  * repeatedly give +1 bit to the sublayer with the largest
@@ -233,6 +250,31 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
 kronq_status kronq_quantize_layer_static(float* Wt, float* HX, int64_t m, int64_t n,
                                          const kronq_quant_params* p, uint8_t* codes, float* scales,
                                          float* zeros, float* E, int* info, kronq_stream_t s);
+
+/* kronq_quantize_layer_act_order -- the same pass with the recipe's
+ * --act_order (KronQ README, "Reproduce from scratch"; not defined on the
+ * pages, read as GPTQ's act-order heuristic): after the dead-column rule
+ * the columns are swept in order of decreasing diagonal of H~_X (ties keep
+ * the column order), groups are consecutive columns of that order, and the
+ * outputs come back in the original column order.
+ *   Wt, codes, E   as kronq_quantize_layer, in the ORIGINAL column order.
+ *   scales, zeros  m x ngroups, one column per group of the SWEEP order.
+ *   g_idx          n ints (device) out: column j uses group g_idx[j]
+ *                  (rank of j in the sweep order / group; 0 for group -1).
+ *   perm           n ints (device) out, may be NULL: perm[k] = the column
+ *                  swept k-th.
+ *   HX             in H~_X; out U of the permuted, damped factor (upper
+ *                  triangle, sweep order).
+ *   flags          KRONQ_WRITE_E and KRONQ_ORDERED_FP32; KRONQ_U_GIVEN is
+ *                  rejected (the order comes from H~_X).
+ *   workspace      >= kronq_quantize_act_order_workspace_bytes(m, n, p)
+ *                  (holds the permuted copies: n^2 + m n floats and more).
+ * Asynchronous on s. */
+size_t kronq_quantize_act_order_workspace_bytes(int64_t m, int64_t n, const kronq_quant_params* p);
+kronq_status kronq_quantize_layer_act_order(float* Wt, float* HX, int64_t m, int64_t n,
+                                            const kronq_quant_params* p, uint8_t* codes, float* scales,
+                                            float* zeros, float* E, int* g_idx, int* perm, int* info,
+                                            void* workspace, size_t ws_bytes, kronq_stream_t s);
 
 /* ---------------------------------------------------------------------------
  * Step 5 -- packing.  KronQ README "Model zoo": W4/W2 as packed int4/int2,

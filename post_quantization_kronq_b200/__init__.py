@@ -15,10 +15,12 @@ from ._lib import (BF16, BIIP_MODES, F32, ORDERED_FP32, U_GIVEN, WRITE_E, KronqE
 
 __all__ = [
     "KronqError", "QuantParams", "U_GIVEN", "ORDERED_FP32", "WRITE_E",
-    "kronq_accumulate_factors", "kronq_sensitivity", "kronq_allocate_bits",
+    "kronq_accumulate_factors", "kronq_sensitivity", "kronq_trace_tokens",
+    "kronq_sensitivity_from_traces", "kronq_allocate_bits",
     "kronq_allocate_topn_types", "kronq_biip_workspace_bytes", "kronq_biip_forward",
     "kronq_biip_inverse", "kronq_quantize_workspace_bytes", "kronq_quantize_layer",
-    "kronq_quantize_layer_static",
+    "kronq_quantize_layer_static", "kronq_quantize_act_order_workspace_bytes",
+    "kronq_quantize_layer_act_order",
     "kronq_pack", "kronq_unpack", "kronq_device_status", "kronq_wait_selftest",
     "kronq_kfac_loss_workspace_bytes",
     "kronq_kfac_loss", "kronq_launch_count", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
@@ -102,6 +104,25 @@ def kronq_sensitivity(HX, HG, ws=None, stream=None):
     return out[0], out[1], out[2]
 
 
+def kronq_trace_tokens(A, trace, zero_first: bool = True, ws=None, stream=None):
+    """trace (one device float64) (+)= sum_t |a_t|^2 = tr(A^T A) for tokens A (T x d)."""
+    T, d = A.shape
+    if A.stride(1) != 1:
+        raise ValueError("A must have unit stride along d (row-major token rows)")
+    _rowmajor(trace, "trace")
+    ws = workspace(int(lib.kronq_trace_tokens_workspace_bytes()), A.device) if ws is None else ws
+    check(lib.kronq_trace_tokens(_ptr(A), _dtype_code(A), T, d, A.stride(0), _ptr(trace),
+                                 1 if zero_first else 0, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def kronq_sensitivity_from_traces(traces, stream=None):
+    """(tr(H_X), tr(H_G), tr(H_G) * tr(H_X)) from two device float64 traces (synchronises)."""
+    _rowmajor(traces, "traces")
+    out = (ctypes.c_double * 3)()
+    check(lib.kronq_sensitivity_from_traces(_ptr(traces), out, _stream(stream)))
+    return out[0], out[1], out[2]
+
+
 def kronq_allocate_bits(sens, sizes, avg_bits: float = 2.5, bmin: int = 2, bmax: int = 4):
     L = len(sens)
     s = (ctypes.c_double * L)(*[float(v) for v in sens])
@@ -171,6 +192,25 @@ def kronq_quantize_layer_static(Wt, HX, params: QuantParams, codes, scales, zero
     check(lib.kronq_quantize_layer_static(_ptr(Wt), _ptr(HX), m, n, ctypes.byref(params),
                                           _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(E),
                                           _ptr(info), _stream(stream)))
+
+
+def kronq_quantize_act_order_workspace_bytes(m: int, n: int, params: QuantParams) -> int:
+    return int(lib.kronq_quantize_act_order_workspace_bytes(m, n, ctypes.byref(params)))
+
+
+def kronq_quantize_layer_act_order(Wt, HX, params: QuantParams, codes, scales, zeros, g_idx, info,
+                                   E=None, perm=None, ws=None, stream=None):
+    """kronq_quantize_layer with the act-order sweep order; outputs in the
+    original column order, scales/zeros per sweep-order group, g_idx (n int32)."""
+    m, n = Wt.shape
+    for t, name in ((Wt, "Wt"), (HX, "HX"), (codes, "codes"), (scales, "scales"), (zeros, "zeros"),
+                    (g_idx, "g_idx"), (info, "info"), (E, "E"), (perm, "perm")):
+        _rowmajor(t, name)
+    if ws is None:
+        ws = workspace(kronq_quantize_act_order_workspace_bytes(m, n, params), Wt.device)
+    check(lib.kronq_quantize_layer_act_order(_ptr(Wt), _ptr(HX), m, n, ctypes.byref(params), _ptr(codes),
+                                             _ptr(scales), _ptr(zeros), _ptr(E), _ptr(g_idx), _ptr(perm),
+                                             _ptr(info), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def kronq_pack(codes, bits: int, out, stream=None):

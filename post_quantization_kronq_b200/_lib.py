@@ -44,6 +44,9 @@ _qp = ctypes.POINTER(QuantParams)
 SIGNATURES = {
     "kronq_accumulate_factors": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _vp]),
     "kronq_sensitivity": (_int, [_vp, _i64, _vp, _i64, _dp, _vp, _sz, _vp]),
+    "kronq_trace_tokens_workspace_bytes": (_sz, []),
+    "kronq_trace_tokens": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp]),
+    "kronq_sensitivity_from_traces": (_int, [_vp, _dp, _vp]),
     "kronq_allocate_bits": (_int, [_dp, _i64p, _int, ctypes.c_double, _int, _int, _ip]),
     "kronq_allocate_topn_types": (_int, [_dp, _ip, _int, _int, _int, _int, _ip]),
     "kronq_biip_workspace_bytes": (_sz, [_i64, _i64]),
@@ -55,6 +58,9 @@ SIGNATURES = {
                                     _vp]),
     "kronq_quantize_layer_static": (_int, [_vp, _vp, _i64, _i64, _qp, _vp, _vp, _vp, _vp, _vp,
                                            _vp]),
+    "kronq_quantize_act_order_workspace_bytes": (_sz, [_i64, _i64, _qp]),
+    "kronq_quantize_layer_act_order": (_int, [_vp, _vp, _i64, _i64, _qp, _vp, _vp, _vp, _vp, _vp,
+                                              _vp, _vp, _vp, _sz, _vp]),
     "kronq_pack": (_int, [_vp, _i64, _i64, _int, _vp, _vp]),
     "kronq_unpack": (_int, [_vp, _i64, _i64, _int, _vp, _vp]),
     "kronq_device_status": (_int, [_ip, _vp]),
