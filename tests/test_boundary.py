@@ -218,3 +218,17 @@ def test_wait_selftest_validation():
     assert _st(L.kronq_wait_selftest(0, 2000000000, FAKE, 16, None)) == _lib.ERR_INVALID_ARG
     assert _st(L.kronq_wait_selftest(1, 1000000, None, 16, None)) == _lib.ERR_INVALID_ARG
     assert _st(L.kronq_wait_selftest(1, 1000000, FAKE, 8, None)) == _lib.ERR_INVALID_ARG
+
+
+def test_act_order_validation():
+    L = _lib.lib
+    p = _lib.QuantParams(bits=2, group=128, asym=1, damp_rel=0.01, block=128, flags=_lib.U_GIVEN)
+    args = [FAKE, FAKE, 8, 256, ctypes.byref(p), FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE, 1 << 30, None]
+    assert _st(L.kronq_quantize_layer_act_order(*args)) == _lib.ERR_INVALID_ARG      # U_GIVEN
+    p.flags = 0
+    args[9] = None
+    assert _st(L.kronq_quantize_layer_act_order(*args)) == _lib.ERR_INVALID_ARG      # no g_idx
+    args[9] = FAKE
+    args[13] = 16
+    assert _st(L.kronq_quantize_layer_act_order(*args)) == _lib.ERR_INVALID_ARG      # workspace
+    assert L.kronq_quantize_act_order_workspace_bytes(8, 256, ctypes.byref(p)) > 256 * 256 * 4
