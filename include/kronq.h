@@ -238,8 +238,9 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
  * workspace: the scratch is a file-scope static device array of 64 MiB that
  * every GPU loading the library holds until the process exits.
  *   - Layers whose kronq_quantize_workspace_bytes(m, n, p) exceeds 64 MiB
- *     (for example n = 4096 with m above ~9000, or n above ~7000 with small
- *     m) are rejected with KRONQ_ERR_INVALID_ARG before anything runs.
+ *     (for example n = 4096 with m above ~6500, or any n above 4096, whose
+ *     blocked factorisation needs more scratch) are rejected with
+ *     KRONQ_ERR_INVALID_ARG before anything runs.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.

@@ -490,9 +490,175 @@ __global__ void __launch_bounds__(RP_THREADS, 1) rowpass_fast_kernel(RowPass p, 
   }
 }
 
+// Rows too long for more than one per CTA (L = 28672: 118 KB of shared
+// memory each) would leave the transposed store one float wide.  A cluster
+// of CL CTAs transforms CL consecutive rows, one per CTA, and then stores
+// together: CTA c writes the output rows j of its slice [c L / CL,
+// (c + 1) L / CL) with the CL values of each j gathered from the cluster's
+// shared memory (distributed shared memory), CL consecutive floats per
+// output row.  Cluster barriers separate the transform, the store and the
+// next group.
+constexpr int CL = 8;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+template <bool BF16, int K, int LOGP>
+__global__ void __launch_bounds__(RP_THREADS, 1) rowpass_cluster_kernel(RowPass p, const float* cf) {
+  using S = FastShape<K, LOGP, 1>;
+  extern __shared__ __align__(16) float sm[];
+  float* buf = sm;
+  float* Cm = sm + S::RS;
+  const int tid = threadIdx.x;
+  const uint32_t rank = cluster_rank();
+  const int64_t cid = blockIdx.x / CL, ncl = gridDim.x / CL;
+  const int64_t ngroups = (p.rows + CL - 1) / CL;
+  if (K > 1) {
+    for (int t = tid; t < K * K; t += RP_THREADS) {
+      const int i = t / K, j = t - (t / K) * K;
+      const double ci = (i == 0) ? sqrt(0.5) : 1.0;
+      Cm[t] = (float)(sqrt(2.0 / K) * ci * cospi((double)((2 * j + 1) * i) / (2.0 * K)));
+    }
+  }
+  // the shared-memory address of buf in every CTA of the cluster
+  uint32_t peer[CL];
+#pragma unroll
+  for (int q = 0; q < CL; ++q) peer[q] = map_to_rank(smem_u32(buf), (uint32_t)q);
+  const float nrm = p.rotate ? (float)(1.0 / sqrt((double)S::P)) : 1.f;
+  float v[S::CPT];
+  auto load = [&](int64_t g) {
+    const int64_t row = g * CL + rank;
+    const bool live = row < p.rows;
+#pragma unroll
+    for (int c = 0; c < S::CPT; ++c) {
+      const int j = tid + c * RP_THREADS;
+      float x = 0.f;
+      if (live && j < S::L) {
+        if (BF16) x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.in)[row * p.ld_in + j]);
+        else x = reinterpret_cast<const float*>(p.in)[row * p.ld_in + j];
+      }
+      v[c] = x;
+    }
+  };
+  int64_t grp = cid;
+  if (grp < ngroups) load(grp);
+  for (; grp < ngroups; grp += ncl) {
+    const int64_t r0 = grp * CL;
+    const int rows_here = (int)((p.rows - r0) < CL ? (p.rows - r0) : CL);
+#pragma unroll
+    for (int c = 0; c < S::CPT; ++c) {
+      const int j = tid + c * RP_THREADS;
+      if (j < S::L) buf[padx(j)] = v[c] * (p.inverse ? 1.f : (cf ? cf[j] : col_factor(p, j)));
+    }
+    __syncthreads();
+    if (grp + ncl < ngroups) load(grp + ncl);
+    if (p.rotate) {
+      if (K > 1) {
+        for (int a = tid; a < S::P; a += RP_THREADS) {
+          float y[K];
+#pragma unroll
+          for (int bb = 0; bb < K; ++bb) y[bb] = buf[padx(a * K + bb)];
+#pragma unroll
+          for (int o = 0; o < K; ++o) {
+            float acc = 0.f;
+#pragma unroll
+            for (int bb = 0; bb < K; ++bb) acc = fmaf(p.inverse ? Cm[bb * K + o] : Cm[o * K + bb], y[bb], acc);
+            buf[padx(a * K + o)] = acc;
+          }
+        }
+        __syncthreads();
+      }
+      fwht_all<K, LOGP, 1, 0>(buf);
+    }
+    cluster_sync_all();   // every row of the group is transformed
+    constexpr int SLICE = S::L / CL;
+    const int j0 = (int)rank * SLICE;
+    const bool vec = rows_here == CL && (p.ld_out % 4) == 0 && (r0 % 4) == 0 &&
+                     ((reinterpret_cast<uintptr_t>(p.out) & 15) == 0);
+    for (int jj = tid; jj < SLICE; jj += RP_THREADS) {
+      const int j = j0 + jj;
+      const uint32_t off = (uint32_t)padx(j) * 4u;
+      float x[CL];
+#pragma unroll
+      for (int q = 0; q < CL; ++q) x[q] = ld_cluster_f32(peer[q] + off) * nrm;
+      if (p.inverse) {
+        const float f = cf ? cf[j] : col_factor(p, j);
+#pragma unroll
+        for (int q = 0; q < CL; ++q) x[q] *= f;
+      }
+      float* o = p.out + (int64_t)j * p.ld_out + r0;
+      if (vec) {
+        reinterpret_cast<float4*>(o)[0] = make_float4(x[0], x[1], x[2], x[3]);
+        reinterpret_cast<float4*>(o)[1] = make_float4(x[4], x[5], x[6], x[7]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < CL; ++q)
+          if (q < rows_here) o[q] = x[q];
+      }
+    }
+    cluster_sync_all();   // the peers have read this CTA's row
+  }
+}
+
 __global__ void colfactor_kernel(RowPass p, float* cf) {
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < (int)p.L; j += gridDim.x * blockDim.x)
     cf[j] = col_factor(p, j);
+}
+
+template <bool BF16, int K, int LOGP>
+kronq_status launch_cluster(const RowPass& p, cudaStream_t s) {
+  using S = FastShape<K, LOGP, 1>;
+  static_assert(S::L % CL == 0, "the row splits into CL slices");
+  const float* cf = nullptr;
+  if (p.cf) {
+    colfactor_kernel<<<(unsigned)ceil_div(S::L, 256), 256, 0, s>>>(p, p.cf);
+    KQ_LAUNCH_CHECK("colfactor_kernel");
+    cf = p.cf;
+  }
+  const int smem = (S::RS + (K > 1 ? K * K : 0)) * (int)sizeof(float);
+  const void* fn = reinterpret_cast<const void*>(&rowpass_cluster_kernel<BF16, K, LOGP>);
+  cudaError_t e = allow_smem(fn, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rowpass_cluster)");
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(RP_THREADS);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // persistent: as many clusters as fit at once, each looping over groups
+  int active = 0;
+  cfg.gridDim = dim3((unsigned)(CL * 16));
+  e = cudaOccupancyMaxActiveClusters(&active, fn, &cfg);
+  if (e != cudaSuccess || active < 1) return e != cudaSuccess ? cuda_fail(e, "cudaOccupancyMaxActiveClusters")
+                                                              : fail(KRONQ_ERR_CUDA, "rowpass: no cluster fits");
+  const int64_t groups = ceil_div(p.rows, CL);
+  const int64_t ncl = groups < (int64_t)active ? groups : (int64_t)active;
+  cfg.gridDim = dim3((unsigned)(CL * ncl));
+  e = cudaLaunchKernelEx(&cfg, rowpass_cluster_kernel<BF16, K, LOGP>, p, cf);
+  count_launch();
+  if (e != cudaSuccess) return cuda_fail(e, "rowpass_cluster_kernel");
+  return KRONQ_OK;
 }
 
 template <bool BF16, int K, int LOGP, int R>
@@ -520,7 +686,7 @@ kronq_status launch_fast(const RowPass& p, cudaStream_t s) {
 template <bool BF16>
 bool try_fast(const RowPass& p, cudaStream_t s, kronq_status& r) {
   switch (p.L) {
-    case 28672: r = launch_fast<BF16, 7, 12, 1>(p, s); return true;   // Llama-3-70B MLP
+    case 28672: r = launch_cluster<BF16, 7, 12>(p, s); return true;   // Llama-3-70B MLP
     case 14336: r = launch_fast<BF16, 7, 11, 2>(p, s); return true;   // Llama-3-8B MLP
     case 11008: r = launch_fast<BF16, 43, 8, 2>(p, s); return true;   // Llama-2-7B MLP
     case 8192: r = launch_fast<BF16, 1, 13, 4>(p, s); return true;    // Llama-3-70B hidden

@@ -24,9 +24,9 @@ def _inputs(m, n, seed, dead=()):
     X[:, list(dead)] = 0.0
     H = X.astype(np.float64).T @ X.astype(np.float64)
     if dead:   # unrotated, so the dead channels keep exact zero rows and columns
-        return W.astype(np.float32), H.astype(np.float32)
+        return np.ascontiguousarray(W, np.float32), np.ascontiguousarray(H, np.float32)
     Wt, Ht, _, _, _ = biip.biip_forward(W, H, None, seed, 0.25, "sv_only")
-    return Wt.astype(np.float32), Ht.astype(np.float32)
+    return np.ascontiguousarray(Wt, np.float32), np.ascontiguousarray(Ht, np.float32)
 
 
 def _run(Wt, Ht, bits, group, flags=0):
