@@ -12,7 +12,8 @@ G N(0, 1e-4) with lognormal per-channel scale), the factors accumulated in
 16 chunks of 16384 tokens; 2-bit group-128 asymmetric (the pages' headline
 2-bit Llama-3-70B), BiIP "full", alpha 0.25, damping 0.01.  Beside it (key
 "also"): a Llama-2-7B q_proj-shaped layer (4096 x 4096, T = 131072) at W2
-and W4.
+and W4, and the Llama-3-8B-shaped stack (224 sublayers) with inter-layer
+mixed precision, timed once after the rest.
 
 One step = the whole pass over every layer of the workload on inputs
 resident in HBM: H_X and H_G accumulation, trace sensitivity, BiIP forward,
@@ -386,6 +387,68 @@ def _time_steps(layers, chunk, steps, warmup, stream, flush, sampler=None, barri
     return per_step, launches, clocks
 
 
+STACK_SUBLAYERS = ["q_proj", "k_proj", "v_proj", "o_proj", "gate_proj", "up_proj", "down_proj"]
+
+
+def stack_bench(dev, blocks: int = 32, tokens: int = 65536, avg_bits: float = 2.5):
+    """The Llama-3-8B-shaped stack (blocks x 7 sublayers, T tokens each) through
+    StackPass: the trace-only first pass, the budget allocation over {2, 3, 4}
+    at avg_bits, and the per-layer passes at the allocated widths (with the
+    built-in trace check).  Only the library calls are timed (CUDA events);
+    the synthetic inputs are drawn between them, once per pass."""
+    import torch
+
+    from post_quantization_kronq_b200.stack import StackPass
+    from synth import LLAMA_SHAPES, llama_layer
+
+    names = [(b, s) for b in range(blocks) for s in STACK_SUBLAYERS]
+    shapes = [LLAMA_SHAPES["llama3_8b_" + s] for _, s in names]
+
+    def data(i):
+        b, sname = names[i]
+        m, n = shapes[i]
+        return llama_layer(m, n, tokens, seed=1000 * b + STACK_SUBLAYERS.index(sname), device=dev,
+                           rectified=(sname == "down_proj"))
+
+    stream = torch.cuda.current_stream()
+    sp = StackPass(shapes, avg_bits=avg_bits, group=128, device=dev)
+    t_trace = t_layers = 0.0
+    sp.sens1 = []
+    for i in range(len(shapes)):
+        _, X, G = data(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        sp.sens1.append(sp.trace_one(X, G))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_trace += e0.elapsed_time(e1)
+        del X, G
+    h0 = time.perf_counter()
+    bits = sp.allocate()
+    t_alloc = (time.perf_counter() - h0) * 1e3
+    sp.sens2 = []
+    for i in range(len(shapes)):
+        W, X, G = data(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        lp = sp.quantize_one(i, W, X, G)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert int(lp.info.item()) == 0
+        t_layers += e0.elapsed_time(e1)
+        del W, X, G
+    weights = sum(m * n for m, n in shapes)
+    total_ms = t_trace + t_alloc + t_layers
+    hist = {b: sum(1 for x in bits if x == b) for b in (2, 3, 4)}
+    avg = sum(b * m * n for b, (m, n) in zip(bits, shapes)) / weights
+    return {"workload": f"llama3-8b stack {blocks} blocks x 7 sublayers, T={tokens} tokens each, "
+                        f"inter-layer mixed precision over {{2,3,4}} bits at {avg_bits} average, g128",
+            "seconds": total_ms / 1e3, "value": weights / (total_ms / 1e3), "unit": UNIT,
+            "phases_ms": {"trace_pass": round(t_trace, 2), "allocation": round(t_alloc, 3),
+                          "layer_passes": round(t_layers, 2)},
+            "bits_histogram": hist, "average_bits": avg, "trace_check": "passed (1e-3)"}
+
+
 def run_kronq(args):
     import torch
 
@@ -532,6 +595,10 @@ def run_kronq(args):
             del lq
             torch.cuda.empty_cache()
 
+    if also is not None and not args.no_stack:
+        also["llama3_8b_stack"] = stack_bench(dev)
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         c = cpu_oracle_sample(wl, wl["bits"], wl["group"])
@@ -570,6 +637,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-also", action="store_true")
+    ap.add_argument("--no-stack", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
