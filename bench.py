@@ -105,16 +105,16 @@ def phase_work(layers, T: int):
                       per element; each factor takes two fp32 passes in and out)
     quantize_and_pack bound by its sequential chains (the diagonal steps of
                       the factorisation, n column steps of the sweep); shown
-                      against the tensor peak with 2 n^3 / 3 + m n^2 flop (the
-                      reverse Cholesky factor and its triangular inverse, and
-                      the error feedback of the sweep)
+                      against the tensor peak with n^3 / 3 + m n^2 flop (the
+                      reverse Cholesky factor R, and the error feedback of the
+                      sweep, which the R form takes from R: no inverse)
     """
     w = {"accumulate_HX_HG": 0, "sensitivity": 0, "biip_forward": 0, "quantize_and_pack": 0}
     for m, n in layers:
         w["accumulate_HX_HG"] += T * n * (n + 1) + T * m * (m + 1)
         w["sensitivity"] += 4 * (n + m)
         w["biip_forward"] += 16 * m * n + 16 * n * n + 16 * m * m
-        w["quantize_and_pack"] += 2 * n ** 3 / 3 + m * n * n
+        w["quantize_and_pack"] += n ** 3 / 3 + m * n * n
     return w
 
 

@@ -78,6 +78,7 @@ typedef enum {
 #define KRONQ_U_GIVEN      1u /* HX already holds U (upper): skip dead columns, damping, factorisation */
 #define KRONQ_ORDERED_FP32 2u /* fixed-order float32 trailing update (bit-exact test mode)             */
 #define KRONQ_WRITE_E      4u /* keep the scaled error E (m x n) in the E argument                      */
+#define KRONQ_R_FORM       8u /* sweep on R itself (H~ = R R^T); U = R^-1 is never formed               */
 
 /* Quantizer settings (KronQ README, "Reproduce from scratch":
  * --w_bits --w_groupsize --w_asym).
@@ -208,10 +209,19 @@ kronq_status kronq_biip_inverse(float* W, int64_t m, int64_t n, uint64_t seed,
  *   (2^b - 1), zero = rint(-x_min / scale)); q = clamp(rint(w / scale) +
  *   zero, 0, 2^b - 1) (round half to even); e = (w - scale (q - zero)) /
  *   U_jj; later columns -= e U[j, later], batched per `block` columns.
+ *   With KRONQ_R_FORM the same decisions are taken from R (H~_X + lambda I
+ *   = R R^T, U = R^-1) and the 128 x 128 diagonal blocks of U only: for the
+ *   swept columns S and the rest T, GPTQ's partial state W~_T - E_S U_ST is
+ *   W~_T + F U_TT with F = (W~ - Q)_S R_ST (W~ before the sweep), so each
+ *   128-column block starts from W~_G + F_G U_GG and is swept as above on
+ *   U_GG, and F accumulates (W~ - Q)_G R_G,later.  Not with KRONQ_U_GIVEN
+ *   or KRONQ_ORDERED_FP32 (KRONQ_ERR_INVALID_ARG); groups of at most 128
+ *   columns or -1 (KRONQ_ERR_UNSUPPORTED otherwise).
  *
  *   Wt     m x n float32: in W~, out the dequantised W~_q.
  *   HX     n x n float32: in H~_X (or U with KRONQ_U_GIVEN), out U (upper
- *          triangle; the strict lower triangle is scratch on return).
+ *          triangle; the strict lower triangle is scratch on return); with
+ *          KRONQ_R_FORM out R instead (upper, H~_X + lambda I = R R^T).
  *   codes  m x n uint8 out, values 0 .. 2^bits - 1.
  *   scales, zeros  m x ngroups float32 out, ngroups = 1 if group == -1 else
  *          ceil(n / group); zeros are integer valued.
@@ -219,7 +229,9 @@ kronq_status kronq_biip_inverse(float* W, int64_t m, int64_t n, uint64_t seed,
  *   info   one int (device) out: 0, or 1 + the largest index j for which the
  *          trailing submatrix (H~_X + lambda I)[j:, j:] was found not
  *          positive definite (codes etc. are then unspecified).
- *   workspace >= kronq_quantize_workspace_bytes(m, n, p), 256-byte aligned.
+ *   workspace >= kronq_quantize_workspace_bytes(m, n, p), 256-byte aligned
+ *          (KRONQ_R_FORM adds m n floats for the copy of W~ and 128^2
+ *          ceil(n / 128) for U's diagonal blocks).
  * ------------------------------------------------------------------------- */
 size_t kronq_quantize_workspace_bytes(int64_t m, int64_t n, const kronq_quant_params* p);
 
@@ -264,10 +276,10 @@ kronq_status kronq_quantize_layer_static(float* Wt, float* HX, int64_t m, int64_
  *                  (rank of j in the sweep order / group; 0 for group -1).
  *   perm           n ints (device) out, may be NULL: perm[k] = the column
  *                  swept k-th.
- *   HX             in H~_X; out U of the permuted, damped factor (upper
- *                  triangle, sweep order).
- *   flags          KRONQ_WRITE_E and KRONQ_ORDERED_FP32; KRONQ_U_GIVEN is
- *                  rejected (the order comes from H~_X).
+ *   HX             in H~_X; out U (R with KRONQ_R_FORM) of the permuted,
+ *                  damped factor (upper triangle, sweep order).
+ *   flags          KRONQ_WRITE_E, KRONQ_ORDERED_FP32 and KRONQ_R_FORM;
+ *                  KRONQ_U_GIVEN is rejected (the order comes from H~_X).
  *   workspace      >= kronq_quantize_act_order_workspace_bytes(m, n, p)
  *                  (holds the permuted copies: n^2 + m n floats and more).
  * Asynchronous on s. */

@@ -27,7 +27,9 @@ Readings fixed here (the pages are silent):
 * Sweep: for j = 0..n-1: quantize column j, e_j = (w_j - deq_j) / U_jj,
   W[:, j+1:] -= e_j U[j, j+1:].  ``block`` > 1 applies the same updates
   lazily (in-block rank-1, then one block product for the later columns),
-  a re-association that is exact in exact arithmetic.
+  a re-association that is exact in exact arithmetic.  gptq_sweep_rform
+  takes the same decisions from R = U^-1 (the factor of H + lambda I
+  itself) and the diagonal blocks of U only.
 """
 from __future__ import annotations
 
@@ -192,6 +194,59 @@ def gptq_sweep(Wt, U, bits: int, group: int, asym: bool = True, block: int = 1,
             W[:, j + 1:b1] -= np.outer(e, U[j, j + 1:b1])
         W[:, b1:] -= E[:, b0:b1] @ U[b0:b1, b1:]
     return dict(codes=codes, scales=scales, zeros=zeros, Q=Q, E=E, W_final=W)
+
+
+def gptq_sweep_rform(Wt, R, bits: int, group: int, asym: bool = True, block: int = 1):
+    """The sweep of gptq_sweep taken from R itself (H + lambda I = R R^T, R
+    upper, so U = R^-1), with only diagonal blocks of U formed.
+
+    With the columns split into the swept ones S and the rest T, and F =
+    (W - Q)_S R_ST (W the weights before the sweep, Q the dequantised values),
+    gptq_sweep's partial state is W_T - E_S U_ST = W_T + F U_TT, because
+    E_S = (W - Q)_S R_SS and R_SS U_ST = -R_ST U_TT.  So:
+      * column j, when its turn comes, holds w_j + F_j / R_jj (U_TT is upper,
+        and its (j, j) entry is 1 / R_jj once every earlier column is in S);
+      * a group G starting at column c is gridded from W_G + F_G U_GG, U_GG =
+        (R_GG)^-1 the group's diagonal block of U;
+      * F accumulates (w_k - deq_k) R_k,: over the swept columns k.
+    The codes, grids and E_j = (w~_j - deq_j) R_jj are those of gptq_sweep
+    (pinned against it in the tests).  ``block`` only batches the updates of
+    F (in-block rank-1, then one product for the later columns).
+    """
+    W0 = np.array(Wt, dtype=np.float64, copy=True)
+    R = np.asarray(R, dtype=np.float64)
+    rd = np.diag(R).copy()
+    m, n = W0.shape
+    F = np.zeros((m, n))
+    ng = 1 if group == -1 else -(-n // group)
+    codes = np.zeros((m, n), dtype=np.int64)
+    scales = np.zeros((m, ng))
+    zeros = np.zeros((m, ng))
+    Q = np.zeros((m, n))
+    E = np.zeros((m, n))
+    D = np.zeros((m, n))
+    Wcur = np.zeros((m, n))
+    scale = zero = None
+    for b0 in range(0, n, block):
+        b1 = min(n, b0 + block)
+        for j in range(b0, b1):
+            start, g0, g1 = _group_bounds(j, n, group, block)
+            if start:
+                UGG = np.linalg.inv(np.triu(R[g0:g1, g0:g1]))
+                scale, zero = grid_params(W0[:, g0:g1] + F[:, g0:g1] @ np.triu(UGG), bits, asym)
+                gi = 0 if group == -1 else j // group
+                scales[:, gi] = scale
+                zeros[:, gi] = zero
+            w = W0[:, j] + F[:, j] / rd[j]
+            Wcur[:, j] = w
+            q, deq = quantize(w, scale, zero, bits)
+            codes[:, j] = q.astype(np.int64)
+            Q[:, j] = deq
+            E[:, j] = (w - deq) * rd[j]
+            D[:, j] = W0[:, j] - deq
+            F[:, j + 1:b1] += np.outer(D[:, j], R[j, j + 1:b1])
+        F[:, b1:] += D[:, b0:b1] @ R[b0:b1, b1:]
+    return dict(codes=codes, scales=scales, zeros=zeros, Q=Q, E=E, W_final=Wcur)
 
 
 def gptq_sweep_f32(Wt, U, bits: int, group: int, asym: bool = True, block: int = 128):

@@ -10,11 +10,11 @@ from __future__ import annotations
 
 import ctypes
 
-from ._lib import (BF16, BIIP_MODES, F32, ORDERED_FP32, U_GIVEN, WRITE_E, KronqError,
+from ._lib import (BF16, BIIP_MODES, F32, ORDERED_FP32, R_FORM, U_GIVEN, WRITE_E, KronqError,
                    QuantParams, check, lib)
 
 __all__ = [
-    "KronqError", "QuantParams", "U_GIVEN", "ORDERED_FP32", "WRITE_E",
+    "KronqError", "QuantParams", "U_GIVEN", "ORDERED_FP32", "WRITE_E", "R_FORM",
     "kronq_accumulate_factors", "kronq_sensitivity", "kronq_trace_tokens",
     "kronq_sensitivity_from_traces", "kronq_allocate_bits",
     "kronq_allocate_topn_types", "kronq_biip_workspace_bytes", "kronq_biip_forward",

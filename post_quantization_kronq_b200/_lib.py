@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libkronq.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NOT_PD, ERR_TIMEOUT = range(6)
 BF16, F32 = 0, 1
 BIIP_MODES = {"full": 0, "no_rescale": 1, "su_only": 2, "sv_only": 3}
-U_GIVEN, ORDERED_FP32, WRITE_E = 1, 2, 4
+U_GIVEN, ORDERED_FP32, WRITE_E, R_FORM = 1, 2, 4, 8
 
 STATUS_NAMES = {0: "KRONQ_OK", 1: "KRONQ_ERR_INVALID_ARG", 2: "KRONQ_ERR_UNSUPPORTED",
                 3: "KRONQ_ERR_CUDA", 4: "KRONQ_ERR_NOT_PD", 5: "KRONQ_ERR_TIMEOUT"}

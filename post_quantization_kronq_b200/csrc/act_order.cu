@@ -102,7 +102,7 @@ struct ActCarve {
   size_t total;
 };
 
-ActCarve act_carve(void* base, int64_t m, int64_t n, bool with_e) {
+ActCarve act_carve(void* base, int64_t m, int64_t n, bool with_e, bool rform) {
   ActCarve c;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -118,7 +118,7 @@ ActCarve act_carve(void* base, int64_t m, int64_t n, bool with_e) {
   c.rank = static_cast<int*>(take((size_t)n * sizeof(int)));
   c.perm = static_cast<int*>(take((size_t)n * sizeof(int)));
   c.dead = static_cast<uint8_t*>(take((size_t)n));
-  c.inner = take(quantize_core_workspace_bytes(m, n));
+  c.inner = take(quantize_core_workspace_bytes(m, n, rform));
   c.total = (off + 255) & ~size_t(255);
   return c;
 }
@@ -133,7 +133,7 @@ extern "C" {
 size_t kronq_quantize_act_order_workspace_bytes(int64_t m, int64_t n, const kronq_quant_params* p) {
   if (m <= 0 || n <= 0) return 0;
   const bool with_e = p && (p->flags & KRONQ_WRITE_E);
-  return act_carve(nullptr, m, n, with_e).total;
+  return act_carve(nullptr, m, n, with_e, p && (p->flags & KRONQ_R_FORM)).total;
 }
 
 kronq_status kronq_quantize_layer_act_order(float* Wt, float* HX, int64_t m, int64_t n,
@@ -146,7 +146,7 @@ kronq_status kronq_quantize_layer_act_order(float* Wt, float* HX, int64_t m, int
     return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer_act_order: the sweep order comes from H~_X, not from U");
   if (!g_idx) return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer_act_order: g_idx is NULL");
   const bool with_e = (p->flags & KRONQ_WRITE_E) != 0;
-  ActCarve c = act_carve(workspace, m, n, with_e);
+  ActCarve c = act_carve(workspace, m, n, with_e, (p->flags & KRONQ_R_FORM) != 0);
   if (!workspace || ws_bytes < c.total || !aligned(workspace, 256))
     return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer_act_order: workspace too small or not 256-byte aligned");
   cudaStream_t st = as_stream(s);
@@ -165,7 +165,8 @@ kronq_status kronq_quantize_layer_act_order(float* Wt, float* HX, int64_t m, int
   // 3. the plain pass on the permuted problem (already damped)
   r = quantize_core(c.Wp, c.P, m, n, p, c.codes_p, scales, zeros, c.Ep, info, c.inner, st, 2);
   if (r != KRONQ_OK) return r;
-  // 4. outputs back to the original column order; U (of the sweep order) to HX
+  // 4. outputs back to the original column order; U or R (of the sweep
+  //    order) to HX
   unpermute_cols_kernel<float><<<grid, 256, 0, st>>>(c.Wp, m, n, c.perm, Wt);
   KQ_LAUNCH_CHECK("unpermute_cols_kernel");
   unpermute_cols_kernel<uint8_t><<<grid, 256, 0, st>>>(c.codes_p, m, n, c.perm, codes);

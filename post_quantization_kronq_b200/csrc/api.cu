@@ -101,7 +101,7 @@ int64_t quant_gblocks(int64_t n) {
   return nblk < 8 ? (nblk < 1 ? 1 : nblk) : 8;
 }
 
-size_t quant_ws(int64_t m, int64_t n) {
+size_t quant_ws(int64_t m, int64_t n, bool rform) {
   Carver c(nullptr);
   c.take<uint8_t>(chol_workspace_bytes(n));
   c.take<uint8_t>((size_t)n);
@@ -111,8 +111,14 @@ size_t quant_ws(int64_t m, int64_t n) {
   c.take<__nv_bfloat16>((size_t)(m * kg));
   c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
   c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
+  if (rform) {
+    c.take<float>((size_t)(m * n));                        // W~ before the sweep
+    c.take<float>((size_t)(128 * 128 * ceil_div(n, 128)));  // diagonal blocks of U
+  }
   return c.size();
 }
+
+bool wants_rform(const kronq_quant_params* p) { return p && (p->flags & KRONQ_R_FORM) != 0; }
 
 }  // namespace
 }  // namespace kq
@@ -338,6 +344,7 @@ kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64
     if ((r = rowpass(h1, st)) != KRONQ_OK) return r;
     RowPass h2 = h1;
     h2.in = T; h2.out = HX;
+    h2.rowwise = true;   // V F H F V^T is symmetric: no transposed store
     if ((r = rowpass(h2, st)) != KRONQ_OK) return r;
   }
   // H~_G = U D_out^-1 H_G D_out^-1 U^T
@@ -348,6 +355,7 @@ kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64
     if ((r = rowpass(g1, st)) != KRONQ_OK) return r;
     RowPass g2 = g1;
     g2.in = T; g2.out = HG;
+    g2.rowwise = true;
     if ((r = rowpass(g2, st)) != KRONQ_OK) return r;
   }
   return KRONQ_OK;
@@ -389,9 +397,8 @@ kronq_status kronq_biip_inverse(float* W, int64_t m, int64_t n, uint64_t seed, k
 }
 
 size_t kronq_quantize_workspace_bytes(int64_t m, int64_t n, const kronq_quant_params* p) {
-  (void)p;
   if (m <= 0 || n <= 0) return 0;
-  return quant_ws(m, n);
+  return quant_ws(m, n, wants_rform(p));
 }
 
 kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
@@ -400,7 +407,7 @@ kronq_status kronq_quantize_layer(float* Wt, float* HX, int64_t m, int64_t n,
                                   size_t ws_bytes, kronq_stream_t s) {
   kronq_status v = check_quant_args(Wt, HX, m, n, p, codes, scales, zeros, E, info, "quantize_layer");
   if (v != KRONQ_OK) return v;
-  if (!workspace || ws_bytes < quant_ws(m, n) || !aligned(workspace, 256))
+  if (!workspace || ws_bytes < quant_ws(m, n, wants_rform(p)) || !aligned(workspace, 256))
     return fail(KRONQ_ERR_INVALID_ARG, "quantize_layer: workspace too small or not 256-byte aligned");
   const int mode = (p->flags & KRONQ_U_GIVEN) ? 1 : 0;
   return quantize_core(Wt, HX, m, n, p, codes, scales, zeros, E, info, workspace, as_stream(s), mode);
@@ -424,15 +431,19 @@ kronq_status check_quant_args(float* Wt, float* HX, int64_t m, int64_t n, const 
     return fail(KRONQ_ERR_INVALID_ARG, w + ": group must be -1, a divisor of 128 or a multiple of 128");
   if (!(p->damp_rel >= 0.f) || !isfinite(p->damp_rel))
     return fail(KRONQ_ERR_INVALID_ARG, w + ": damp_rel must be finite and >= 0");
-  if (p->flags & ~(KRONQ_U_GIVEN | KRONQ_ORDERED_FP32 | KRONQ_WRITE_E))
+  if (p->flags & ~(KRONQ_U_GIVEN | KRONQ_ORDERED_FP32 | KRONQ_WRITE_E | KRONQ_R_FORM))
     return fail(KRONQ_ERR_INVALID_ARG, w + ": unknown flag");
+  if ((p->flags & KRONQ_R_FORM) && (p->flags & (KRONQ_U_GIVEN | KRONQ_ORDERED_FP32)))
+    return fail(KRONQ_ERR_INVALID_ARG, w + ": KRONQ_R_FORM excludes KRONQ_U_GIVEN and KRONQ_ORDERED_FP32");
+  if ((p->flags & KRONQ_R_FORM) && p->group > 128)
+    return fail(KRONQ_ERR_UNSUPPORTED, w + ": KRONQ_R_FORM takes groups of at most 128 columns (or -1)");
   if ((p->flags & KRONQ_WRITE_E) && !E) return fail(KRONQ_ERR_INVALID_ARG, w + ": KRONQ_WRITE_E needs E");
   if (m > ((int64_t)1 << 31) / 16 || n > ((int64_t)1 << 20))
     return fail(KRONQ_ERR_INVALID_ARG, w + ": size out of range");
   return KRONQ_OK;
 }
 
-size_t quantize_core_workspace_bytes(int64_t m, int64_t n) { return quant_ws(m, n); }
+size_t quantize_core_workspace_bytes(int64_t m, int64_t n, bool rform) { return quant_ws(m, n, rform); }
 
 kronq_status quantize_core(float* Wt, float* HX, int64_t m, int64_t n, const kronq_quant_params* p,
                            uint8_t* codes, float* scales, float* zeros, float* E, int* info,
@@ -447,15 +458,25 @@ kronq_status quantize_core(float* Wt, float* HX, int64_t m, int64_t n, const kro
   __nv_bfloat16* Uh = c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
   __nv_bfloat16* Ul = c.take<__nv_bfloat16>((size_t)(kg * quant_ldu(n)));
   const bool u_given = mode == 1;
+  const bool rform = !u_given && wants_rform(p);
+  float* W0 = rform ? c.take<float>((size_t)(m * n)) : nullptr;
+  float* Ublk = rform ? c.take<float>((size_t)(128 * 128 * ceil_div(n, 128))) : nullptr;
   kronq_status r;
   if (u_given) {
     r = chol_upper_inverse(HX, 0, 0.f, true, nullptr, info, cws, st);  // resets info only
   } else if (mode == 2) {
-    r = chol_upper_inverse(HX, n, 0.f, true, nullptr, info, cws, st);  // already damped
+    r = chol_upper_inverse(HX, n, 0.f, true, nullptr, info, cws, st, !rform);  // already damped
   } else {
-    r = chol_upper_inverse(HX, n, p->damp_rel, false, dead, info, cws, st);
+    r = chol_upper_inverse(HX, n, p->damp_rel, false, dead, info, cws, st, !rform);
   }
   if (r != KRONQ_OK) return r;
+  if (rform) {
+    // W0 = W~, W~ := 0 (it accumulates the feedback F), U's diagonal blocks
+    r = diag_block_inverse(HX, n, Ublk, info, st);
+    if (r != KRONQ_OK) return r;
+    KQ_CUDA(cudaMemcpyAsync(W0, Wt, (size_t)(m * n) * sizeof(float), cudaMemcpyDeviceToDevice, st));
+    KQ_CUDA(cudaMemsetAsync(Wt, 0, (size_t)(m * n) * sizeof(float), st));
+  }
   SweepDesc d;
   d.W = Wt; d.U = HX; d.m = m; d.n = n;
   d.bits = p->bits; d.group = p->group; d.asym = p->asym != 0;
@@ -469,6 +490,8 @@ kronq_status quantize_core(float* Wt, float* HX, int64_t m, int64_t n, const kro
   d.Eh = Eh; d.El = El; d.Uh = Uh; d.Ul = Ul; d.ldu = quant_ldu(n);
   d.lde = kg;
   d.gblocks = (int)quant_gblocks(n);
+  d.W0 = W0;
+  d.Ublk = Ublk;
   return gptq_sweep(d, st);
 }
 

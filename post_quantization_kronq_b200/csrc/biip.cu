@@ -320,12 +320,23 @@ __global__ void __launch_bounds__(RP_THREADS) rowpass_kernel(RPArgs A) {
     }
 
     // 4. transposed store: consecutive threads take consecutive rows of one
-    //    column, so every warp writes R-float runs of the output rows.
+    //    column, so every warp writes R-float runs of the output rows (or,
+    //    row-wise, consecutive threads take consecutive columns of a row).
     const float nrm = p.rotate ? A.norm : 1.f;
     const int tot = L << A.logR;
     const int rr = tid & (R - 1);
     const int jstep = RP_THREADS >> A.logR;
-    if (rr < rows_here) {
+    if (p.rowwise) {
+      for (int q = 0; q < rows_here; ++q) {
+        const float* src = cur + q * RS;
+        float* o = p.out + (r0 + q) * p.ld_out;
+        for (int j = tid; j < L; j += RP_THREADS) {
+          float x = src[padx(j)] * nrm;
+          if (p.inverse) x = x * (F4096 ? cfs[j] : col_factor(p, j));
+          o[j] = x;
+        }
+      }
+    } else if (rr < rows_here) {
       float* o = p.out + (int64_t)(tid >> A.logR) * p.ld_out + r0 + rr;
       const int64_t ostep = (int64_t)jstep * p.ld_out;
       const float* src = cur + rr * RS;
@@ -474,11 +485,38 @@ __global__ void __launch_bounds__(RP_THREADS, 1) rowpass_fast_kernel(RowPass p, 
       fwht_all<K, LOGP, R, 0>(buf);
     }
     // 4. transposed store: consecutive threads take consecutive rows of one
-    //    column (R-float runs of the output rows)
+    //    column (R-float runs of the output rows); row-wise: four
+    //    consecutive columns of a row per thread (16-byte stores)
     const float nrm = p.rotate ? (float)(1.0 / sqrt((double)S::P)) : 1.f;
     const int rr = tid & (R - 1);
     constexpr int JSTEP = RP_THREADS >> S::LOGR;
-    if (rr < rows_here) {
+    if (p.rowwise) {
+      static_assert(S::L % 4 == 0, "row-wise stores take four columns at a time");
+      const bool v4 = (p.ld_out % 4) == 0 && ((reinterpret_cast<uintptr_t>(p.out) & 15) == 0);
+      for (int q = 0; q < rows_here; ++q) {
+        const float* src = buf + q * S::RS;
+        float* o = p.out + (r0 + q) * p.ld_out;
+        for (int j = 4 * tid; j < S::L; j += 4 * RP_THREADS) {
+          // j .. j + 3 sit in one 32-float run of the padded row
+          float4 x = make_float4(src[padx(j)] * nrm, src[padx(j) + 1] * nrm, src[padx(j) + 2] * nrm,
+                                 src[padx(j) + 3] * nrm);
+          if (p.inverse) {
+            x.x *= cf ? cf[j] : col_factor(p, j);
+            x.y *= cf ? cf[j + 1] : col_factor(p, j + 1);
+            x.z *= cf ? cf[j + 2] : col_factor(p, j + 2);
+            x.w *= cf ? cf[j + 3] : col_factor(p, j + 3);
+          }
+          if (v4) {
+            *reinterpret_cast<float4*>(o + j) = x;
+          } else {
+            o[j] = x.x;
+            o[j + 1] = x.y;
+            o[j + 2] = x.z;
+            o[j + 3] = x.w;
+          }
+        }
+      }
+    } else if (rr < rows_here) {
       const float* src = buf + rr * S::RS;
       for (int j = tid >> S::LOGR; j < S::L; j += JSTEP) {
         float x = src[padx(j)] * nrm;
@@ -686,7 +724,9 @@ kronq_status launch_fast(const RowPass& p, cudaStream_t s) {
 template <bool BF16>
 bool try_fast(const RowPass& p, cudaStream_t s, kronq_status& r) {
   switch (p.L) {
-    case 28672: r = launch_cluster<BF16, 7, 12>(p, s); return true;   // Llama-3-70B MLP
+    case 28672:                                                        // Llama-3-70B MLP
+      r = p.rowwise ? launch_fast<BF16, 7, 12, 1>(p, s) : launch_cluster<BF16, 7, 12>(p, s);
+      return true;
     case 14336: r = launch_fast<BF16, 7, 11, 2>(p, s); return true;   // Llama-3-8B MLP
     case 11008: r = launch_fast<BF16, 43, 8, 2>(p, s); return true;   // Llama-2-7B MLP
     case 8192: r = launch_fast<BF16, 1, 13, 4>(p, s); return true;    // Llama-3-70B hidden

@@ -286,7 +286,8 @@ __device__ __forceinline__ void load_chunk(const float* H, int64_t n, int64_t j0
 // ncta: returns false (uniformly over the CTA) when a pivot is not
 // positive, after CTA 0 has recorded info.  256 threads.
 __device__ bool diag_step(DiagSmem& S, float* H, int64_t n, int64_t j0, int nb, int* info,
-                          __nv_bfloat16* splits, float* stage, int vec4, int cta, int ncta) {
+                          __nv_bfloat16* splits, float* stage, float* stage_r, int vec4, int cta,
+                          int ncta) {
   const int tid = threadIdx.x;
   {
     const int tx = tid & 63, ty = tid >> 6;
@@ -312,6 +313,16 @@ __device__ bool diag_step(DiagSmem& S, float* H, int64_t n, int64_t j0, int nb, 
   if (!factor_invert_block(S)) {
     if (tid == 0 && cta == 0) *info = (int)(j0 + S.bad);
     return false;  // uniform: read after the barrier
+  }
+  // CTA 0 stages R_JJ when the factor itself is kept (before U_JJ^T
+  // overwrites it)
+  if (stage_r && cta == 0) {
+    float* dst = stage_r + j0 * NB;
+    for (int t = tid; t < nb * NB; t += blockDim.x) {
+      const int r = t >> 6, c = t & 63;
+      dst[t] = (c >= r) ? S.x.a[r][c] : 0.f;
+    }
+    __syncthreads();
   }
   // U_JJ^T (over R_JJ, no longer needed); CTA 0 stages U_JJ.
   for (int t = tid; t < NB * NB; t += blockDim.x) {
@@ -385,10 +396,10 @@ __device__ bool diag_step(DiagSmem& S, float* H, int64_t n, int64_t j0, int nb, 
 
 __global__ void __launch_bounds__(256) diag_panel_kernel(float* H, int64_t n, int64_t j0, int nb,
                                                          int* info, __nv_bfloat16* splits,
-                                                         float* stage, int vec4) {
+                                                         float* stage, float* stage_r, int vec4) {
   if (*info != 0) return;
   __shared__ DiagSmem S;
-  diag_step(S, H, n, j0, nb, info, splits, stage, vec4, blockIdx.x, gridDim.x);
+  diag_step(S, H, n, j0, nb, info, splits, stage, stage_r, vec4, blockIdx.x, gridDim.x);
 }
 
 // ---------------------------------------------------------------------------
@@ -461,8 +472,9 @@ __device__ __forceinline__ void panel_product(const DiagSmemP& S, int rg, int cg
 // ---- leader CTA: the chain of diagonal blocks -----------------------------
 // On entry S.x.a holds the diagonal block (upper triangle; identity beyond
 // nb), S.u is zero and S.bad is zero.  Factors and inverts it, stages U_JJ
-// (64 x 64 row-major at stage[j0 * 64]) and leaves U_JJ^T in S.y.wk.
-__device__ bool leader_factor(DiagSmemP& S, int64_t j0, int* info, float* stage) {
+// (64 x 64 row-major at stage[j0 * 64]) and, when stage_r is given, R_JJ
+// (at stage_r[j0 * 64]), and leaves U_JJ^T in S.y.wk.
+__device__ bool leader_factor(DiagSmemP& S, int64_t j0, int* info, float* stage, float* stage_r) {
   const int tid = threadIdx.x;
   if (!factor_invert_block(S)) {
     if (tid == 0) *info = (int)(j0 + S.bad);
@@ -471,10 +483,12 @@ __device__ bool leader_factor(DiagSmemP& S, int64_t j0, int* info, float* stage)
   // all 64 x 64 (a short block's identity padding too: the panel CTAs
   // multiply by the whole U_JJ; the staging area has room for it)
   float* dst = stage + j0 * NB;
+  float* dstr = stage_r ? stage_r + j0 * NB : nullptr;
   for (int t = tid; t < NB * NB; t += blockDim.x) {
     const int k = t >> 6, c = t & 63;
     S.y.wk[k][c] = S.u[c][k];
-    dst[t] = S.u[t >> 6][t & 63];
+    dst[t] = S.u[k][c];
+    if (dstr) dstr[t] = (c >= k) ? S.x.a[k][c] : 0.f;
   }
   return true;
 }
@@ -778,6 +792,7 @@ struct PersistArgs {
   int nblk;
   __nv_bfloat16* splits[2];
   float* stage;
+  float* stage_r;   // R_JJ staging (nullptr: only U_JJ)
   int* info;
   int* ctr;     // panel_done, colready, schur_done, uready, diagready (nblk each), abort
   int vec4;
@@ -917,7 +932,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
     for (int J = nblk - 1; J >= 0; --J) {
       const int64_t j0 = (int64_t)J * NB;
       const int nb = (int)((j0 + NB <= n) ? NB : n - j0);
-      if (!leader_factor(F, j0, a.info, a.stage)) {
+      if (!leader_factor(F, j0, a.info, a.stage, a.stage_r)) {
         if (threadIdx.x == 0) atomicExch(abortf, 2);  // stop every other CTA
         break;
       }
@@ -1071,9 +1086,10 @@ cudaError_t status_fetch_chol(int* out, cudaStream_t s) {
 
 static size_t tbuf_bytes(int64_t n) {
   // recursive inverse: products T of the pairs of one level (at most n*n/4
-  // floats); before it, the staged diagonal blocks U_JJ (n x 64 floats)
+  // floats); before it, the staged diagonal blocks U_JJ and R_JJ (n x 64
+  // floats each)
   int64_t f = (n * n) / 4 + n + 64;
-  if (f < n * NB + NB * NB) f = n * NB + NB * NB;
+  if (f < 2 * n * NB + NB * NB) f = 2 * n * NB + NB * NB;
   return (((size_t)f * sizeof(float)) + 255) & ~size_t(255);
 }
 
@@ -1101,7 +1117,7 @@ kronq_status damp_factor(float* H, int64_t n, float damp_rel, uint8_t* dead, int
 }
 
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
-                                uint8_t* dead, int* info, void* ws, cudaStream_t s) {
+                                uint8_t* dead, int* info, void* ws, cudaStream_t s, bool want_u) {
   if (!skip_damp) {
     damp_kernel<<<1, 1024, 0, s>>>(H, n, damp_rel, dead, info);
     KQ_LAUNCH_CHECK("damp_kernel");
@@ -1110,12 +1126,13 @@ kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_d
     KQ_LAUNCH_CHECK("zero_info_kernel");
   }
   if (n <= 0) return KRONQ_OK;
-  if (n > kOuterBlock) return chol_blocked(H, n, info, ws, s);
-  return chol_core(H, n, info, ws, s);
+  if (n > kOuterBlock) return chol_blocked(H, n, info, ws, s, want_u);
+  return chol_core(H, n, info, ws, s, want_u);
 }
 
-kronq_status chol_core(float* H, int64_t n, int* info, void* ws, cudaStream_t s) {
+kronq_status chol_core(float* H, int64_t n, int* info, void* ws, cudaStream_t s, bool want_u) {
   float* Tbuf = reinterpret_cast<float*>(ws);
+  float* stage_r = want_u ? nullptr : Tbuf + n * NB;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   __nv_bfloat16* splits = reinterpret_cast<__nv_bfloat16*>(wsb + tbuf_bytes(n));
   __nv_bfloat16* splits1 = reinterpret_cast<__nv_bfloat16*>(wsb + tbuf_bytes(n) + splits_bytes(n));
@@ -1158,6 +1175,7 @@ kronq_status chol_core(float* H, int64_t n, int* info, void* ws, cudaStream_t s)
     pa.splits[0] = splits;
     pa.splits[1] = splits1;
     pa.stage = Tbuf;
+    pa.stage_r = stage_r;
     pa.info = info;
     pa.ctr = ctr;
     pa.vec4 = vec4;
@@ -1175,13 +1193,25 @@ kronq_status chol_core(float* H, int64_t n, int* info, void* ws, cudaStream_t s)
     // of panel rows per CTA where that suffices.
     int64_t pg = j0 > 0 ? ceil_div(j0, PR) : 1;
     if (pg > pmax) pg = pmax;
-    diag_panel_kernel<<<(unsigned)pg, 256, 0, s>>>(H, n, j0, nb, info, splits, Tbuf, vec4);
+    diag_panel_kernel<<<(unsigned)pg, 256, 0, s>>>(H, n, j0, nb, info, splits, Tbuf, stage_r, vec4);
     KQ_LAUNCH_CHECK("diag_panel_kernel");
     if (j0 == 0) break;
     kronq_status r = schur_update_tc(&maps, H, n, j0, info, s);
     if (r != KRONQ_OK) return r;
   }
-  diag_store_kernel<<<(unsigned)nblk, 256, 0, s>>>(H, n, Tbuf, info);
+  if (!want_u) {
+    // R: its diagonal blocks R_JJ from the staging, the blocks above them
+    // already hold R.  The staged U_JJ stay for chol_core_finish_u.
+    diag_store_kernel<<<(unsigned)nblk, 256, 0, s>>>(H, n, stage_r, info);
+    KQ_LAUNCH_CHECK("diag_store_kernel");
+    return KRONQ_OK;
+  }
+  return chol_core_finish_u(H, n, info, ws, s);
+}
+
+kronq_status chol_core_finish_u(float* H, int64_t n, int* info, void* ws, cudaStream_t s) {
+  float* Tbuf = reinterpret_cast<float*>(ws);
+  diag_store_kernel<<<(unsigned)ceil_div(n, NB), 256, 0, s>>>(H, n, Tbuf, info);
   KQ_LAUNCH_CHECK("diag_store_kernel");
   return chol_inverse_levels(H, n, NB, Tbuf, info, s);
 }

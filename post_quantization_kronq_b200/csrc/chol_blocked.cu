@@ -21,7 +21,10 @@
 //      next block can read its rows left of the diagonal.
 //
 // Finally the off-diagonal blocks of U come from the recursive two-block
-// formula level by level, starting from the B x B diagonal blocks.
+// formula level by level, starting from the B x B diagonal blocks.  When R
+// itself is wanted (the sweep's R form), step 1 keeps R_JJ in the diagonal
+// block (U_JJ, still needed by step 2, is formed in the contiguous copy) and
+// the last stage is skipped: the upper triangle then holds R.
 //
 // Compared with one chain of 64-wide steps over the whole order, each
 // element of the trailing matrix goes through HBM once per B columns
@@ -398,7 +401,7 @@ size_t chol_blocked_workspace_bytes(int64_t n) {
          chol_core_workspace_bytes(B) + 256;
 }
 
-kronq_status chol_blocked(float* H, int64_t n, int* info, void* ws, cudaStream_t s) {
+kronq_status chol_blocked(float* H, int64_t n, int* info, void* ws, cudaStream_t s, bool want_u) {
   const int64_t B = kOuterBlock;
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* Tbuf = reinterpret_cast<float*>(w);
@@ -425,13 +428,18 @@ kronq_status chol_blocked(float* H, int64_t n, int* info, void* ws, cudaStream_t
     copy_block_kernel<<<copy_grid, 256, 0, s>>>(Sbuf, nb, H + j0 * n + j0, n, nb, nb, 1, info);
     KQ_LAUNCH_CHECK("copy_block_kernel");
     KQ_CUDA(cudaMemsetAsync(info_local, 0, sizeof(int), s));
-    kronq_status r = chol_core(Sbuf, nb, info_local, core_ws, s);
+    // (for R: R_JJ first, copied out, then turned into U_JJ for step 2)
+    kronq_status r = chol_core(Sbuf, nb, info_local, core_ws, s, want_u);
     if (r != KRONQ_OK) return r;
     merge_info_kernel<<<1, 1, 0, s>>>(info, info_local, j0);
     KQ_LAUNCH_CHECK("merge_info_kernel");
     copy_block_kernel<<<copy_grid, 256, 0, s>>>(H + j0 * n + j0, n, Sbuf, nb, nb, nb, 1, info);
     KQ_LAUNCH_CHECK("copy_block_kernel");
     if (j0 == 0) break;
+    if (!want_u) {
+      r = chol_core_finish_u(Sbuf, nb, info_local, core_ws, s);
+      if (r != KRONQ_OK) return r;
+    }
     // 2. T = U_JJ A[J, 0:j0]  (nb x j0)
     TriGemm t;
     t.M = nb; t.N = j0; t.K = nb;
@@ -466,6 +474,7 @@ kronq_status chol_blocked(float* H, int64_t n, int* info, void* ws, cudaStream_t
     schur_k_kernel<<<(unsigned)grid, SK_THREADS, SK_SMEM, s>>>(maps[0], maps[1], maps[2], a);
     KQ_LAUNCH_CHECK("schur_k_kernel");
   }
+  if (!want_u) return KRONQ_OK;   // R: the diagonal blocks R_JJ and R above them
   return chol_inverse_levels(H, n, B, Tbuf, info, s);
 }
 

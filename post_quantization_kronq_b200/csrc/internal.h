@@ -104,6 +104,10 @@ struct RowPass {
   bool inverse = false;
   uint64_t sign_state = 0;  // 2 * seed + side
   float* cf = nullptr;      // optional scratch of L floats for the column factors
+  // false: out = the transformed rows, transposed (out[j * ld_out + row]);
+  // true: stored as rows (out[row * ld_out + j]), for a result that is
+  // symmetric anyway (the second pass of V F H F V^T)
+  bool rowwise = false;
 };
 kronq_status rowpass(const RowPass& p, cudaStream_t s);
 // sum of squares along columns (colsq[n]) and rows (rowsq[m]) of W.
@@ -125,8 +129,10 @@ kronq_status schur_maps(SchurMaps* sm, const __nv_bfloat16* splits, float* H, in
 kronq_status schur_update_tc(const SchurMaps* sm, float* H, int64_t n, int64_t j0, const int* info,
                              cudaStream_t s);
 cudaError_t status_fetch_schur(int* out, cudaStream_t s);
-// In: H (n x n) full symmetric.  Out: U (upper) with U^T U = (H + lambda I)^-1,
-// dead-column flags, info.  ws: see chol_workspace_bytes.
+// In: H (n x n) full symmetric.  Out (upper triangle): U with U^T U =
+// (H + lambda I)^-1, or with want_u false the factor R = U^-1 itself
+// (H + lambda I = R R^T, R upper); dead-column flags, info.  ws: see
+// chol_workspace_bytes.
 size_t chol_workspace_bytes(int64_t n);
 // Above this order the factorisation is blocked in two levels (chol_blocked).
 constexpr int64_t kOuterBlock = 4096;
@@ -134,21 +140,24 @@ constexpr int64_t kOuterBlock = 4096;
 // info untouched unless a pivot fails) and its workspace.
 size_t chol_core_workspace_bytes(int64_t n);
 size_t chol_tbuf_bytes(int64_t n);
-kronq_status chol_core(float* H, int64_t n, int* info, void* ws, cudaStream_t s);
+// want_u false: R instead of U (the diagonal blocks U_JJ stay staged in ws,
+// and chol_core_finish_u then turns R into U in place).
+kronq_status chol_core(float* H, int64_t n, int* info, void* ws, cudaStream_t s, bool want_u = true);
+kronq_status chol_core_finish_u(float* H, int64_t n, int* info, void* ws, cudaStream_t s);
 // U = R^-1 from the diagonal blocks U_JJ of size S0 (aligned from the top)
 // and the off-diagonal blocks of R, level by level (tensor-core products).
 kronq_status chol_inverse_levels(float* H, int64_t n, int64_t S0, float* Tbuf, const int* info,
                                  cudaStream_t s);
 // Two-level blocked factorisation for n > kOuterBlock (after damping).
 size_t chol_blocked_workspace_bytes(int64_t n);
-kronq_status chol_blocked(float* H, int64_t n, int* info, void* ws, cudaStream_t s);
+kronq_status chol_blocked(float* H, int64_t n, int* info, void* ws, cudaStream_t s, bool want_u = true);
 cudaError_t status_fetch_schurk(int* out, cudaStream_t s);
 // One CTA whose bounded wait (which 0: mbarrier, 1: cross-CTA counter) is
 // never satisfied; gives up after limit_ns.  w: 3 device ints.
 kronq_status wait_selftest(int which, unsigned long long limit_ns, int* w, cudaStream_t s);
 cudaError_t status_fetch_chol(int* out, cudaStream_t s);
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
-                                uint8_t* dead, int* info, void* ws, cudaStream_t s);
+                                uint8_t* dead, int* info, void* ws, cudaStream_t s, bool want_u = true);
 
 // ------------------------------------------------------------ sweep
 // Storage for the four TMA descriptors of the tensor-core trailing update
@@ -194,13 +203,27 @@ struct SweepDesc {
   int64_t ldu = 0;
   int64_t lde = 128;
   int gblocks = 1;
+  // R form (not with ordered; groups of at most 128 columns, or one per
+  // row): U points at R (upper, H~ = R R^T) and U = R^-1 is not formed.
+  // W holds the feedback F = (W0 - Q)_done R_done,: (zero at the start),
+  // W0 the weights before the sweep, Ublk the 128 x 128 diagonal blocks
+  // U_GG = (R_GG)^-1 (block b at rows 128 b .., row stride 128).  A block
+  // starts from W0_G + F_G U_GG (GPTQ's partial state of its columns) and is
+  // swept on U_GG as in the U form; its later columns then get F += (W0 -
+  // Q)_G R_G,later.
+  const float* W0 = nullptr;
+  const float* Ublk = nullptr;
 };
 kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s);
+// The 128 x 128 diagonal blocks of U = R^-1 for the R form (ceil(n / 128)
+// blocks of 128 x 128 floats, row stride 128).
+kronq_status diag_block_inverse(const float* R, int64_t n, float* Ublk, const int* info, cudaStream_t s);
 
 // The body of kronq_quantize_layer after validation.  mode 0: dead columns,
 // damping and factorisation of HX; 1: HX holds U already; 2: HX is damped
-// already (no dead-column rule), factorisation only.
-size_t quantize_core_workspace_bytes(int64_t m, int64_t n);
+// already (no dead-column rule), factorisation only.  KRONQ_R_FORM in the
+// flags (modes 0 and 2): the factor is left as R and the sweep runs on it.
+size_t quantize_core_workspace_bytes(int64_t m, int64_t n, bool rform);
 kronq_status check_quant_args(float* Wt, float* HX, int64_t m, int64_t n, const kronq_quant_params* p,
                               uint8_t* codes, float* scales, float* zeros, float* E, int* info,
                               const char* who);

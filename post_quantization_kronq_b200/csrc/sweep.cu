@@ -30,6 +30,16 @@
 // After each block the later columns get W[:, later] -= E_blk U[blk, later]
 // (the lazy-batch update), either as a fast GEMM or, in the ordered test mode,
 // with one rounding per product and per sum in ascending k.
+//
+// R form (SweepDesc::W0 set): the factor is R (H~ = R R^T) and only the
+// diagonal blocks U_GG = (R_GG)^-1 of U = R^-1 are formed.  For the swept
+// columns S and the rest T, GPTQ's partial state W_T - E_S U_ST equals
+// W_T + F U_TT with F = (W0 - Q)_S R_ST, since E_S = (W0 - Q)_S R_SS and
+// R_SS U_ST = -R_ST U_TT.  W then holds F; a block G starts from
+// W0_G + F_G U_GG (its columns' partial state, from which GPTQ grids the
+// group), is swept on U_GG exactly as in the U form, and hands
+// D = deq - W0 of its columns to the trailing update with R's rows:
+// F_later -= D_G R_G,later.
 #include "common.cuh"
 #include "internal.h"
 
@@ -53,6 +63,10 @@ constexpr int ROWS_PER_CTA = WARPS * 32 / LPR * 2;   // 32
 constexpr int UP_LD = 18;
 constexpr int UP_ROW = LPR * UP_LD;
 constexpr int SWEEP_SMEM = (BW * UP_ROW + BW) * (int)sizeof(float);
+// R form: the CTA's rows of W0 for the block (odd stride: the four rows a
+// warp reads at once sit in distinct banks) and the diagonal of U_GG
+constexpr int W0_LD = BW + 1;
+constexpr int RF_SMEM = SWEEP_SMEM + (ROWS_PER_CTA * W0_LD + BW) * (int)sizeof(float);
 constexpr int UB_PER_THREAD = (BW * BW / 4) / (WARPS * 32);   // float4 loads of the U block
 
 struct BlockArgs {
@@ -183,13 +197,19 @@ __device__ __forceinline__ void split4(float4 x, __nv_bfloat16* dh, __nv_bfloat1
 // With groups of 32 columns or more the grid is fixed within a round: the
 // owner keeps the rounded quotient and the error and the outputs are formed
 // when the round retires; otherwise the owner keeps deq and the code.
-template <bool ORD, int GM>
+template <bool ORD, int GM, bool RF>
 __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a) {
+  static_assert(!(ORD && RF), "the ordered mode takes U");
   constexpr bool PERCOL = (GM == 15 || GM == -2);
   const SweepDesc& d = a.d;
   extern __shared__ __align__(16) float smem[];
   float* Up = smem;
   float* iu = smem + BW * UP_ROW;
+  float* w0s = iu + BW;                 // R form only
+  float* ud = w0s + ROWS_PER_CTA * W0_LD;
+  // the in-block factor: U's rows j0 .. (U form) or the diagonal block U_GG
+  const float* ublk = RF ? d.Ublk + a.j0 * BW : d.U + a.j0 * d.n + a.j0;
+  const int64_t ldub = RF ? BW : d.n;
   const int tid = threadIdx.x, lane = tid & 31;
   const int q = lane & (LPR - 1);
   const int64_t n = d.n, j0 = a.j0;
@@ -197,6 +217,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
   const int64_t r0 = (int64_t)blockIdx.x * ROWS_PER_CTA + (tid >> 4) * 2;   // rows r0, r0 + 1
   const bool live[2] = {r0 < d.m, r0 + 1 < d.m};
   const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(d.U) & 15) == 0);
+  const bool uvec = RF || vec;
   const int64_t j1 = j0 + bw;
 
   // Issue every load of the block's inputs first: the U block (16-byte
@@ -211,8 +232,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
     const int k = idx >> 5, c = (idx & 31) * 4;
     ub[it] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (k < bw && c < bw) {
-      const float* src = d.U + (j0 + k) * n + j0 + c;
-      if (vec) {
+      const float* src = ublk + k * ldub + c;
+      if (uvec) {
         ub[it] = *reinterpret_cast<const float4*>(src);
       } else {
         ub[it].x = src[0];
@@ -222,7 +243,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
       }
     }
   }
-  const float udiag = (tid < bw) ? d.U[(j0 + tid) * n + j0 + tid] : 1.f;
+  const float udiag = (tid < bw) ? ublk[tid * ldub + tid] : 1.f;
   float2 v[2][NP];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -231,6 +252,18 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
     for (int p = 0; p < NP; ++p) {
       const int c0 = 32 * p + q, c1 = c0 + 16;
       v[h][p] = make_float2((live[h] && c0 < bw) ? wrow[c0] : 0.f, (live[h] && c1 < bw) ? wrow[c1] : 0.f);
+    }
+  }
+  float2 w0v[2][NP];   // R form: the weights before the sweep
+  if (RF) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float* wrow = d.W0 + (r0 + h) * n + j0;
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const int c0 = 32 * p + q, c1 = c0 + 16;
+        w0v[h][p] = make_float2((live[h] && c0 < bw) ? wrow[c0] : 0.f, (live[h] && c1 < bw) ? wrow[c1] : 0.f);
+      }
     }
   }
   // The tensor-core trailing update reads bf16 hi/lo copies of this block's
@@ -256,6 +289,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
       for (int h = 0; h < 2; ++h) {
         if (z0) v[h][p].x = 0.f;
         if (z1) v[h][p].y = 0.f;
+        if (RF && z0) w0v[h][p].x = 0.f;
+        if (RF && z1) w0v[h][p].y = 0.f;
       }
     }
   }
@@ -278,6 +313,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
     *reinterpret_cast<float2*>(Up + row * UP_LD + NREG + 2 * p) = make_float2(0.f, 0.f);
   }
   if (tid < BW) iu[tid] = (tid < bw) ? __frcp_rn(udiag) : 0.f;
+  if (RF) {
+    if (tid < BW) ud[tid] = (tid < bw) ? udiag : 0.f;
+    const int rl0 = (tid >> 4) * 2;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        w0s[(rl0 + h) * W0_LD + 32 * p + q] = w0v[h][p].x;
+        w0s[(rl0 + h) * W0_LD + 32 * p + q + 16] = w0v[h][p].y;
+      }
+  }
 
   if (split_fast) {
     const int64_t k = blockIdx.x;
@@ -322,6 +368,38 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
   __syncthreads();
 
   const int src_base = lane & ~(LPR - 1);
+  if (RF) {
+    // the block's partial state: W0_G + F_G U_GG (F in v): the diagonal
+    // term, then every row t of U_GG's strictly upper part
+    float2 acc[2][NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const float2 dg = make_float2(ud[32 * p + q], ud[32 * p + q + 16]);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) acc[h][p] = __ffma2_rn(v[h][p], dg, w0v[h][p]);
+    }
+#pragma unroll
+    for (int kk = 0; kk < NREG; ++kk) {          // row t = 16 kk + o of U_GG, F_t from lane o
+#pragma unroll 4
+      for (int o = 0; o < LPR; ++o) {
+        const int t = LPR * kk + o;
+        const float2* u2 = reinterpret_cast<const float2*>(Up + (t * LPR + q) * UP_LD);
+        float ft[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) ft[h] = __shfl_sync(0xffffffffu, reg_of(v[h], kk), src_base + o);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const float2 u = u2[p];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) acc[h][p] = __ffma2_rn(make_float2(ft[h], ft[h]), u, acc[h][p]);
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int p = 0; p < NP; ++p) v[h][p] = acc[h][p];
+  }
   // the windows: columns 0 and 1 (register 0 of lanes 0 and 1)
   float win[2][2];
 #pragma unroll
@@ -414,10 +492,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sweep_block_kernel(BlockArgs a)
         d.codes[r * n + j0 + col] = (uint8_t)code;
         if (a.Eb) a.Eb[r * a.lde + col] = e;
         if (!ORD) {
-          const __nv_bfloat16 hb = __float2bfloat16_rn(e);
+          // the trailing update's left operand: e (U form) or deq - w0
+          const float et = RF ? __fsub_rn(deq, w0s[((tid >> 4) * 2 + h) * W0_LD + col]) : e;
+          const __nv_bfloat16 hb = __float2bfloat16_rn(et);
           const int64_t eo = r * d.lde + (int64_t)a.slot * BW + col;
           d.Eh[eo] = hb;
-          d.El[eo] = __float2bfloat16_rn(e - __bfloat162float(hb));
+          d.El[eo] = __float2bfloat16_rn(et - __bfloat162float(hb));
         }
       }
     }
@@ -439,8 +519,9 @@ __global__ void group_params_kernel(SweepDesc d, int64_t j0, int64_t gw, int64_t
   if (r >= d.m) return;
   float lo = INFINITY, hi = -INFINITY;
   const int64_t j1 = (j0 + gw < d.n) ? j0 + gw : d.n;
+  const float* src = d.W0 ? d.W0 : d.W;   // R form: only at column 0, where F = 0
   for (int64_t j = j0 + lane; j < j1; j += 32) {
-    float x = d.W[r * d.n + j];
+    float x = src[r * d.n + j];
     if (d.dead && d.dead[j]) x = 0.f;
     lo = fminf(lo, x);
     hi = fmaxf(hi, x);
@@ -457,33 +538,79 @@ __global__ void group_params_kernel(SweepDesc d, int64_t j0, int64_t gw, int64_t
   }
 }
 
-template <bool ORD, int GM>
+template <bool ORD, int GM, bool RF>
 cudaError_t launch_gm(const BlockArgs& a, unsigned grid, cudaStream_t s) {
-  const void* fn = reinterpret_cast<const void*>(&sweep_block_kernel<ORD, GM>);
-  cudaError_t e = allow_smem(fn, SWEEP_SMEM);
+  const void* fn = reinterpret_cast<const void*>(&sweep_block_kernel<ORD, GM, RF>);
+  const int smem = RF ? RF_SMEM : SWEEP_SMEM;
+  cudaError_t e = allow_smem(fn, smem);
   if (e != cudaSuccess) return e;
-  sweep_block_kernel<ORD, GM><<<grid, WARPS * 32, SWEEP_SMEM, s>>>(a);
+  sweep_block_kernel<ORD, GM, RF><<<grid, WARPS * 32, smem, s>>>(a);
   count_launch();
   return cudaGetLastError();
 }
 
 // Picks the instance for the block's group layout.
-template <bool ORD>
+template <bool ORD, bool RF>
 cudaError_t launch_block(const BlockArgs& a, unsigned grid, cudaStream_t s) {
-  if (a.wide) return launch_gm<ORD, -1>(a, grid, s);
+  if (a.wide) return launch_gm<ORD, -1, RF>(a, grid, s);
   switch (a.d.group) {
-    case 128: return launch_gm<ORD, 127>(a, grid, s);
-    case 64: return launch_gm<ORD, 63>(a, grid, s);
-    case 32: return launch_gm<ORD, 31>(a, grid, s);
-    case 16: return launch_gm<ORD, 15>(a, grid, s);
-    default: return launch_gm<ORD, -2>(a, grid, s);
+    case 128: return launch_gm<ORD, 127, RF>(a, grid, s);
+    case 64: return launch_gm<ORD, 63, RF>(a, grid, s);
+    case 32: return launch_gm<ORD, 31, RF>(a, grid, s);
+    case 16: return launch_gm<ORD, 15, RF>(a, grid, s);
+    default: return launch_gm<ORD, -2, RF>(a, grid, s);
   }
+}
+
+// U_GG = (R_GG)^-1 for the 128 x 128 diagonal blocks of R (one CTA of 128
+// threads per block; the last block padded with the identity): thread c
+// forms column c by back substitution in float64, u_cc = 1 / R_cc and
+// u_ic = -(sum_{k = i+1 .. c} R_ik u_kc) / R_ii for i = c - 1 .. 0, and
+// rounds it to float once.  Out: Ublk[(128 b + i) * 128 + c], zero below the
+// diagonal.
+constexpr int DBI_LD = BW + 1;
+constexpr int DBI_SMEM = BW * DBI_LD * (int)(sizeof(float) + sizeof(double));
+
+__global__ void __launch_bounds__(BW) diag_block_inverse_kernel(const float* R, int64_t n, float* Ublk,
+                                                                const int* info) {
+  if (info && *info != 0) return;
+  extern __shared__ __align__(16) unsigned char dbi_raw[];
+  double* sU = reinterpret_cast<double*>(dbi_raw);
+  float* sR = reinterpret_cast<float*>(sU + BW * DBI_LD);
+  const int64_t j0 = (int64_t)blockIdx.x * BW;
+  const int bw = (int)((n - j0) < BW ? (n - j0) : BW);
+  const int c = threadIdx.x;
+  for (int r = 0; r < BW; ++r) {
+    float x = (r == c) ? 1.f : 0.f;
+    if (r < bw && c < bw) x = (c >= r) ? R[(j0 + r) * n + j0 + c] : 0.f;
+    sR[r * DBI_LD + c] = x;
+  }
+  __syncthreads();
+  sU[c * DBI_LD + c] = 1.0 / (double)sR[c * DBI_LD + c];
+  for (int i = c - 1; i >= 0; --i) {
+    double acc = 0.0;
+    for (int k = i + 1; k <= c; ++k) acc = fma((double)sR[i * DBI_LD + k], sU[k * DBI_LD + c], acc);
+    sU[i * DBI_LD + c] = -acc / (double)sR[i * DBI_LD + i];
+  }
+  for (int r = 0; r < BW; ++r) Ublk[(j0 + r) * BW + c] = (r <= c) ? (float)sU[r * DBI_LD + c] : 0.f;
 }
 
 }  // namespace
 
+kronq_status diag_block_inverse(const float* R, int64_t n, float* Ublk, const int* info, cudaStream_t s) {
+  if (n <= 0) return KRONQ_OK;
+  const void* fn = reinterpret_cast<const void*>(&diag_block_inverse_kernel);
+  cudaError_t e = allow_smem(fn, DBI_SMEM);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(diag_block_inverse)");
+  diag_block_inverse_kernel<<<(unsigned)ceil_div(n, BW), BW, DBI_SMEM, s>>>(R, n, Ublk, info);
+  KQ_LAUNCH_CHECK("diag_block_inverse_kernel");
+  return KRONQ_OK;
+}
+
 kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
   const int64_t n = d.n, m = d.m;
+  if (d.W0 && (d.ordered || !d.Ublk || d.group > BW))
+    return fail(KRONQ_ERR_INVALID_ARG, "sweep: the R form takes groups of at most 128 columns, no ordered mode");
   const unsigned grid = (unsigned)ceil_div(m, ROWS_PER_CTA);
   TrailingMaps maps;
   if (!d.ordered && n > BW) {
@@ -520,7 +647,9 @@ kronq_status gptq_sweep(const SweepDesc& d, cudaStream_t s) {
       a.Eb = nullptr;   // the tensor-core update reads the bf16 hi/lo copies
       a.lde = BW;
     }
-    cudaError_t el = d.ordered ? launch_block<true>(a, grid, s) : launch_block<false>(a, grid, s);
+    cudaError_t el = d.ordered ? launch_block<true, false>(a, grid, s)
+                               : (d.W0 ? launch_block<false, true>(a, grid, s)
+                                       : launch_block<false, false>(a, grid, s));
     if (el != cudaSuccess) return cuda_fail(el, "sweep_block_kernel");
     const int64_t j1 = j0 + bw;
     if (j1 < n && !d.ordered) {

@@ -10,15 +10,22 @@ from __future__ import annotations
 
 import torch
 
-from . import (QuantParams, kronq_accumulate_factors, kronq_biip_forward,
+from . import (R_FORM, QuantParams, kronq_accumulate_factors, kronq_biip_forward,
                kronq_biip_workspace_bytes, kronq_pack, kronq_quantize_layer,
                kronq_quantize_workspace_bytes, kronq_sensitivity, words_per_row, workspace)
 
 
 class LayerPass:
+    """flags: the kronq_quant_params flags; None picks KRONQ_R_FORM (the sweep
+    on the factor R, no inverse formed; HX holds R after quantize) wherever it
+    applies (groups of at most 128 columns or one per row), else 0 (HX holds
+    U after quantize)."""
+
     def __init__(self, m: int, n: int, bits: int = 4, group: int = 128, asym: bool = True,
                  damp_rel: float = 0.01, seed: int = 0, alpha: float = 0.25, mode: str = "full",
-                 flags: int = 0, device="cuda"):
+                 flags: int | None = None, device="cuda"):
+        if flags is None:
+            flags = R_FORM if (group == -1 or group <= 128) else 0
         self.m, self.n, self.bits, self.group = m, n, bits, group
         self.seed, self.alpha, self.mode = seed, alpha, mode
         dev = torch.device(device)

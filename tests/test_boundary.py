@@ -62,6 +62,9 @@ def _qp(**kw):
     (dict(damp_rel=float("nan")), _lib.ERR_INVALID_ARG),
     (dict(flags=64), _lib.ERR_INVALID_ARG),
     (dict(flags=_lib.WRITE_E), _lib.ERR_INVALID_ARG),   # E is NULL below
+    (dict(flags=_lib.R_FORM | _lib.U_GIVEN), _lib.ERR_INVALID_ARG),
+    (dict(flags=_lib.R_FORM | _lib.ORDERED_FP32), _lib.ERR_INVALID_ARG),
+    (dict(flags=_lib.R_FORM, group=256), _lib.ERR_UNSUPPORTED),
 ])
 def test_quantize_layer_validation(kw, status):
     p = _qp(**kw)
@@ -82,6 +85,21 @@ def test_quantize_layer_null_and_workspace():
     r = _lib.lib.kronq_quantize_layer(FAKE, FAKE, 0, 256, ctypes.byref(p), FAKE, FAKE, FAKE, None,
                                       FAKE, FAKE, need, None)
     assert _st(r) == _lib.ERR_INVALID_ARG
+
+
+def test_r_form_workspace():
+    # the R form keeps a copy of W~ (m n floats) and U's 128 x 128 diagonal
+    # blocks (ceil(n / 128) of them) on top
+    for m, n in [(64, 256), (1000, 4500), (8192, 28672)]:
+        base = _lib.lib.kronq_quantize_workspace_bytes(m, n, ctypes.byref(_qp()))
+        rf = _lib.lib.kronq_quantize_workspace_bytes(m, n, ctypes.byref(_qp(flags=_lib.R_FORM)))
+        extra = rf - base
+        want = 4 * (m * n + 128 * 128 * (-(-n // 128)))
+        assert want <= extra <= want + 512
+        p = _qp(flags=_lib.R_FORM)
+        r = _lib.lib.kronq_quantize_layer(FAKE, FAKE, m, n, ctypes.byref(p), FAKE, FAKE, FAKE, None,
+                                          FAKE, FAKE, rf - 1, None)
+        assert _st(r) == _lib.ERR_INVALID_ARG
 
 
 def test_accumulate_validation():

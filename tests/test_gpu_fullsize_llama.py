@@ -18,23 +18,24 @@ can compute piece by piece, fed the GPU's output of the previous stage:
   the GPU factor's diagonal;
 * BiIP: the rescale vectors, and sampled rows of W~, H~_X and H~_G (rows of
   the oracle's rotations times the rescaled inputs, then the rotation);
-* the factor U: against the oracle's U of the GPU's damped H~_X (for
-  n = 28672 its trailing 4096 x 4096 block, which the reverse factorisation
-  computes from that block of H alone, and U^T U A e_j = e_j on sampled
-  columns j), within twice the error of a float32 LAPACK factorisation of
-  the same matrix -- float32 is the precision of the kernels, and its error
-  grows with the condition number (1e5 and more for the rectified down_proj
-  inputs);
-* the sweep: 64 sampled rows of the GPU's W~ through the float64 sweep
-  given the GPU's U (codes within 0.5 %), and end to end against the
-  oracle's U: codes within 0.5 %, or within 1.5 x the disagreement that the
-  float32 LAPACK factor alone causes when that is larger; the rows'
-  quadratic error within 1 %.
+* the factor: the layer pass runs the sweep on R (H~_X + lambda I = R R^T,
+  the default R form), so HX returns R; against the float64 R of the GPU's
+  damped H~_X (for n = 28672 its trailing 4096 x 4096 block, which the
+  reverse factorisation computes from that block of H alone, and
+  R R^T e_j = A e_j on sampled columns j), within twice the error of a
+  float32 LAPACK factorisation of the same matrix -- float32 is the
+  precision of the kernels, and its error grows with the condition number
+  (1e5 and more for the rectified down_proj inputs);
+* the sweep: 64 sampled rows of the GPU's W~ through the oracle's float64
+  R-form sweep given the GPU's R (codes within 0.5 %), and end to end
+  against the oracle's U-form sweep on its own U: codes within 0.5 %, or
+  within 1.5 x the disagreement that a float32 LAPACK factor alone causes
+  when that is larger; the rows' quadratic error within 1 %.
 """
 import numpy as np
 import pytest
+import scipy.linalg as sl
 import torch
-from scipy.linalg import solve_triangular
 
 from oracle import biip, factors, sweep
 from post_quantization_kronq_b200.layer import LayerPass
@@ -83,6 +84,12 @@ def _rotation_rows(rows, L, seed, side):
     E = np.zeros((len(rows), L))
     E[np.arange(len(rows)), rows] = 1.0
     return biip.rotate_rows(E, seed, side, inverse=True)
+
+
+def reverse_chol(A, dtype):
+    """R upper with A = R R^T (LAPACK on the index-reversed matrix)."""
+    L = sl.cholesky(np.ascontiguousarray(np.asarray(A, dtype)[::-1, ::-1]), lower=True, check_finite=False)
+    return np.ascontiguousarray(L[::-1, ::-1]).astype(np.float64)
 
 
 def _u_times(U, V, chunk=2048, transpose=False):
@@ -148,22 +155,23 @@ def test_llama_mlp_full_size_sampled(case):
     del HX, HG
     torch.cuda.empty_cache()
 
-    # ---- the factor U of the damped H~_X, held to the float32 floor: the
+    # ---- the factor R of the damped H~_X, held to the float32 floor: the
     # error of a float32 LAPACK factorisation of the same matrix (it grows
     # with the condition number; rectified down_proj inputs give a large
     # common mean and condition numbers of 1e5 and more)
     hxt_diag = to_np(torch.diagonal(HXt))
     dead = hxt_diag == 0
     lam = 0.01 * float(np.mean(np.where(dead, 1.0, hxt_diag)))
-    Ug = np.triu(to_np(lp.HX))
-    U = U32 = None
+    Rg = np.triu(to_np(lp.HX))
+    U = U32 = R64 = None
     if n <= 11008:
         H1, _, _ = sweep.dead_columns(to_np(HXt), np.zeros((1, n)))
         A, _ = sweep.damp(H1, 0.01)
+        R64 = reverse_chol(A, np.float64)
+        e_gpu, e_32 = rel(Rg, R64), rel(reverse_chol(A, np.float32), R64)
+        assert e_gpu <= max(2 * e_32, 2e-6), (e_gpu, e_32)
         U = sweep.chol_upper_of_inverse(A)
         U32 = sweep.chol_upper_of_inverse_f32(A)
-        e_gpu, e_32 = rel(Ug, U), rel(U32, U)
-        assert e_gpu <= max(2 * e_32, 2e-5), (e_gpu, e_32)
         del A, H1
     else:
         # the reverse factorisation's trailing block depends on that block
@@ -172,20 +180,19 @@ def test_llama_mlp_full_size_sampled(case):
         H1, _, _ = sweep.dead_columns(to_np(HXt[j:, j:]), np.zeros((1, 4096)))
         Hs = H1.copy()
         Hs[np.diag_indices_from(Hs)] += lam     # the damping of the whole matrix
-        Ut = sweep.chol_upper_of_inverse(Hs)
-        Ut32 = sweep.chol_upper_of_inverse_f32(Hs)
-        e_gpu, e_32 = rel(Ug[j:, j:], Ut), rel(Ut32, Ut)
-        assert e_gpu <= max(2 * e_32, 2e-5), (e_gpu, e_32)
-        del H1, Hs, Ut, Ut32
-        # U^T U A e_j = e_j on sampled columns of the whole matrix (a loose
-        # bound: the float32 residual scales with the condition number)
+        Rt = reverse_chol(Hs, np.float64)
+        e_gpu, e_32 = rel(Rg[j:, j:], Rt), rel(reverse_chol(Hs, np.float32), Rt)
+        assert e_gpu <= max(2 * e_32, 2e-6), (e_gpu, e_32)
+        del H1, Hs, Rt
+        # R R^T e_j = A e_j on sampled columns of the whole matrix (float32
+        # factorisations are backward stable: a small normwise residual)
         cols = np.array([0, 37, 63, 64, 5000, n // 2, n - 4097, n - 1])
         Acols = to_np(HXt.index_select(1, torch.as_tensor(cols, device=DEV)))
         Acols[cols, np.arange(len(cols))] += lam
-        Z = _u_times(lp.HX, _u_times(lp.HX, Acols), transpose=True)
-        Eye = np.zeros_like(Z)
+        Eye = np.zeros((n, len(cols)))
         Eye[cols, np.arange(len(cols))] = 1.0
-        assert rel(Z, Eye) < 0.1, rel(Z, Eye)
+        Z = _u_times(lp.HX, _u_times(lp.HX, Eye, transpose=True))
+        assert rel(Z, Acols) < 1e-4, rel(Z, Acols)
 
     # ---- the sweep on sampled rows
     rows = np.sort(rng.choice(m, 64, replace=False))
@@ -194,7 +201,7 @@ def test_llama_mlp_full_size_sampled(case):
     got = lp.codes[torch.as_tensor(rows, device=DEV)].cpu().numpy().astype(np.int64)
     Q = to_np(lp.Wt[torch.as_tensor(rows, device=DEV)])
     # given the GPU's factor, the float64 sweep takes the same decisions
-    ref_g = sweep.gptq_sweep(W1, Ug, bits, group, True, block=128)
+    ref_g = sweep.gptq_sweep_rform(W1, Rg, bits, group, True, block=128)
     dis_g = float(np.mean(got != ref_g["codes"]))
     assert dis_g <= 0.005, dis_g
     if U is not None:
@@ -205,13 +212,12 @@ def test_llama_mlp_full_size_sampled(case):
         dis = float(np.mean(got != ref["codes"]))
         dis_32 = float(np.mean(ref32["codes"] != ref["codes"]))
         assert dis <= max(0.005, 1.5 * dis_32), (dis, dis_32)
-        Uq = U
+        Rq = R64
     else:
         ref = ref_g
-        Uq = Ug
+        Rq = Rg
     # quadratic error of the rows under the damped factor: with dW = E U it
-    # is |E|^2 = |dW U^-1|^2, compared with the oracle sweep's
+    # is |E|^2 = |dW U^-1|^2 = |dW R|^2, compared with the oracle sweep's
     e_ref = float(np.sum(ref["E"] ** 2))
-    Ginv = solve_triangular(Uq, (W1 - Q).T, trans="T", lower=False).T   # dW U^-1
-    e_gpu = float(np.sum(Ginv ** 2))
+    e_gpu = float(np.sum(((W1 - Q) @ Rq) ** 2))
     assert abs(e_gpu - e_ref) / e_ref < 0.01, (e_gpu, e_ref)

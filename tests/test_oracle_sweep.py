@@ -244,3 +244,57 @@ def test_float32_factorisation_floor():
     e_good = np.linalg.norm(U32 - U) / np.linalg.norm(U)
     e_bad = np.linalg.norm(Ur32 - Ur) / np.linalg.norm(Ur)
     assert e_bad > 3 * e_good
+
+
+@pytest.mark.parametrize("bits,group,block", [(2, 128, 1), (3, 16, 128), (4, 1, 16), (2, -1, 128),
+                                              (3, 64, 64)])
+def test_r_form_sweep_equals_u_form(bits, group, block):
+    """gptq_sweep_rform(W, R) takes GPTQ's decisions: the same codes, grids and
+    scaled errors as gptq_sweep(W, U) with U the Cholesky factor of the damped
+    inverse (computed by its definition) and R the factor of the damped matrix
+    (LAPACK on the index-reversed matrix), float64 both."""
+    m, n = 24, 300
+    W, X, _ = tiny_layer(m=m, n=n, T=3 * n, seed=bits * 100 + n)
+    H = X.astype(np.float64).T @ X.astype(np.float64)
+    A, _ = sweep.damp(H, 0.01)
+    U = sweep.chol_upper_of_inverse(A)
+    R = np.linalg.cholesky(A[::-1, ::-1])[::-1, ::-1]
+    assert np.allclose(R @ R.T, A, rtol=1e-10, atol=1e-8 * np.abs(A).max())
+    ru = sweep.gptq_sweep(W, U, bits, group, True, block=block)
+    rr = sweep.gptq_sweep_rform(W, R, bits, group, True, block=block)
+    assert np.array_equal(ru["codes"], rr["codes"])
+    assert np.allclose(ru["scales"], rr["scales"], rtol=1e-12, atol=0)
+    assert np.allclose(ru["Q"], rr["Q"], rtol=1e-12, atol=1e-15)
+    assert np.allclose(ru["E"], rr["E"], rtol=1e-7, atol=1e-9)
+    # the value of each column at its turn (gptq_sweep's final W holds it)
+    assert np.allclose(ru["W_final"], rr["W_final"], rtol=1e-8, atol=1e-10)
+
+
+def test_r_form_sweep_slips_are_caught():
+    """Two plausible slips in the R form change codes: feeding the updated
+    weight instead of the weight before the sweep into the feedback, and
+    gridding a group from w + F / R_jj (the diagonal of U only) instead of
+    W + F U_GG."""
+    m, n, bits = 24, 384, 2
+    W, X, _ = tiny_layer(m=m, n=n, T=3 * n, seed=3)
+    A, _ = sweep.damp(X.astype(np.float64).T @ X.astype(np.float64), 0.01)
+    R = np.linalg.cholesky(A[::-1, ::-1])[::-1, ::-1]
+    U = sweep.chol_upper_of_inverse(A)
+    ref = sweep.gptq_sweep(W, U, bits, 128, True)
+    rd = np.diag(R)
+    for slip in ("updated weight", "diagonal grid"):
+        W0 = W.astype(np.float64)
+        F = np.zeros_like(W0)
+        codes = np.zeros((m, n), dtype=np.int64)
+        for j in range(n):
+            if j % 128 == 0:
+                cur = W0[:, j:j + 128] + F[:, j:j + 128] / rd[j:j + 128]
+                if slip == "updated weight":
+                    cur = W0[:, j:j + 128] + F[:, j:j + 128] @ np.linalg.inv(np.triu(R[j:j + 128, j:j + 128]))
+                scale, zero = sweep.grid_params(cur, bits, True)
+            w = W0[:, j] + F[:, j] / rd[j]
+            q, deq = sweep.quantize(w, scale, zero, bits)
+            codes[:, j] = q
+            d = (w - deq) if slip == "updated weight" else (W0[:, j] - deq)
+            F[:, j + 1:] += np.outer(d, R[j, j + 1:])
+        assert np.mean(codes != ref["codes"]) > 0.01, slip
