@@ -25,6 +25,9 @@
 //    loop, so the CTAs walk the tokens nearly in step).  A row-major order
 //    over a wide H makes every concurrent tile read different columns and
 //    the kernel DRAM-bound.
+//  * from d = 2048 on, the same on SM pairs (syrk_pair_kernel below):
+//    256 x 256 tiles, one tcgen05 instruction for two SMs, a third fewer
+//    operand bytes per flop and six stages instead of four.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -45,6 +48,8 @@ constexpr int THREADS = 192;
 constexpr int EPI_WARPS = 4;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int STRIP = 16;                              // tile rows per raster strip
+// From this order on the factor is accumulated on SM pairs (256 x 256 tiles)
+constexpr int64_t kSyrkPairMinD = 2048;
 
 struct SyrkArgs {
   float* H;
@@ -288,6 +293,279 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same accumulation on SM pairs (tcgen05 cta_group::2): a cluster of
+// two CTAs owns 256 x 256 tiles of H's upper triangle (square tiles, tile
+// row <= tile column).  Each CTA loads, per 64-token slice, the 128 token
+// columns of its half of the tile's rows (A) and of its half of the
+// tile's columns (B): 32 KB per stage instead of 48 KB for a 128 x 256
+// tile of one SM, so six stages fit and the operand bytes per flop drop by
+// a third.  The even CTA's warp 1 issues one M = 256, N = 256, K = 16 MMA
+// per 16 tokens for both; each CTA's TMEM holds its 128 rows x 256
+// columns (two accumulators of 256 columns, double-buffered across
+// tiles), and each CTA's four epilogue warps write its rows.
+// Barriers: full[s] in the even CTA (its producer expects both CTAs'
+// bytes; both CTAs' TMA loads complete on it), empty[s] and accfull[b] in
+// both CTAs (the MMA commits arrive on both), accempty[b] in the even CTA
+// (the eight epilogue warps of the pair arrive on it).
+constexpr int PM = 256, PN = 256, PH = 128;         // pair tile, per-CTA half
+constexpr int P_STAGES = 6;
+constexpr int P_BOX = 64 * BK * 2;                  // 8 KB: 64 columns x 64 tokens
+constexpr int P_HALF = PH * BK * 2;                 // 16 KB
+constexpr int P_STAGE = 2 * P_HALF;                 // 32 KB: A half + B half
+constexpr int P_NBARS = 2 * P_STAGES + 5;           // full, empty, accfull[2], accempty[2], done
+constexpr int P_SMEM = P_STAGES * P_STAGE + 1024 + 256;
+constexpr uint32_t P_TMEM = 2 * PN;
+constexpr int P_STRIP = 8;                          // tile rows (of 256) per raster strip
+
+struct SyrkPairArgs {
+  float* H;
+  int64_t d;
+  int nk;
+  int nt;        // 256-tiles per side
+  int ntiles;    // upper-triangle tiles
+  int accumulate;
+};
+
+// Upper-triangle tile t (tr <= tc) in strips of P_STRIP tile rows,
+// column-major inside a strip.
+__device__ __forceinline__ void pair_tile_of(int t, int nt, int& tr, int& tc) {
+  for (int s0 = 0; s0 < nt; s0 += P_STRIP) {
+    const int s1 = min(s0 + P_STRIP, nt);
+    int cnt = 0;
+    for (int r = s0; r < s1; ++r) cnt += nt - r;
+    if (t < cnt) {
+      for (int c = s0; c < nt; ++c) {
+        const int k = min(s1, c + 1) - s0;
+        if (t < k) {
+          tr = s0 + t;
+          tc = c;
+          return;
+        }
+        t -= k;
+      }
+    }
+    t -= cnt;
+  }
+  tr = tc = nt;  // unreachable for t < ntiles
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    syrk_pair_kernel(const __grid_constant__ CUtensorMap tmap, SyrkPairArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_NBARS);
+  volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t full0 = smem_u32(&bars[0]);
+  const uint32_t empty0 = smem_u32(&bars[P_STAGES]);
+  const uint32_t accfull0 = smem_u32(&bars[2 * P_STAGES]);
+  const uint32_t accempty0 = smem_u32(&bars[2 * P_STAGES + 2]);
+  const uint32_t done = smem_u32(&bars[2 * P_STAGES + 4]);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cl_rank();
+  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accfull0 + 8 * b, 1);
+      mbar_init(accempty0 + 8 * b, 2 * EPI_WARPS);
+    }
+    mbar_init(done, 1);
+    *abort_s = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), P_TMEM);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cl_sync();   // both CTAs' barriers initialised, both TMEM allocations made
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t stage0 = smem_u32(smem);
+  const int nk = args.nk;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t full_lead = cl_map(full0, 0);   // the even CTA's full barriers
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < args.ntiles; t += npairs) {
+        int tr, tc;
+        pair_tile_of(t, args.nt, tr, tc);
+        const int ra = tr * PM + PH * (int)rank;   // this CTA's rows of the tile (A)
+        const int cb = tc * PN + PH * (int)rank;   // this CTA's columns of the tile (B)
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          if (*abort_s || !mbar_wait(empty0 + 8 * s, ph ^ 1)) {
+            *abort_s = 1;
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * P_STAGE);
+          const uint32_t a = stage0 + s * P_STAGE;
+          const uint32_t b = a + P_HALF;
+          const uint32_t fb = full_lead + 8 * s;
+          const int y = kb * BK;
+          tma_load_2d_pair(a, &tmap, fb, ra, y);
+          tma_load_2d_pair(a + P_BOX, &tmap, fb, ra + 64, y);
+          tma_load_2d_pair(b, &tmap, fb, cb, y);
+          tma_load_2d_pair(b + P_BOX, &tmap, fb, cb + 64, y);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(PM, PN, true, true);
+      uint32_t it = 0;
+      int tl = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int t = pair; ok && t < args.ntiles; t += npairs, ++tl) {
+        const int b = tl & 1;
+        const uint32_t u = (uint32_t)(tl >> 1);
+        // both CTAs' epilogues have read accumulator b (tile tl - 2)
+        if (u > 0 && (*abort_s || !mbar_wait(accempty0 + 8 * b, (u - 1) & 1))) {
+          *abort_s = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(b * PN);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t s = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          if (*abort_s || !mbar_wait(full0 + 8 * s, ph)) {
+            *abort_s = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = stage0 + s * P_STAGE;
+          const uint32_t bb = a + P_HALF;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a + kk * 2048, P_BOX, 1024);
+            const uint64_t bd = smem_desc_sw128(bb + kk * 2048, P_BOX, 1024);
+            mma_bf16_pair(acc, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit_pair_mc(empty0 + 8 * s, 0x3);
+        }
+        if (ok) mma_commit_pair_mc(accfull0 + 8 * b, 0x3);
+      }
+      // every MMA issued has completed (they write both CTAs' TMEM) before
+      // the pair frees its TMEM
+      if (issued) {
+        mma_commit_pair_mc(done, 0x1);
+        mbar_wait(done, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // Epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 of this CTA: rows
+    // ra + 32 (w % 4) + lane of H, the tile's 256 columns.
+    const int q = warp & 3;
+    const int64_t d = args.d;
+    float* H = args.H;
+    const int accm = args.accumulate;
+    const uint32_t accempty_lead = cl_map(accempty0, 0);
+    int tl = 0;
+    for (int t = pair; t < args.ntiles; t += npairs, ++tl) {
+      const int b = tl & 1;
+      const uint32_t u = (uint32_t)(tl >> 1);
+      int ok = 1;
+      if (lane == 0) ok = (!*abort_s && mbar_wait(accfull0 + 8 * b, u & 1)) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      if (!ok) {
+        if (lane == 0) *abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      int tr, tc;
+      pair_tile_of(t, args.nt, tr, tc);
+      const int64_t i = (int64_t)tr * PM + PH * rank + q * 32 + lane;
+      const int64_t c0 = (int64_t)tc * PN;
+#pragma unroll 1
+      for (int cc = 0; cc < PN / 32; ++cc) {
+        const int64_t jb = c0 + cc * 32;
+        // 32 columns left of every row of this warp: nothing of them is kept
+        // (uniform over the warp, which loads TMEM collectively)
+        if (jb + 31 < (int64_t)tr * PM + PH * rank + q * 32) continue;
+        const bool dense = (i < d) && (jb >= i) && (jb + 32 <= d) &&
+                           ((reinterpret_cast<uintptr_t>(H + i * d + jb) & 15) == 0);
+        float old[32], mir[32];
+        if (accm) {
+          if (dense) {
+            const float4* src = reinterpret_cast<const float4*>(H + i * d + jb);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float4 o = src[e];
+              old[4 * e] = o.x; old[4 * e + 1] = o.y; old[4 * e + 2] = o.z; old[4 * e + 3] = o.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int64_t j = jb + e;
+              old[e] = (i < d && j < d && i <= j) ? H[i * d + j] : 0.f;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int64_t j = jb + e;
+            mir[e] = (i < d && j < d && i < j) ? H[j * d + i] : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) old[e] = mir[e] = 0.f;
+        }
+        uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(b * PN + cc * 32), v);
+        tmem_wait_ld();
+        if (dense) {
+          float4* dst = reinterpret_cast<float4*>(H + i * d + jb);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]) + old[4 * e], __uint_as_float(v[4 * e + 1]) + old[4 * e + 1],
+                                 __uint_as_float(v[4 * e + 2]) + old[4 * e + 2],
+                                 __uint_as_float(v[4 * e + 3]) + old[4 * e + 3]);
+        } else if (i < d) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int64_t j = jb + e;
+            if (j < d && i <= j) H[i * d + j] = __uint_as_float(v[e]) + old[e];
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int64_t j = jb + e;
+          if (i < d && j < d && i < j) H[j * d + i] = __uint_as_float(v[e]) + mir[e];
+        }
+      }
+      // accumulator b may be refilled once the pair's eight warps have read it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(accempty_lead + 8 * b);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cl_sync();   // no pair MMA, TMEM read or remote arrive is left in either CTA
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, P_TMEM);
+  }
+}
+
 __global__ void fill_kernel(float* p, int64_t count, float v) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count;
        i += (int64_t)gridDim.x * blockDim.x)
@@ -346,6 +624,42 @@ kronq_status syrk_bf16_tc(const void* A, int64_t T, int64_t d, int64_t lda, floa
   for (int tr = 0; tr < args.nr; ++tr) ntiles += args.nc - (tr * BM) / BN;
   args.ntiles = (int)ntiles;
 
+  if (d >= kSyrkPairMinD) {
+    // SM pairs: 256 x 256 tiles, as many clusters of two as fit at once
+    SyrkPairArgs pa;
+    pa.H = H;
+    pa.d = d;
+    pa.nk = args.nk;
+    pa.nt = (int)ceil_div(d, PM);
+    pa.ntiles = pa.nt * (pa.nt + 1) / 2;
+    pa.accumulate = args.accumulate;
+    const void* fn = reinterpret_cast<const void*>(&syrk_pair_kernel);
+    cudaError_t e = allow_smem(fn, P_SMEM);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(syrk pair)");
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = (size_t)P_SMEM;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)(2 * (sm_count() / 2)));
+    int active = 0;
+    e = cudaOccupancyMaxActiveClusters(&active, fn, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(syrk pair)");
+    if (active >= 1) {
+      const int64_t npairs = pa.ntiles < (int64_t)active ? pa.ntiles : (int64_t)active;
+      cfg.gridDim = dim3((unsigned)(2 * npairs));
+      e = cudaLaunchKernelEx(&cfg, syrk_pair_kernel, map, pa);
+      count_launch();
+      if (e != cudaSuccess) return cuda_fail(e, "syrk_pair_kernel");
+      return KRONQ_OK;
+    }
+  }
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(&syrk_bf16_tc_kernel), SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(syrk)");
   const int64_t grid = ntiles < (int64_t)sm_count() ? ntiles : (int64_t)sm_count();
