@@ -62,10 +62,13 @@ WORKLOADS = {
         layers=[("q_proj", 4096, 4096, False)]),
 }
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one syrk_bf16_tc_kernel
-# launch (ncu, B200), keyed by (d, tokens per launch); None until the
-# current kernel has been captured at that shape.
-SYRK_TRAFFIC = {}
+# dram__bytes_read.sum + dram__bytes_write.sum of one factor-accumulation
+# launch (syrk_pair_kernel, ncu on a B200, one capture each), keyed by
+# (d, tokens per launch); shapes not captured give traffic null.
+SYRK_TRAFFIC = {
+    (28672, 16384): 33008609792 + 3273005312,
+    (8192, 16384): 1136330496 + 250929152,
+}
 
 
 def _peaks():
@@ -507,7 +510,8 @@ def run_kronq(args):
             tkeys.append((d, T if chunk is None else chunk))
     if all(k in SYRK_TRAFFIC for k in tkeys):
         traffic = sum(SYRK_TRAFFIC[k] for k in tkeys) / len(tkeys)
-    roofline = {"bound": "tensor", "kernel": "syrk_bf16_tc_kernel", "achieved": achieved, "peak": tpk,
+    kname = "syrk_pair_kernel" if min(min(m, n) for m, n in shapes) >= 2048 else "syrk_bf16_tc_kernel"
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": tpk,
                 "unit": "TFLOP/s", "frac": achieved / tpk, "traffic": traffic,
                 "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean per launch "
                                   "over the step's launch shapes" if traffic else None,
