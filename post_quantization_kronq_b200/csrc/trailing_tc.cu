@@ -26,6 +26,8 @@ namespace kq {
 namespace {
 
 constexpr int BM = 128, BN = 128, KC = 64, NSTAGE = 2;
+// The group-end updates (K of a whole group) run on SM pairs
+constexpr int64_t kTrailPairMinK = 512;
 constexpr int A_BOX = BM * KC * 2;         // 16 KB: 128 rows x 64 k (K-major, 128 B rows)
 constexpr int B_BOX = 64 * KC * 2;         // 8 KB: 64 k rows x 64 columns (MN-major)
 constexpr int B_SPLIT = (BN / 64) * B_BOX; // 16 KB: one split of the B chunk
@@ -198,6 +200,240 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 
+// ---------------------------------------------------------------------------
+// The same update on SM pairs (tcgen05 cta_group::2), persistent: a cluster
+// of two CTAs walks 256 x 256 tiles of W[:, cols] (column-major over the
+// tiles, so the pairs in flight share U's columns while E, small, stays in
+// L2).  Per 64-deep k chunk each CTA loads its 128 rows of E hi/lo and its
+// 128 columns of U hi/lo (64 KB; three stages), the even CTA issues the
+// three split products for both (M = 256, N = 256, K = 16, 12 MMAs per
+// chunk) into one of two 256-column TMEM accumulators, and each CTA's four
+// epilogue warps subtract their 128 rows from W in place (rows of 32
+// columns at a time, loads before stores) while the next tile's MMAs run.
+// Barriers as in the pair factor accumulation.
+constexpr int TP_M = 256, TP_N = 256, TP_H = 128;
+constexpr int TP_STAGES = 3;
+constexpr int TP_ABOX = TP_H * KC * 2;              // 16 KB: 128 rows x 64 k (K-major)
+constexpr int TP_BBOX = 64 * KC * 2;                // 8 KB: 64 columns x 64 k (MN-major)
+constexpr int TP_STAGE = 2 * TP_ABOX + 4 * TP_BBOX; // 64 KB: E hi, E lo, U hi (2 boxes), U lo (2 boxes)
+constexpr int TP_NBARS = 2 * TP_STAGES + 5;
+constexpr int TP_SMEM = TP_STAGES * TP_STAGE + 1024 + 256;
+constexpr int TP_THREADS = 192;
+constexpr int TP_EPI = 4;
+constexpr uint32_t TP_TMEM = 2 * TP_N;
+
+struct TrailPairArgs {
+  float* W;
+  int64_t m, n;
+  int64_t c_begin, c_end;   // the columns updated: [c_begin, c_end)
+  int k0;
+  int nkc;
+  int tiles_m, tiles_n, ntiles;
+  const int* info;
+};
+
+__global__ void __launch_bounds__(TP_THREADS, 1)
+    trailing_pair_kernel(const __grid_constant__ CUtensorMap mEh, const __grid_constant__ CUtensorMap mEl,
+                         const __grid_constant__ CUtensorMap mUh, const __grid_constant__ CUtensorMap mUl,
+                         TrailPairArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TP_STAGES * TP_STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + TP_NBARS);
+  volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t full0 = smem_u32(&bars[0]);
+  const uint32_t empty0 = smem_u32(&bars[TP_STAGES]);
+  const uint32_t accfull0 = smem_u32(&bars[2 * TP_STAGES]);
+  const uint32_t accempty0 = smem_u32(&bars[2 * TP_STAGES + 2]);
+  const uint32_t done = smem_u32(&bars[2 * TP_STAGES + 4]);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cl_rank();
+  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+  // a failed factorisation leaves nothing to update (uniform over the grid)
+  const bool skip = args.info && *args.info != 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TP_STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accfull0 + 8 * b, 1);
+      mbar_init(accempty0 + 8 * b, 2 * TP_EPI);
+    }
+    mbar_init(done, 1);
+    *abort_s = skip ? 1 : 0;
+    fence_mbar_init();
+    prefetch_tmap(&mEh);
+    prefetch_tmap(&mEl);
+    prefetch_tmap(&mUh);
+    prefetch_tmap(&mUl);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TP_TMEM);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cl_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t stage0 = smem_u32(smem);
+  const int nkc = args.nkc;
+  const int ntiles = skip ? 0 : args.ntiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t full_lead = cl_map(full0, 0);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < ntiles; t += npairs) {
+        const int tm = t % args.tiles_m, tn = t / args.tiles_m;   // column-major over the tiles
+        const int ra = tm * TP_M + TP_H * (int)rank;
+        const int cb = (int)args.c_begin + tn * TP_N + TP_H * (int)rank;
+        for (int c = 0; c < nkc; ++c, ++it) {
+          const uint32_t s = it % TP_STAGES;
+          const uint32_t ph = (it / TP_STAGES) & 1;
+          if (*abort_s || !mbar_wait(empty0 + 8 * s, ph ^ 1)) {
+            *abort_s = 1;
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * TP_STAGE);
+          const uint32_t st = stage0 + s * TP_STAGE;
+          const uint32_t fb = full_lead + 8 * s;
+          const int k = args.k0 + c * KC;
+          tma_load_2d_pair(st, &mEh, fb, k, ra);
+          tma_load_2d_pair(st + TP_ABOX, &mEl, fb, k, ra);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tma_load_2d_pair(st + 2 * TP_ABOX + h * TP_BBOX, &mUh, fb, cb + 64 * h, k);
+            tma_load_2d_pair(st + 2 * TP_ABOX + 2 * TP_BBOX + h * TP_BBOX, &mUl, fb, cb + 64 * h, k);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(TP_M, TP_N, false, true);
+      uint32_t it = 0;
+      int tl = 0;
+      bool ok = true, issued = false;
+      for (int t = pair; ok && t < ntiles; t += npairs, ++tl) {
+        const int b = tl & 1;
+        const uint32_t u = (uint32_t)(tl >> 1);
+        if (u > 0 && (*abort_s || !mbar_wait(accempty0 + 8 * b, (u - 1) & 1))) {
+          *abort_s = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(b * TP_N);
+        for (int c = 0; c < nkc; ++c, ++it) {
+          const uint32_t s = it % TP_STAGES;
+          const uint32_t ph = (it / TP_STAGES) & 1;
+          if (*abort_s || !mbar_wait(full0 + 8 * s, ph)) {
+            *abort_s = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = stage0 + s * TP_STAGE;
+          const uint32_t ah = st, al = st + TP_ABOX;
+          const uint32_t bh = st + 2 * TP_ABOX, bl = st + 2 * TP_ABOX + 2 * TP_BBOX;
+#pragma unroll
+          for (int kk = 0; kk < KC / 16; ++kk) {
+            // A K-major: 16 k = 32 bytes along each 128-byte row.  B MN-major:
+            // 16 k rows of 128 bytes = 2048 bytes inside every 64-column box.
+            const uint64_t dah = smem_desc_sw128(ah + kk * 32, 16, 1024);
+            const uint64_t dal = smem_desc_sw128(al + kk * 32, 16, 1024);
+            const uint64_t dbh = smem_desc_sw128(bh + kk * 2048, TP_BBOX, 1024);
+            const uint64_t dbl = smem_desc_sw128(bl + kk * 2048, TP_BBOX, 1024);
+            mma_bf16_pair(acc, dah, dbh, idesc, (c | kk) != 0 ? 1u : 0u);
+            mma_bf16_pair(acc, dah, dbl, idesc, 1u);
+            mma_bf16_pair(acc, dal, dbh, idesc, 1u);
+          }
+          issued = true;
+          mma_commit_pair_mc(empty0 + 8 * s, 0x3);
+        }
+        if (ok) mma_commit_pair_mc(accfull0 + 8 * b, 0x3);
+      }
+      if (issued) {
+        mma_commit_pair_mc(done, 0x1);
+        mbar_wait(done, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int64_t n = args.n;
+    float* W = args.W;
+    const uint32_t accempty_lead = cl_map(accempty0, 0);
+    int tl = 0;
+    for (int t = pair; t < ntiles; t += npairs, ++tl) {
+      const int b = tl & 1;
+      const uint32_t u = (uint32_t)(tl >> 1);
+      int good = 1;
+      if (lane == 0) good = (!*abort_s && mbar_wait(accfull0 + 8 * b, u & 1)) ? 1 : 0;
+      good = __shfl_sync(0xffffffffu, good, 0);
+      __syncwarp();
+      if (!good) {
+        if (lane == 0) *abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      const int tm = t % args.tiles_m, tn = t / args.tiles_m;
+      const int64_t i = (int64_t)tm * TP_M + TP_H * rank + q * 32 + lane;
+      const int64_t c0 = args.c_begin + (int64_t)tn * TP_N;
+#pragma unroll 1
+      for (int cc = 0; cc < TP_N / 32; ++cc) {
+        const int64_t jb = c0 + cc * 32;
+        if (jb >= args.c_end) break;   // uniform over the warp
+        const bool dense = (i < args.m) && (jb + 32 <= args.c_end) &&
+                           ((reinterpret_cast<uintptr_t>(W + i * n + jb) & 15) == 0);
+        float old[32];
+        if (dense) {
+          const float4* src = reinterpret_cast<const float4*>(W + i * n + jb);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 o = src[e];
+            old[4 * e] = o.x; old[4 * e + 1] = o.y; old[4 * e + 2] = o.z; old[4 * e + 3] = o.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            old[e] = (i < args.m && jb + e < args.c_end) ? W[i * n + jb + e] : 0.f;
+        }
+        uint32_t v[32];
+        __syncwarp();  // the TMEM load is warp-collective
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(b * TP_N + cc * 32), v);
+        tmem_wait_ld();
+        if (dense) {
+          float4* dst = reinterpret_cast<float4*>(W + i * n + jb);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(old[4 * e] - __uint_as_float(v[4 * e]), old[4 * e + 1] - __uint_as_float(v[4 * e + 1]),
+                                 old[4 * e + 2] - __uint_as_float(v[4 * e + 2]),
+                                 old[4 * e + 3] - __uint_as_float(v[4 * e + 3]));
+        } else if (i < args.m) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (jb + e < args.c_end) W[i * n + jb + e] = old[e] - __uint_as_float(v[e]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(accempty_lead + 8 * b);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cl_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TP_TMEM);
+  }
+}
+
 }  // namespace
 
 cudaError_t status_fetch_trailing(int* out, cudaStream_t s) {
@@ -235,6 +471,47 @@ kronq_status trailing_update_tc(const TrailingMaps* tm, float* W, int64_t m, int
                                 int64_t ncols, int64_t k0, int64_t K, const int* info, cudaStream_t s) {
   if (ncols <= 0 || K <= 0) return KRONQ_OK;
   const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(tm->raw);
+  if (K >= kTrailPairMinK && m >= TP_M) {
+    // SM pairs, persistent over 256 x 256 tiles
+    TrailPairArgs pa;
+    pa.W = W;
+    pa.m = m;
+    pa.n = n;
+    pa.c_begin = c_begin;
+    pa.c_end = c_begin + ncols;
+    pa.k0 = (int)k0;
+    pa.nkc = (int)((K + KC - 1) / KC);
+    pa.tiles_m = (int)ceil_div(m, TP_M);
+    pa.tiles_n = (int)ceil_div(ncols, TP_N);
+    pa.ntiles = pa.tiles_m * pa.tiles_n;
+    pa.info = info;
+    const void* fn = reinterpret_cast<const void*>(&trailing_pair_kernel);
+    cudaError_t e = allow_smem(fn, TP_SMEM);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(trailing pair)");
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(TP_THREADS);
+    cfg.dynamicSmemBytes = (size_t)TP_SMEM;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)(2 * (sm_count() / 2)));
+    int active = 0;
+    e = cudaOccupancyMaxActiveClusters(&active, fn, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(trailing pair)");
+    if (active >= 1) {
+      const int64_t npairs = pa.ntiles < (int64_t)active ? pa.ntiles : (int64_t)active;
+      cfg.gridDim = dim3((unsigned)(2 * npairs));
+      e = cudaLaunchKernelEx(&cfg, trailing_pair_kernel, maps[0], maps[1], maps[2], maps[3], pa);
+      count_launch();
+      if (e != cudaSuccess) return cuda_fail(e, "trailing_pair_kernel");
+      return KRONQ_OK;
+    }
+  }
   TrailArgs a;
   a.W = W;
   a.m = m;
