@@ -110,8 +110,10 @@ typedef struct {
  *         exact-fp32 SIMT kernel (small layers).
  *   zero_first  nonzero: H is overwritten with A^T A instead of added to.
  *   Call once per token chunk to stream T (pass zero_first only first).
- *   Both triangles of H are kept equal.  T == 0 is allowed (no-op, or a
- *   zero fill when zero_first).
+ *   Both triangles of H are kept equal; when adding, H must be symmetric on
+ *   input (as every call leaves it): from d = 2048 on only its upper
+ *   triangle is read.  T == 0 is allowed (no-op, or a zero fill when
+ *   zero_first).
  * ------------------------------------------------------------------------- */
 kronq_status kronq_accumulate_factors(const void* A, kronq_dtype dt, int64_t T, int64_t d,
                                       int64_t lda, float* H, int zero_first, kronq_stream_t s);

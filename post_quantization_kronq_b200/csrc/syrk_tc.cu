@@ -500,9 +500,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         // 32 columns left of every row of this warp: nothing of them is kept
         // (uniform over the warp, which loads TMEM collectively)
         if (jb + 31 < (int64_t)tr * PM + PH * rank + q * 32) continue;
+        // H is symmetric on input (every call leaves both triangles equal):
+        // the upper element is read, and it and its mirror get the sum
         const bool dense = (i < d) && (jb >= i) && (jb + 32 <= d) &&
                            ((reinterpret_cast<uintptr_t>(H + i * d + jb) & 15) == 0);
-        float old[32], mir[32];
+        float old[32];
         if (accm) {
           if (dense) {
             const float4* src = reinterpret_cast<const float4*>(H + i * d + jb);
@@ -518,37 +520,32 @@ __global__ void __launch_bounds__(THREADS, 1)
               old[e] = (i < d && j < d && i <= j) ? H[i * d + j] : 0.f;
             }
           }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int64_t j = jb + e;
-            mir[e] = (i < d && j < d && i < j) ? H[j * d + i] : 0.f;
-          }
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) old[e] = mir[e] = 0.f;
+          for (int e = 0; e < 32; ++e) old[e] = 0.f;
         }
         uint32_t v[32];
         __syncwarp();  // the TMEM load is warp-collective
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(b * PN + cc * 32), v);
         tmem_wait_ld();
+        float sum[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sum[e] = __uint_as_float(v[e]) + old[e];
         if (dense) {
           float4* dst = reinterpret_cast<float4*>(H + i * d + jb);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(v[4 * e]) + old[4 * e], __uint_as_float(v[4 * e + 1]) + old[4 * e + 1],
-                                 __uint_as_float(v[4 * e + 2]) + old[4 * e + 2],
-                                 __uint_as_float(v[4 * e + 3]) + old[4 * e + 3]);
+          for (int e = 0; e < 8; ++e) dst[e] = make_float4(sum[4 * e], sum[4 * e + 1], sum[4 * e + 2], sum[4 * e + 3]);
         } else if (i < d) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int64_t j = jb + e;
-            if (j < d && i <= j) H[i * d + j] = __uint_as_float(v[e]) + old[e];
+            if (j < d && i <= j) H[i * d + j] = sum[e];
           }
         }
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int64_t j = jb + e;
-          if (i < d && j < d && i < j) H[j * d + i] = __uint_as_float(v[e]) + mir[e];
+          if (i < d && j < d && i < j) H[j * d + i] = sum[e];
         }
       }
       // accumulator b may be refilled once the pair's eight warps have read it
