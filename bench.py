@@ -66,8 +66,8 @@ WORKLOADS = {
 # launch (syrk_pair_kernel, ncu on a B200, one capture each), keyed by
 # (d, tokens per launch); shapes not captured give traffic null.
 SYRK_TRAFFIC = {
-    (28672, 16384): 33008609792 + 3273005312,
-    (8192, 16384): 1136330496 + 250929152,
+    (28672, 16384): 32839476992 + 3274788864,
+    (8192, 16384): 1161290496 + 251058688,
 }
 
 
@@ -521,6 +521,31 @@ def run_kronq(args):
         roofline["frac_of_burst"] = achieved / peaks["bf16_tflops"]
         roofline["frac_of_sustained"] = achieved / peaks["bf16_tflops_sustained"]
 
+    # The packing kernel on its own (HBM-bound: m n (1 + b/8) bytes per
+    # layer), timed with CUDA events over repeated calls on the step's codes
+    # (larger than L2).
+    kernel_rooflines = {}
+    pk_ms = pk_bytes = 0.0
+    for _, _, _, _, lp in layers:
+        if lp.packed is None:
+            continue
+        kq.kronq_pack(lp.codes, lp.bits, lp.packed, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        e0.record(stream)
+        for _ in range(reps):
+            kq.kronq_pack(lp.codes, lp.bits, lp.packed, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pk_ms += e0.elapsed_time(e1) / reps
+        pk_bytes += lp.m * lp.n * (1 + lp.bits / 8)
+    if pk_ms > 0:
+        gbs = pk_bytes / (pk_ms / 1e3) / 1e9
+        kernel_rooflines["pack_kernel"] = {"bound": "hbm", "achieved": gbs, "peak": hpk, "unit": "GB/s",
+                                           "frac": gbs / hpk, "bytes_per_step": pk_bytes,
+                                           "ms_per_step": pk_ms,
+                                           "peak_source": "measured hbm_gbs" if peaks else "fallback"}
+
     # End to end through the public API: inputs copied from pinned host memory
     # every step, packed codes, scales and zeros copied back.
     e2e = None
@@ -623,6 +648,7 @@ def run_kronq(args):
         "gpu_launches": launches,
         "phases_ms": {k: round(v, 4) for k, v in phases.items()},
         "phase_roofline": phase_rooflines(phases, shapes, T, tpk, hpk, src),
+        "kernel_roofline": kernel_rooflines,
         "sensitivity": sens, "also": also,
     }
     print(json.dumps(line), flush=True)

@@ -291,6 +291,47 @@ kronq_status kronq_quantize_layer_act_order(float* Wt, float* HX, int64_t m, int
                                             float* zeros, float* E, int* g_idx, int* perm, int* info,
                                             void* workspace, size_t ws_bytes, kronq_stream_t s);
 
+/* kronq_quantize_two_sided -- two-sided rounding that uses H_G inside the
+ * sweep ("BaKron: Efficient Quantization with Kronecker-Factored Hessians"
+ * page, abstract: GPTQ-style rounding in the vectorised weight domain under
+ * the Kronecker-factored Hessian, anti-diagonal parallelism, O(m + n)
+ * sequential steps, O(mn(m + n)) work).  The abstract gives no algorithm;
+ * the reading implemented is GPTQ on vec(W) with the upper factor
+ * U = U_X (x) U_G of the damped inverse Hessian:
+ *   - both factors damped by the relative rule (lambda = damp_rel * mean
+ *     diagonal; no dead-column rule), U_X^T U_X = (H~_X + lambda_X I)^-1,
+ *     U_G^T U_G = (H~_G + lambda_G I)^-1, both upper;
+ *   - static per-row group grids taken from W~ before the sweep (the grid
+ *     rule of kronq_quantize_layer; a grid taken at a group start would
+ *     depend on the processing order);
+ *   - element (i, j): q = clamp(rint(w~ / scale) + zero, 0, 2^b - 1),
+ *     e_ij = (w~_ij - deq) / (U_X[j, j] U_G[i, i]), and
+ *     w~_i'j' -= e_ij U_G[i, i'] U_X[j, j'] for every later (i' >= i,
+ *     j' >= j) element.  Every order that respects that partial order gives
+ *     the same result; the library runs 32 x 128 tiles along anti-diagonals.
+ *   Wt     m x n float32: in W~, out the dequantised W~_q.
+ *   HX     n x n float32: in H~_X (or U_X with KRONQ_U_GIVEN), out U_X
+ *          (upper triangle; the strict lower triangle is scratch).
+ *   HG     m x m float32: in H~_G (or U_G with KRONQ_U_GIVEN), out U_G.
+ *   codes  m x n uint8 out; scales, zeros m x ngroups float32 out.
+ *   E      m x n float32 out (the scaled errors e_ij) with KRONQ_WRITE_E,
+ *          else NULL.
+ *   info   TWO ints (device) out: info[0] for H~_X, info[1] for H~_G, each
+ *          0 or 1 + the largest index whose trailing submatrix was found not
+ *          positive definite (the outputs are then unspecified).
+ *   flags  KRONQ_U_GIVEN and KRONQ_WRITE_E; KRONQ_R_FORM and
+ *          KRONQ_ORDERED_FP32 are rejected (KRONQ_ERR_INVALID_ARG).
+ *          block must be 128; groups as kronq_quantize_layer.
+ *   workspace >= kronq_quantize_two_sided_workspace_bytes(m, n, p), 256-byte
+ *          aligned (2 m n floats plus the factorisation scratch of the larger
+ *          factor).
+ * Asynchronous on s. */
+size_t kronq_quantize_two_sided_workspace_bytes(int64_t m, int64_t n, const kronq_quant_params* p);
+kronq_status kronq_quantize_two_sided(float* Wt, float* HX, float* HG, int64_t m, int64_t n,
+                                      const kronq_quant_params* p, uint8_t* codes, float* scales,
+                                      float* zeros, float* E, int* info, void* workspace, size_t ws_bytes,
+                                      kronq_stream_t s);
+
 /* ---------------------------------------------------------------------------
  * Step 5 -- packing.  KronQ README "Model zoo": W4/W2 as packed int4/int2,
  * W3 not bit-packable (bits == 3 -> KRONQ_ERR_INVALID_ARG).  Layout: per

@@ -20,7 +20,7 @@ __all__ = [
     "kronq_allocate_topn_types", "kronq_biip_workspace_bytes", "kronq_biip_forward",
     "kronq_biip_inverse", "kronq_quantize_workspace_bytes", "kronq_quantize_layer",
     "kronq_quantize_layer_static", "kronq_quantize_act_order_workspace_bytes",
-    "kronq_quantize_layer_act_order",
+    "kronq_quantize_layer_act_order", "kronq_quantize_two_sided_workspace_bytes", "kronq_quantize_two_sided",
     "kronq_pack", "kronq_unpack", "kronq_device_status", "kronq_wait_selftest",
     "kronq_kfac_loss_workspace_bytes",
     "kronq_kfac_loss", "kronq_launch_count", "kronq_last_error", "kronq_version", "workspace", "words_per_row",
@@ -211,6 +211,26 @@ def kronq_quantize_layer_act_order(Wt, HX, params: QuantParams, codes, scales, z
     check(lib.kronq_quantize_layer_act_order(_ptr(Wt), _ptr(HX), m, n, ctypes.byref(params), _ptr(codes),
                                              _ptr(scales), _ptr(zeros), _ptr(E), _ptr(g_idx), _ptr(perm),
                                              _ptr(info), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def kronq_quantize_two_sided_workspace_bytes(m: int, n: int, params: QuantParams) -> int:
+    return int(lib.kronq_quantize_two_sided_workspace_bytes(m, n, ctypes.byref(params)))
+
+
+def kronq_quantize_two_sided(Wt, HX, HG, params: QuantParams, codes, scales, zeros, info, E=None, ws=None,
+                             stream=None):
+    """Two-sided rounding under H_X (x) H_G; info holds two int32 (H_X, H_G)."""
+    m, n = Wt.shape
+    for t, name in ((Wt, "Wt"), (HX, "HX"), (HG, "HG"), (codes, "codes"), (scales, "scales"),
+                    (zeros, "zeros"), (info, "info"), (E, "E")):
+        _rowmajor(t, name)
+    if info.numel() < 2:
+        raise ValueError("info: two int32 (H_X, H_G)")
+    if ws is None:
+        ws = workspace(kronq_quantize_two_sided_workspace_bytes(m, n, params), Wt.device)
+    check(lib.kronq_quantize_two_sided(_ptr(Wt), _ptr(HX), _ptr(HG), m, n, ctypes.byref(params), _ptr(codes),
+                                       _ptr(scales), _ptr(zeros), _ptr(E), _ptr(info), _ptr(ws), ws.numel(),
+                                       _stream(stream)))
 
 
 def kronq_pack(codes, bits: int, out, stream=None):

@@ -61,6 +61,9 @@ SIGNATURES = {
     "kronq_quantize_act_order_workspace_bytes": (_sz, [_i64, _i64, _qp]),
     "kronq_quantize_layer_act_order": (_int, [_vp, _vp, _i64, _i64, _qp, _vp, _vp, _vp, _vp, _vp,
                                               _vp, _vp, _vp, _sz, _vp]),
+    "kronq_quantize_two_sided_workspace_bytes": (_sz, [_i64, _i64, _qp]),
+    "kronq_quantize_two_sided": (_int, [_vp, _vp, _vp, _i64, _i64, _qp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _sz, _vp]),
     "kronq_pack": (_int, [_vp, _i64, _i64, _int, _vp, _vp]),
     "kronq_unpack": (_int, [_vp, _i64, _i64, _int, _vp, _vp]),
     "kronq_device_status": (_int, [_ip, _vp]),

@@ -32,14 +32,16 @@ namespace {
 
 constexpr int NB = 64;
 
+// fix_zero: a zero diagonal entry becomes 1 before the mean is taken (the
+// one-sided pass's dead-column rule); without it the diagonal is damped as is.
 __global__ void __launch_bounds__(1024) damp_kernel(float* H, int64_t n, float damp_rel,
-                                                    uint8_t* dead, int* info) {
+                                                    uint8_t* dead, int* info, bool fix_zero) {
   __shared__ double red[32];
   if (threadIdx.x == 0) *info = 0;
   double acc = 0.0;
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
     float h = H[j * n + j];
-    const bool isdead = (h == 0.f);
+    const bool isdead = fix_zero && (h == 0.f);
     if (isdead) {
       h = 1.f;
       H[j * n + j] = 1.f;
@@ -1110,8 +1112,14 @@ size_t chol_workspace_bytes(int64_t n) {
 
 size_t chol_tbuf_bytes(int64_t n) { return tbuf_bytes(n); }
 
+kronq_status damp_only(float* H, int64_t n, float damp_rel, int* info, cudaStream_t s) {
+  damp_kernel<<<1, 1024, 0, s>>>(H, n, damp_rel, nullptr, info, false);
+  KQ_LAUNCH_CHECK("damp_kernel");
+  return KRONQ_OK;
+}
+
 kronq_status damp_factor(float* H, int64_t n, float damp_rel, uint8_t* dead, int* info, cudaStream_t s) {
-  damp_kernel<<<1, 1024, 0, s>>>(H, n, damp_rel, dead, info);
+  damp_kernel<<<1, 1024, 0, s>>>(H, n, damp_rel, dead, info, true);
   KQ_LAUNCH_CHECK("damp_kernel");
   return KRONQ_OK;
 }
@@ -1119,7 +1127,7 @@ kronq_status damp_factor(float* H, int64_t n, float damp_rel, uint8_t* dead, int
 kronq_status chol_upper_inverse(float* H, int64_t n, float damp_rel, bool skip_damp,
                                 uint8_t* dead, int* info, void* ws, cudaStream_t s, bool want_u) {
   if (!skip_damp) {
-    damp_kernel<<<1, 1024, 0, s>>>(H, n, damp_rel, dead, info);
+    damp_kernel<<<1, 1024, 0, s>>>(H, n, damp_rel, dead, info, true);
     KQ_LAUNCH_CHECK("damp_kernel");
   } else {
     zero_info_kernel<<<1, 1, 0, s>>>(info);

@@ -232,6 +232,9 @@ kronq_status quantize_core(float* Wt, float* HX, int64_t m, int64_t n, const kro
                            void* workspace, cudaStream_t st, int mode);
 // Dead-column rule and damping of H in place (dead flags out, info reset).
 kronq_status damp_factor(float* H, int64_t n, float damp_rel, uint8_t* dead, int* info, cudaStream_t s);
+// Damping alone (zero diagonal entries stay zero before lambda is added),
+// info reset.
+kronq_status damp_only(float* H, int64_t n, float damp_rel, int* info, cudaStream_t s);
 
 // ------------------------------------------------------------ pack / misc
 kronq_status pack_codes(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* out,

@@ -7,6 +7,7 @@
     python -m post_quantization_kronq_b200.opbench pack --m 8192 --n 28672 --bits 2
     python -m post_quantization_kronq_b200.opbench kronfactors --est flipflop --tokens 131072 --m 4096 --n 4096
     python -m post_quantization_kronq_b200.opbench decode --m 4096 --n 4096 --bits 2 --reps 100
+    python -m post_quantization_kronq_b200.opbench twosided --m 4096 --n 4096 --bits 2 [--u-given]
 
 Meant for profiling a single kernel family (e.g. under ncu) at a size that
 is smaller than the full benchmark; prints one JSON line with the mean
@@ -33,7 +34,9 @@ def main(argv=None):
 
     ap = argparse.ArgumentParser()
     ap.add_argument("op", choices=["accumulate", "biip", "biip_inverse", "quantize", "pack", "kronfactors",
-                                   "decode"])
+                                   "decode", "twosided"])
+    ap.add_argument("--u-given", action="store_true",
+                    help="twosided: factor once, time the sweep alone (KRONQ_U_GIVEN)")
     ap.add_argument("--est", choices=["input", "marginal", "frobenius", "flipflop"], default="flipflop")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--tokens", type=int, default=16384)
@@ -87,6 +90,33 @@ def main(argv=None):
         # SYRKs (T n (n+1) and T m (m+1))
         units = {"flops_per_sweep": 2 * a.tokens * (a.m * a.m + a.n * a.n)
                  + a.tokens * (a.n * (a.n + 1) + a.m * (a.m + 1))}
+    elif a.op == "twosided":
+        W, X, G = llama_layer(a.m, a.n, 2 * max(a.m, a.n), seed=1, device=dev)
+        HX0 = torch.empty(a.n, a.n, device=dev)
+        HG0 = torch.empty(a.m, a.m, device=dev)
+        kq.kronq_accumulate_factors(X, HX0, zero_first=True)
+        kq.kronq_accumulate_factors(G, HG0, zero_first=True)
+        W0 = W.float().contiguous()
+        ng = 1 if a.group == -1 else -(-a.n // a.group)
+        Wt, HX, HG = W0.clone(), HX0.clone(), HG0.clone()
+        codes = torch.empty(a.m, a.n, dtype=torch.uint8, device=dev)
+        sc = torch.empty(a.m, ng, device=dev)
+        zp = torch.empty(a.m, ng, device=dev)
+        info = torch.zeros(2, dtype=torch.int32, device=dev)
+        p = kq.QuantParams(bits=a.bits, group=a.group, asym=1, damp_rel=0.01, block=128, flags=0)
+        ws = kq.workspace(kq.kronq_quantize_two_sided_workspace_bytes(a.m, a.n, p), dev)
+        if a.u_given:
+            kq.kronq_quantize_two_sided(Wt, HX, HG, p, codes, sc, zp, info, ws=ws)
+            HX0, HG0 = HX.clone(), HG.clone()
+            p = kq.QuantParams(bits=a.bits, group=a.group, asym=1, damp_rel=0.01, block=128, flags=kq.U_GIVEN)
+
+        def run():
+            Wt.copy_(W0)
+            HX.copy_(HX0)
+            HG.copy_(HG0)
+            kq.kronq_quantize_two_sided(Wt, HX, HG, p, codes, sc, zp, info, ws=ws)
+        # the feedback as two triangular products, E U_X and U_G^T (E U_X)
+        units = {"weights": a.m * a.n, "flops": a.m * a.n * (a.m + a.n)}
     else:
         W, X, G = llama_layer(a.m, a.n, 2 * max(a.m, a.n), seed=1, device=dev)
         lp = LayerPass(a.m, a.n, bits=a.bits, group=a.group, device=dev)
@@ -124,6 +154,9 @@ def main(argv=None):
     ms = e0.elapsed_time(e1) / a.reps
     if a.op in ("decode", "biip_inverse"):
         units["gbs"] = units["bytes"] / (ms / 1e3) / 1e9
+    if a.op == "twosided":
+        units["info"] = info.tolist()
+        units["tflops"] = units["flops"] / (ms / 1e3) / 1e12
     if a.op == "kronfactors":
         units["info"] = int(info.item())
         units["tflops"] = units["flops_per_sweep"] * a.iters / (ms / 1e3) / 1e12

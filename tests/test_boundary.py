@@ -250,3 +250,27 @@ def test_act_order_validation():
     args[13] = 16
     assert _st(L.kronq_quantize_layer_act_order(*args)) == _lib.ERR_INVALID_ARG      # workspace
     assert L.kronq_quantize_act_order_workspace_bytes(8, 256, ctypes.byref(p)) > 256 * 256 * 4
+
+
+def test_two_sided_validation():
+    L = _lib.lib
+    p = _qp(bits=2)
+    need = L.kronq_quantize_two_sided_workspace_bytes(96, 300, ctypes.byref(p))
+    # two m x n float32 buffers (P = E U_X and the scaled errors) on top of
+    # the factorisation scratch
+    assert need >= 2 * 4 * 96 * 300
+    assert L.kronq_quantize_two_sided_workspace_bytes(0, 300, ctypes.byref(p)) == 0
+
+    def call(p, HG=FAKE, ws=need, m=96, n=300, E=None):
+        return _st(L.kronq_quantize_two_sided(FAKE, FAKE, HG, m, n, ctypes.byref(p), FAKE, FAKE, FAKE, E, FAKE,
+                                              FAKE, ws, None))
+
+    assert call(p, HG=None) == _lib.ERR_INVALID_ARG
+    assert call(p, ws=need - 1) == _lib.ERR_INVALID_ARG
+    assert call(p, m=0) == _lib.ERR_INVALID_ARG
+    assert call(p, m=(1 << 20) + 1, ws=1 << 62) == _lib.ERR_INVALID_ARG
+    for flags in (_lib.R_FORM, _lib.ORDERED_FP32, _lib.WRITE_E, 64):   # WRITE_E: E is NULL
+        assert call(_qp(bits=2, flags=flags)) == _lib.ERR_INVALID_ARG
+    assert call(_qp(bits=5)) == _lib.ERR_INVALID_ARG
+    assert call(_qp(group=96)) == _lib.ERR_INVALID_ARG
+    assert call(_qp(block=64)) == _lib.ERR_UNSUPPORTED

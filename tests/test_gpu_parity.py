@@ -424,7 +424,8 @@ def test_kfac_loss_diagnostic():
 
 
 # ------------------------------------------------------------------ packing
-@pytest.mark.parametrize("bits,m,n", [(4, 64, 4096), (2, 33, 1000), (4, 5, 13), (2, 1, 16)])
+@pytest.mark.parametrize("bits,m,n", [(4, 64, 4096), (2, 33, 1000), (4, 5, 13), (2, 1, 16), (2, 48, 4096),
+                                      (2, 7, 192), (4, 3, 96), (2, 3, 4160)])
 def test_pack_unpack_bit_exact(bits, m, n):
     rng = np.random.default_rng(n)
     codes = rng.integers(0, 2 ** bits, size=(m, n)).astype(np.uint8)
