@@ -328,6 +328,7 @@ kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64
   p1.rows = m; p1.L = n;
   p1.scale = d_in; p1.scale_mode = need_in ? 1 : 0;
   p1.rotate = use_in; p1.inverse = false; p1.sign_state = s_in; p1.cf = cfbuf;
+  p1.tmp = Wt; p1.ld_tmp = n;   // scratch for a row-wise pass + transpose (Wt is written by p2)
   if ((r = rowpass(p1, st)) != KRONQ_OK) return r;
   RowPass p2;
   p2.in = T; p2.ld_in = m;
@@ -335,14 +336,17 @@ kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64
   p2.rows = n; p2.L = m;
   p2.scale = d_out; p2.scale_mode = need_out ? 1 : 0;
   p2.rotate = use_out; p2.inverse = false; p2.sign_state = s_out; p2.cf = cfbuf;
+  p2.tmp = T; p2.ld_tmp = m;    // in place
   if ((r = rowpass(p2, st)) != KRONQ_OK) return r;
   // H~_X = V D_in^-1 H_X D_in^-1 V^T
   if (use_in) {
     RowPass h1;
     h1.in = HX; h1.ld_in = n; h1.out = T; h1.ld_out = n; h1.rows = n; h1.L = n;
     h1.scale = d_in; h1.scale_mode = need_in ? 2 : 0; h1.rotate = true; h1.sign_state = s_in; h1.cf = cfbuf;
+    h1.tmp = HX; h1.ld_tmp = n;   // in place
     if ((r = rowpass(h1, st)) != KRONQ_OK) return r;
     RowPass h2 = h1;
+    h2.tmp = nullptr;
     h2.in = T; h2.out = HX;
     h2.rowwise = true;   // V F H F V^T is symmetric: no transposed store
     if ((r = rowpass(h2, st)) != KRONQ_OK) return r;
@@ -352,8 +356,10 @@ kronq_status kronq_biip_forward(const void* W, kronq_dtype wdt, float* Wt, int64
     RowPass g1;
     g1.in = HG; g1.ld_in = m; g1.out = T; g1.ld_out = m; g1.rows = m; g1.L = m;
     g1.scale = d_out; g1.scale_mode = need_out ? 2 : 0; g1.rotate = true; g1.sign_state = s_out; g1.cf = cfbuf;
+    g1.tmp = HG; g1.ld_tmp = m;   // in place
     if ((r = rowpass(g1, st)) != KRONQ_OK) return r;
     RowPass g2 = g1;
+    g2.tmp = nullptr;
     g2.in = T; g2.out = HG;
     g2.rowwise = true;
     if ((r = rowpass(g2, st)) != KRONQ_OK) return r;

@@ -719,6 +719,237 @@ kronq_status launch_fast(const RowPass& p, cudaStream_t s) {
   return KRONQ_OK;
 }
 
+// ------------------------------------------------------------ register-resident rows of 7 x 4096
+// Forward rows of L = 28672 = 7 x 4096 (the Llama-3-70B MLP length), stored
+// by rows.  One CTA of 256 threads per SM.  A row passes through shared
+// memory only to arrive (one bulk copy; the CTA's next row is copied into the
+// second buffer while this one is transformed), for two exchanges, and to
+// leave (one bulk copy).  Thread (w, l) holds 16 values of the Hadamard index
+// a times the 7 values of the DCT index b in registers; the twelve bits of a
+// are transformed four at a time, always in registers:
+//   phase 1: a = 256 u + 32 w + l          (registers: bits 8-11)
+//            column factors, the DCT along b, radix 16
+//   phase 2: a = u + 16 l + 512 w          (bits 0-3), radix 16
+//   phase 3: a = (l & 15) + 16 u + 256 (l >> 4) + 512 w   (bits 4-7), radix 16
+// The exchanges use the layout 7 a + b + (a >> 4) (one word of padding per
+// 16 a), on which the phase-2 and phase-3 accesses of a warp hit 32 distinct
+// banks; the arriving and the departing row use 7 a + b.  Per element the
+// arithmetic is that of rowpass_kernel (column factor, DCT, unnormalised
+// butterflies, 1 / sqrt(P)); the butterflies over the bits of a run in
+// another order, which changes only rounding.
+constexpr int R7_THREADS = 256;
+constexpr int R7_K = 7;
+constexpr int R7_P = 4096;
+constexpr int R7_L = R7_K * R7_P;
+constexpr int R7_BUF = R7_L + R7_P / 16;                     // floats per buffer
+constexpr int R7_SMEM = 2 * R7_BUF * (int)sizeof(float) + 16;  // two buffers, two mbarriers
+
+struct Dct7 {
+  float c[R7_K * R7_K];   // orthonormal DCT-II, c[o * 7 + b]; a kernel parameter, read from the constant bank
+};
+
+__device__ __forceinline__ void radix16_regs(float (&x)[16][R7_K]) {
+#pragma unroll
+  for (int b = 0; b < R7_K; ++b)
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if ((u & h) == 0) {
+          const float s0 = x[u][b], s1 = x[u | h][b];
+          x[u][b] = s0 + s1;
+          x[u | h][b] = s0 - s1;
+        }
+}
+
+__device__ __forceinline__ int r7_pad(int a) { return 7 * a + (a >> 4); }
+
+template <bool BF16>
+__global__ void __launch_bounds__(R7_THREADS, 1) rowpass_r7_kernel(const void* in, int64_t ld_in, float* out,
+                                                                   int64_t ld_out, int64_t rows, const float* cf,
+                                                                   Dct7 C) {
+  extern __shared__ __align__(16) float sm[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * R7_BUF);
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const uint32_t bar0 = smem_u32(&bars[0]);
+  constexpr uint32_t esz = BF16 ? 2u : 4u;
+  constexpr uint32_t in_bytes = R7_L * esz;
+  constexpr uint32_t out_bytes = R7_L * 4u;
+  const char* inb = static_cast<const char*>(in);
+  if (tid == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  int64_t row = blockIdx.x;
+  // loads issued and not yet waited for, bit k for buffer k (thread 0 only)
+  uint32_t pending = 0;
+  if (tid == 0 && row < rows) {
+    mbar_arrive_expect_tx(bar0, in_bytes);
+    bulk_load(smem_u32(sm), inb + row * ld_in * esz, in_bytes, bar0);
+    pending = 1u;
+  }
+  for (int i = 0; row < rows; ++i, row += gridDim.x) {
+    const int b = i & 1;
+    float* buf = sm + b * R7_BUF;
+    const int64_t nrow = row + gridDim.x;
+    if (tid == 0 && nrow < rows) {
+      tma_store_wait_read();   // the row stored from the other buffer has been read out
+      mbar_arrive_expect_tx(bar0 + 8 * (b ^ 1), in_bytes);
+      bulk_load(smem_u32(sm + (b ^ 1) * R7_BUF), inb + nrow * ld_in * esz, in_bytes, bar0 + 8 * (b ^ 1));
+      pending |= 1u << (b ^ 1);
+    }
+    const bool arrived = mbar_wait(bar0 + 8 * b, (uint32_t)(i >> 1) & 1u);
+    if (tid == 0 && arrived) pending &= ~(1u << b);
+    if (!__syncthreads_and(arrived)) break;   // timed out (recorded): stop the whole CTA
+
+    // phase 1: the arrived row (7 a + b), column factors, DCT along b
+    float x[16][R7_K];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int a = 256 * u + 32 * w + l;
+      float v[R7_K];
+#pragma unroll
+      for (int bb = 0; bb < R7_K; ++bb) {
+        const int j = 7 * a + bb;
+        const float e = BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(buf)[j]) : buf[j];
+        v[bb] = e * __ldg(cf + j);
+      }
+#pragma unroll
+      for (int o = 0; o < R7_K; ++o) {
+        float acc = 0.f;
+#pragma unroll
+        for (int bb = 0; bb < R7_K; ++bb) acc = fmaf(C.c[o * R7_K + bb], v[bb], acc);
+        x[u][o] = acc;
+      }
+    }
+    radix16_regs(x);
+    __syncthreads();   // every thread has read the arrived row
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int pa = r7_pad(256 * u + 32 * w + l);
+#pragma unroll
+      for (int bb = 0; bb < R7_K; ++bb) buf[pa + bb] = x[u][bb];
+    }
+    __syncthreads();
+    // phase 2: bits 0-3 in registers (each thread writes back what it read)
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int pa = r7_pad(u + 16 * l + 512 * w);
+#pragma unroll
+      for (int bb = 0; bb < R7_K; ++bb) x[u][bb] = buf[pa + bb];
+    }
+    radix16_regs(x);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int pa = r7_pad(u + 16 * l + 512 * w);
+#pragma unroll
+      for (int bb = 0; bb < R7_K; ++bb) buf[pa + bb] = x[u][bb];
+    }
+    __syncthreads();
+    // phase 3: bits 4-7 in registers
+    const int a3 = (l & 15) + 256 * (l >> 4) + 512 * w;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int pa = r7_pad(a3 + 16 * u);
+#pragma unroll
+      for (int bb = 0; bb < R7_K; ++bb) x[u][bb] = buf[pa + bb];
+    }
+    radix16_regs(x);
+    __syncthreads();   // every phase-3 read is done: the row layout overwrites
+    const float nrm = 1.f / 64.f;   // 1 / sqrt(4096), exact
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int j = 7 * (a3 + 16 * u);
+#pragma unroll
+      for (int bb = 0; bb < R7_K; ++bb) buf[j + bb] = x[u][bb] * nrm;
+    }
+    fence_proxy_async_smem();   // the row's writes, before the bulk copy reads them
+    __syncthreads();
+    if (tid == 0) {
+      bulk_store(out + row * ld_out, smem_u32(buf), out_bytes);
+      tma_store_commit();
+    }
+  }
+  if (tid == 0) {
+    // a load left in flight only after a timeout: wait for it (bounded)
+    for (int k = 0; k < 2; ++k)
+      if (pending & (1u << k)) (void)mbar_wait(bar0 + 8 * k, 0u);
+    tma_store_wait_all();
+  }
+}
+
+// out[j * ldo + r] = in[r * ldi + j] for r < rows, j < cols: 64 x 64 tiles.
+__global__ void __launch_bounds__(256) transpose_f32_kernel(const float* in, int64_t ldi, float* out, int64_t ldo,
+                                                            int64_t rows, int64_t cols) {
+  __shared__ float t[64][65];
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int64_t r = r0 + ty + 4 * k, c = c0 + tx;
+    if (r < rows && c < cols) t[ty + 4 * k][tx] = in[r * ldi + c];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int64_t j = c0 + ty + 4 * k, r = r0 + tx;
+    if (j < cols && r < rows) out[j * ldo + r] = t[tx][ty + 4 * k];
+  }
+}
+
+// The register-resident pass for rows of 28672 when its operands allow the
+// bulk copies; a transposed pass runs as a row-wise pass into p.tmp and a
+// transpose.  Returns false when it does not apply.
+#define KQ_LAUNCH_CHECK_R(r, name)                       \
+  do {                                                   \
+    ::kq::count_launch();                                \
+    cudaError_t e__ = cudaGetLastError();                \
+    if (e__ != cudaSuccess) {                            \
+      (r) = ::kq::cuda_fail(e__, name);                  \
+      return true;                                       \
+    }                                                    \
+  } while (0)
+
+bool try_r7(const RowPass& p, cudaStream_t s, kronq_status& r) {
+  if (!(p.L == R7_L && p.rotate && !p.inverse && p.cf && p.rows > 0)) return false;
+  const size_t esz = p.in_bf16 ? 2 : 4;
+  float* dst = p.rowwise ? p.out : p.tmp;
+  const int64_t ldd = p.rowwise ? p.ld_out : p.ld_tmp;
+  if (!dst || !aligned(p.in, 16) || (p.ld_in * esz) % 16 != 0 || !aligned(dst, 16) || (ldd * 4) % 16 != 0)
+    return false;
+  if (!p.rowwise && p.in_bf16 && static_cast<const void*>(dst) == p.in) return false;
+  colfactor_kernel<<<(unsigned)ceil_div(R7_L, 256), 256, 0, s>>>(p, p.cf);
+  KQ_LAUNCH_CHECK_R(r, "colfactor_kernel");
+  Dct7 C;
+  for (int o = 0; o < R7_K; ++o)
+    for (int b = 0; b < R7_K; ++b) {
+      const double co = (o == 0) ? sqrt(0.5) : 1.0;
+      C.c[o * R7_K + b] = (float)(sqrt(2.0 / R7_K) * co * cos(acos(-1.0) * (double)((2 * b + 1) * o) / (2.0 * R7_K)));
+    }
+  const void* fn = p.in_bf16 ? reinterpret_cast<const void*>(&rowpass_r7_kernel<true>)
+                             : reinterpret_cast<const void*>(&rowpass_r7_kernel<false>);
+  cudaError_t e = allow_smem(fn, R7_SMEM);
+  if (e != cudaSuccess) {
+    r = cuda_fail(e, "cudaFuncSetAttribute(rowpass_r7)");
+    return true;
+  }
+  const int64_t grid = p.rows < (int64_t)sm_count() ? p.rows : (int64_t)sm_count();
+  if (p.in_bf16)
+    rowpass_r7_kernel<true><<<(unsigned)grid, R7_THREADS, R7_SMEM, s>>>(p.in, p.ld_in, dst, ldd, p.rows, p.cf, C);
+  else
+    rowpass_r7_kernel<false><<<(unsigned)grid, R7_THREADS, R7_SMEM, s>>>(p.in, p.ld_in, dst, ldd, p.rows, p.cf, C);
+  KQ_LAUNCH_CHECK_R(r, "rowpass_r7_kernel");
+  if (!p.rowwise) {
+    dim3 g((unsigned)ceil_div(R7_L, 64), (unsigned)ceil_div(p.rows, 64));
+    transpose_f32_kernel<<<g, 256, 0, s>>>(dst, ldd, p.out, p.ld_out, p.rows, R7_L);
+    KQ_LAUNCH_CHECK_R(r, "transpose_f32_kernel");
+  }
+  r = KRONQ_OK;
+  return true;
+}
+
 // The compile-time variants: (odd factor, log2 of the power of two, rows
 // per group).  Returns false when the length has none.
 template <bool BF16>
@@ -840,6 +1071,7 @@ kronq_status rowpass(const RowPass& p, cudaStream_t s) {
   while ((1 << A.logR) < R) ++A.logR;
   if (p.rotate) {
     kronq_status r = KRONQ_OK;
+    if (try_r7(p, s, r)) return r;
     if (p.in_bf16 ? try_fast<true>(p, s, r) : try_fast<false>(p, s, r)) return r;
   }
   const bool f4096 = (p.L == 4096 && K == 1);

@@ -108,6 +108,11 @@ struct RowPass {
   // true: stored as rows (out[row * ld_out + j]), for a result that is
   // symmetric anyway (the second pass of V F H F V^T)
   bool rowwise = false;
+  // optional scratch of rows x L floats (row stride ld_tmp; it may be `in`
+  // itself when that is float32 and may be overwritten): a transposed pass
+  // may then run as a row-wise pass into it followed by a transpose
+  float* tmp = nullptr;
+  int64_t ld_tmp = 0;
 };
 kronq_status rowpass(const RowPass& p, cudaStream_t s);
 // sum of squares along columns (colsq[n]) and rows (rowsq[m]) of W.
