@@ -358,12 +358,14 @@ def _time_steps(layers, chunk, steps, warmup, stream, flush, sampler=None, barri
             if r:
                 r[4].record(stream)
 
-    for _ in range(warmup):
+    for w in range(warmup):
         flush.zero_()
         step()
-    torch.cuda.synchronize()
-    for _, _, _, _, lp in layers:
-        assert int(lp.info.item()) == 0, "factorisation reported a non-positive pivot"
+        torch.cuda.synchronize()
+        for name, _, _, _, lp in layers:
+            info = int(lp.info.item())
+            assert info == 0, (f"factorisation of {name} reported a non-positive pivot (info {info}) in "
+                               f"warm-up step {w}; device status {kq.kronq_device_status()}")
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     recs = [[[ev() for _ in range(5)] for _ in layers] for _ in range(steps)]
     if sampler:
