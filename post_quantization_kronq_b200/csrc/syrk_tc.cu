@@ -317,6 +317,8 @@ constexpr int P_NBARS = 2 * P_STAGES + 5;           // full, empty, accfull[2], 
 constexpr int P_SMEM = P_STAGES * P_STAGE + 1024 + 256;
 constexpr uint32_t P_TMEM = 2 * PN;
 constexpr int P_STRIP = 8;                          // tile rows (of 256) per raster strip
+constexpr int64_t kSyrkSplitMinD = 16384;
+constexpr int64_t kSyrkSplitT = 8192;
 
 struct SyrkPairArgs {
   float* H;
@@ -598,6 +600,20 @@ cudaError_t status_fetch_syrk(int* out, cudaStream_t s) {
 
 kronq_status syrk_bf16_tc(const void* A, int64_t T, int64_t d, int64_t lda, float* H,
                           bool zero_first, cudaStream_t s) {
+  // From d = 16384 on, the tokens go in launches of at most 8192: the 256
+  // token columns of the ~18 tile rows and columns that a wave of 74 SM
+  // pairs touches then take ~72 MB and stay in L2 while the wave runs (at
+  // 16384 tokens, ~144 MB do not, and the chunk is read from DRAM ~35
+  // times), for one more read-modify-write of H per 8192 tokens.
+  if (d >= kSyrkSplitMinD && T > kSyrkSplitT) {
+    for (int64_t t0 = 0; t0 < T; t0 += kSyrkSplitT) {
+      const int64_t tn = (T - t0) < kSyrkSplitT ? (T - t0) : kSyrkSplitT;
+      kronq_status r = syrk_bf16_tc(static_cast<const __nv_bfloat16*>(A) + t0 * lda, tn, d, lda, H,
+                                    zero_first && t0 == 0, s);
+      if (r != KRONQ_OK) return r;
+    }
+    return KRONQ_OK;
+  }
   auto encode = tma_encode_fn();
   if (!encode) return fail(KRONQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   CUtensorMap map;
