@@ -63,12 +63,23 @@ WORKLOADS = {
 }
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one factor-accumulation
-# launch (syrk_pair_kernel, ncu on a B200, one capture each), keyed by
-# (d, tokens per launch); shapes not captured give traffic null.
+# launch (syrk_pair_kernel, ncu on a B200), keyed by (d, tokens per
+# launch); shapes not captured give traffic null.  (28672, 8192): the mean
+# of the two launches of a 16384-token chunk.
 SYRK_TRAFFIC = {
-    (28672, 16384): 32839476992 + 3274788864,
+    (28672, 8192): (6687214336 + 3252186624 + 9249690880 + 3250075648) // 2,
     (8192, 16384): 1161290496 + 251058688,
 }
+# The library's launch rule for the factor accumulation: from d = 16384 on,
+# a call's tokens go in launches of at most 8192.
+SYRK_SPLIT_MIN_D, SYRK_SPLIT_T = 16384, 8192
+
+
+def syrk_launches(d: int, tokens: int):
+    """(launches, tokens per launch) of one accumulation call."""
+    if d >= SYRK_SPLIT_MIN_D and tokens > SYRK_SPLIT_T:
+        return -(-tokens // SYRK_SPLIT_T), SYRK_SPLIT_T
+    return 1, tokens
 
 
 def _peaks():
@@ -498,20 +509,23 @@ def run_kronq(args):
     peaks = _peaks()
     tpk, hpk, src = choose_peak(peaks, clocks)
     # Roofline of the dominant kernel: the tcgen05 SYRK.  The accumulation
-    # phase is SYRK launches only (two factors per layer, one launch per
-    # token chunk); algorithmic flops T d (d + 1) per factor.
+    # phase is SYRK launches only (two factors per layer, one call per token
+    # chunk, split into launches by the library's rule); algorithmic flops
+    # T d (d + 1) per factor.
     acc_ms = phases["accumulate_HX_HG"]
     flops = sum(T * n * (n + 1) + T * m * (m + 1) for m, n in shapes)
-    per_layer_launches = 2 * (1 if chunk is None else -(-T // chunk))
-    nl = per_layer_launches * len(shapes)
-    achieved = flops / (acc_ms / 1e3) / 1e12
-    traffic = None
-    tkeys = []
+    calls = 1 if chunk is None else -(-T // chunk)
+    per_call = T if chunk is None else chunk
+    shapes_l = []   # (d, tokens per launch, launches per step)
     for m, n in shapes:
         for d in (n, m):
-            tkeys.append((d, T if chunk is None else chunk))
-    if all(k in SYRK_TRAFFIC for k in tkeys):
-        traffic = sum(SYRK_TRAFFIC[k] for k in tkeys) / len(tkeys)
+            k, tl = syrk_launches(d, per_call)
+            shapes_l.append((d, tl, k * calls))
+    nl = sum(c for _, _, c in shapes_l)
+    achieved = flops / (acc_ms / 1e3) / 1e12
+    traffic = None
+    if all((d, tl) in SYRK_TRAFFIC for d, tl, _ in shapes_l):
+        traffic = sum(SYRK_TRAFFIC[(d, tl)] * c for d, tl, c in shapes_l) / nl
     kname = "syrk_pair_kernel" if min(min(m, n) for m, n in shapes) >= 2048 else "syrk_bf16_tc_kernel"
     roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": tpk,
                 "unit": "TFLOP/s", "frac": achieved / tpk, "traffic": traffic,

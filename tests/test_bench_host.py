@@ -51,3 +51,12 @@ def test_workloads_name_the_configured_shapes():
     assert [(m, n) for _, m, n, _ in wl["layers"]] == [(28672, 8192), (8192, 28672)]
     q = bench.WORKLOADS["llama2_7b_q_proj"]
     assert q["tokens"] == 131072 and [(m, n) for _, m, n, _ in q["layers"]] == [(4096, 4096)]
+
+
+def test_syrk_launch_rule():
+    # d >= 16384: a 16384-token call is two 8192-token launches; smaller d one launch
+    assert bench.syrk_launches(28672, 16384) == (2, 8192)
+    assert bench.syrk_launches(28672, 8192) == (1, 8192)
+    assert bench.syrk_launches(28672, 20000) == (3, 8192)
+    assert bench.syrk_launches(8192, 16384) == (1, 16384)
+    assert bench.syrk_launches(14336, 65536) == (1, 65536)
