@@ -484,8 +484,6 @@ __global__ void __launch_bounds__(T_THREADS, 1)
         const int k = warp + 8 * t, nn = 4 * lane;
         bv[t] = *reinterpret_cast<const float4*>(F + TF_A + (nn >> 5) * TF_BBOX + sw128_f32(k, nn & 31));
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(fempty(fs));
       if (bu > 0 && !mbar_wait(bempty(bs), (bu - 1) & 1)) { ok = false; break; }
       uint8_t* Sb = bst + bs * TS_STAGE;
 #pragma unroll
@@ -513,9 +511,17 @@ __global__ void __launch_bounds__(T_THREADS, 1)
         if (!(kin && col + 3 < g.N && (!g.b_upper || k <= col + 3))) v.w = 0.f;
         split_store4(Sb + 3 * TS_SPLIT, mn_off(nn, kl), TS_SPLIT, v);
       }
+      // The fp32 stage is released only now: its values were consumed by the
+      // splits above, and the fence orders these generic reads before the
+      // TMA (async-proxy) write of the chunk that refills the stage.  An
+      // arrive right after the loads let that write overtake loads still in
+      // flight, so that a few percent of calls used a later chunk's values.
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bfull(bs));
+      if (lane == 0) {
+        mbar_arrive(fempty(fs));
+        mbar_arrive(bfull(bs));
+      }
       // the last chunk of segment sg is converted: the segment before it is
       // (or soon will be) complete in its accumulator
       const int sg = s / T_SEG;
@@ -669,14 +675,7 @@ kronq_status trigemm_tc(const TriGemm& t, cudaStream_t s) {
     dy = (int)(stride / ld);
     return (x0 % 4) == 0 && (dx % 4) == 0 && stride >= 0;
   };
-  // The TMA-fed kernel is not dispatched: repeated calls on identical inputs
-  // returned results that differ from run to run (a few percent of the
-  // recursive-inverse calls at n = 4096, ~1e-4 relative in single output
-  // tile columns; every second two-level factorisation at n = 28672), while
-  // the kernel below, fed by plain loads, returned identical results in
-  // every run.  The cause inside trigemm_tma_kernel is not known yet.
-  constexpr bool kTmaFed = false;
-  bool use_tma = kTmaFed && t.holdA && t.holdB && (t.lda % 4) == 0 && (t.ldb % 4) == 0 &&
+  bool use_tma = t.holdA && t.holdB && (t.lda % 4) == 0 && (t.ldb % 4) == 0 &&
                  aligned(t.holdA, 16) && aligned(t.holdB, 16) &&
                  origin(t.holdA, t.lda, t.A, t.batch > 1 ? t.strideA : 0, tt.ax0, tt.ay0, tt.adx, tt.ady) &&
                  origin(t.holdB, t.ldb, t.B, t.batch > 1 ? t.strideB : 0, tt.bx0, tt.by0, tt.bdx, tt.bdy);
