@@ -305,7 +305,8 @@ kronq_status kronq_quantize_layer_act_order(float* Wt, float* HX, int64_t m, int
  *     rule of kronq_quantize_layer; a grid taken at a group start would
  *     depend on the processing order);
  *   - element (i, j): q = clamp(rint(w~ / scale) + zero, 0, 2^b - 1),
- *     e_ij = (w~_ij - deq) / (U_X[j, j] U_G[i, i]), and
+ *     e_ij = (w~_ij - deq) / (U_X[j, j] U_G[i, i]) (in float32, the
+ *     divisions as products with the float32 reciprocals), and
  *     w~_i'j' -= e_ij U_G[i, i'] U_X[j, j'] for every later (i' >= i,
  *     j' >= j) element.  Every order that respects that partial order gives
  *     the same result; the library runs 32 x 128 tiles along anti-diagonals.
