@@ -22,6 +22,8 @@
  *                                                    -> kronq_kron_factors
  *   - the deploy path's matvec from packed codes (KronQ README intro: fused
  *     dequant + BiIP matvec for single-token decode) -> kronq_decode_matvec
+ *   - two-sided rounding that uses H_G inside the sweep ("BaKron" abstract:
+ *     GPTQ on vec(W) under H_X (x) H_G)            -> kronq_quantize_two_sided
  *
  * Conventions (all calls):
  *   - Matrices are row-major.  W is m x n (out x in), X is T x n, G is T x m.
